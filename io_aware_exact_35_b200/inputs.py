@@ -1,0 +1,132 @@
+"""Seeded synthetic inputs shared by the tests, the benchmark and the oracle checks.
+
+This module draws random numbers and rounds them to bf16; it holds none of the
+attention arithmetic.  Every draw uses a CPU ``torch.Generator`` seeded
+explicitly, so both the CUDA path and the fp64 oracle see bit-identical inputs.
+
+Recipe (the pages' seed 42 is the base; each workload adds its index):
+
+* forward:  q, k, v ~ iid N(0,1) * std, drawn in that order as float32, then
+  rounded to bf16 (round-to-nearest-even);
+* backward: q, k, v, dO drawn in that order the same way;
+* decode:   seqlens ~ U{Lmin .. Lmax} (both ends inclusive) first, then
+  q ~ N(0,1) [B, H, d], then for each sequence b in order: K_b, V_b ~ N(0,1)
+  of shape [H, L_b, d].  Cache rows at or beyond L_b hold NaN so that any
+  read past the prefix shows up in the outputs.
+"""
+
+from __future__ import annotations
+
+from dataclasses import dataclass, field
+
+import numpy as np
+import torch
+
+BASE_SEED = 42
+
+
+@dataclass(frozen=True)
+class Workload:
+    name: str
+    kind: str            # "fwd" | "bwd" | "decode"
+    B: int
+    H: int
+    d: int
+    N: int = 0           # sequence length (fwd / bwd)
+    causal: bool = False
+    std: float = 1.0
+    Lmin: int = 0        # decode: cache length range, inclusive
+    Lmax: int = 0
+    seed: int = BASE_SEED
+
+    @property
+    def scale(self) -> float:
+        return 1.0 / float(np.sqrt(self.d))
+
+
+# The five workloads: the shapes of a 2K-context prefill layer, a 32K
+# long-context prefill, an 8K causal backward and a batched KV-cache decode,
+# plus a small non-causal case that the oracle finishes instantly.
+WORKLOADS = {
+    w.name: w for w in (
+        Workload("fwd_noncausal_B1_H2_N256_d64", "fwd", 1, 2, 64, N=256,
+                 causal=False, seed=BASE_SEED + 0),
+        Workload("fwd_causal_B4_H16_N2048_d128", "fwd", 4, 16, 128, N=2048,
+                 causal=True, seed=BASE_SEED + 1),
+        Workload("fwd_causal_B1_H32_N32768_d128", "fwd", 1, 32, 128, N=32768,
+                 causal=True, std=0.5, seed=BASE_SEED + 2),
+        Workload("bwd_causal_B2_H16_N8192_d128", "bwd", 2, 16, 128, N=8192,
+                 causal=True, seed=BASE_SEED + 3),
+        Workload("decode_B16_H32_d128_L4096-16384", "decode", 16, 32, 128,
+                 Lmin=4096, Lmax=16384, seed=BASE_SEED + 4),
+    )
+}
+
+
+def _gen(seed: int) -> torch.Generator:
+    return torch.Generator(device="cpu").manual_seed(int(seed))
+
+
+def _randn_bf16(g: torch.Generator, shape, std: float = 1.0) -> torch.Tensor:
+    x = torch.randn(shape, generator=g, dtype=torch.float32)
+    if std != 1.0:
+        x.mul_(std)
+    return x.to(torch.bfloat16)
+
+
+def fwd_inputs(B: int, H: int, N: int, d: int, seed: int, std: float = 1.0):
+    """q, k, v as contiguous bf16 CPU tensors [B, H, N, d]."""
+    g = _gen(seed)
+    return tuple(_randn_bf16(g, (B, H, N, d), std) for _ in range(3))
+
+
+def bwd_inputs(B: int, H: int, N: int, d: int, seed: int, std: float = 1.0):
+    """q, k, v, dO as contiguous bf16 CPU tensors [B, H, N, d]."""
+    g = _gen(seed)
+    return tuple(_randn_bf16(g, (B, H, N, d), std) for _ in range(4))
+
+
+def decode_inputs(B: int, H: int, d: int, Lmin: int, Lmax: int, seed: int,
+                  Lcap: int | None = None, seqlens=None, poison: bool = True):
+    """q [B,H,d], kcache/vcache [B,H,Lcap,d] bf16, seqlens int32 [B].
+
+    ``seqlens`` may be given explicitly (edge-case tests); otherwise it is
+    drawn first from the generator.  ``Lcap`` (the cache capacity) defaults
+    to Lmax.
+    """
+    g = _gen(seed)
+    if seqlens is None:
+        seqlens = torch.randint(Lmin, Lmax + 1, (B,), generator=g, dtype=torch.int64)
+    seqlens = torch.as_tensor(seqlens, dtype=torch.int64)
+    Lcap = int(Lcap if Lcap is not None else max(Lmax, int(seqlens.max().item()) if B else 0))
+    q = _randn_bf16(g, (B, H, d))
+    fill = float("nan") if poison else 0.0
+    kc = torch.full((B, H, Lcap, d), fill, dtype=torch.bfloat16)
+    vc = torch.full((B, H, Lcap, d), fill, dtype=torch.bfloat16)
+    for b in range(B):
+        L = int(seqlens[b])
+        kc[b, :, :L] = _randn_bf16(g, (H, L, d))
+        vc[b, :, :L] = _randn_bf16(g, (H, L, d))
+    return q, kc, vc, seqlens.to(torch.int32)
+
+
+def workload_inputs(w: Workload):
+    if w.kind == "fwd":
+        return fwd_inputs(w.B, w.H, w.N, w.d, w.seed, w.std)
+    if w.kind == "bwd":
+        return bwd_inputs(w.B, w.H, w.N, w.d, w.seed, w.std)
+    return decode_inputs(w.B, w.H, w.d, w.Lmin, w.Lmax, w.seed)
+
+
+def sample_rows(N: int, n_random: int, seed: int, edge: int = 128) -> np.ndarray:
+    """Sorted row indices: the first and last ``edge`` rows plus random ones."""
+    rng = np.random.default_rng(seed)
+    head = np.arange(min(edge, N))
+    tail = np.arange(max(0, N - edge), N)
+    mid = rng.integers(0, N, size=n_random) if N else np.zeros(0, np.int64)
+    return np.unique(np.concatenate([head, tail, mid]))
+
+
+def to_f64(t: torch.Tensor) -> np.ndarray:
+    """Exact conversion of a (bf16 / fp32) tensor to a float64 numpy array."""
+    return t.detach().to("cpu").to(torch.float64).numpy()
