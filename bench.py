@@ -1,0 +1,443 @@
+#!/usr/bin/env python
+"""Benchmark of the exact-attention hot path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+One step is one call of the library on one batch of synthetic input of the
+chosen workload (default: the causal 2K-context prefill, B=4 H=16 N=2048
+d=128).  The timed region is exactly K steps bracketed by a barrier and a
+device synchronisation; each launch is timed with CUDA events on the stream it
+runs on.  Rank 0 prints one JSON line.  Under torchrun every rank runs the
+same workload on its own GPU (independent (batch, head) partitions, weak
+scaling, no data-path collective) and the time is the maximum over ranks.
+
+``--impl reference`` times the fp64 CPU oracle (the deliberately slow
+definition) on the host cores, on a bounded sample of the same workload.
+"""
+
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from io_aware_exact_35_b200 import inputs  # noqa: E402
+
+METRIC = "bf16 attention TFLOP/s fwd & bwd; decode KV-read GB/s; % of roofline"
+DEFAULT_WORKLOAD = "fwd_causal_B4_H16_N2048_d128"
+L2_BYTES = 126 * 1024 * 1024
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+# ----------------------------------------------------------------------------- helpers
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def kernel_sources_sha():
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "io_aware_exact_35_b200", "csrc")
+    for name in sorted(os.listdir(csrc)):
+        with open(os.path.join(csrc, name), "rb") as f:
+            h.update(name.encode() + f.read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic(kernel_key):
+    """DRAM bytes per launch from the committed ncu summary, if still current."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        d = json.load(f)
+    ent = d.get(kernel_key)
+    if not ent or ent.get("source_sha") != kernel_sources_sha():
+        return None
+    return ent.get("dram_bytes_per_launch")
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle sampling during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.proc = None
+        self.lines = []
+        self.dev = device_index
+
+    def start(self):
+        cmd = ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+               "-lms", "100"]
+        try:
+            uuid = str(torch.cuda.get_device_properties(self.dev).uuid)
+            cmd += ["-i", uuid if uuid.startswith("GPU-") else "GPU-" + uuid]
+        except Exception:
+            pass
+        try:
+            self.proc = subprocess.Popen(cmd, stdout=subprocess.PIPE, stderr=subprocess.DEVNULL,
+                                         text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except (OSError, ValueError):
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.thread.join(timeout=2)
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax.append(float(parts[2]))
+            except ValueError:
+                continue
+            for nm, val in zip(names, parts[5:9]):
+                if val.lower() == "active":
+                    reasons.add(nm)
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(smax) if smax else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ----------------------------------------------------------------------------- workloads
+def fwd_flops(w):
+    f = 4.0 * w.B * w.H * w.N * w.N * w.d
+    return f * 0.5 if w.causal else f
+
+
+def decode_bytes(w, seqlens):
+    return float(sum(int(L) for L in seqlens)) * w.H * w.d * 2 * 2
+
+
+class Runner:
+    """Holds device buffers of one workload and launches one step on demand."""
+
+    def __init__(self, w, dev):
+        from io_aware_exact_35_b200 import fa
+        self.fa, self.w, self.dev = fa, w, dev
+        self.host = inputs.workload_inputs(w)
+        self.dbuf = [t.to(dev) for t in self.host]
+        if w.kind == "fwd":
+            q, k, v = self.dbuf
+            self.o = torch.empty_like(q)
+            self.lse = torch.empty(q.shape[:3], dtype=torch.float32, device=dev)
+            self.work = fwd_flops(w)
+            self.unit, self.kind_bound = "TFLOP/s", "tensor"
+            self.launches_per_step = 1
+            self.kernel_key = f"fa_fwd_kernel<{w.d},{str(w.causal).lower()}>"
+            self.out_host = torch.empty(self.o.shape, dtype=torch.bfloat16).pin_memory()
+        elif w.kind == "bwd":
+            q, k, v, do = self.dbuf
+            self.o, self.lse = fa.fwd(q, k, v, causal=w.causal, scale=w.scale)
+            self.dq, self.dk, self.dv = (torch.empty_like(q) for _ in range(3))
+            self.ws = torch.empty(fa.bwd_workspace_size(w.B, w.H, w.N, w.d), dtype=torch.uint8,
+                                  device=dev)
+            self.work = 2.5 * fwd_flops(w)
+            self.unit, self.kind_bound = "TFLOP/s", "tensor"
+            self.launches_per_step = 3
+            self.kernel_key = f"fa_bwd_kernel<{w.d},{str(w.causal).lower()}>"
+            self.out_host = torch.empty(self.dq.shape, dtype=torch.bfloat16).pin_memory()
+        else:
+            q, kc, vc, sl = self.dbuf
+            self.o = torch.empty_like(q)
+            self.lse = torch.empty(q.shape[:2], dtype=torch.float32, device=dev)
+            self.ws = torch.empty(fa.decode_workspace_size(w.B, w.H, kc.shape[2], w.d),
+                                  dtype=torch.uint8, device=dev)
+            self.work = decode_bytes(w, self.host[3].tolist())
+            self.unit, self.kind_bound = "GB/s", "hbm"
+            self.launches_per_step = 2
+            self.kernel_key = f"fa_decode_split_kernel<{w.d}>"
+            self.out_host = torch.empty(self.o.shape, dtype=torch.bfloat16).pin_memory()
+        self.working_set = sum(t.numel() * t.element_size() for t in self.dbuf)
+        self.flush = None
+        if self.working_set < 2 * L2_BYTES:
+            self.flush = torch.empty(2 * L2_BYTES, dtype=torch.uint8, device=dev)
+
+    def step(self, bufs=None):
+        w, fa = self.w, self.fa
+        b = bufs if bufs is not None else self.dbuf
+        if w.kind == "fwd":
+            fa.fwd(b[0], b[1], b[2], causal=w.causal, scale=w.scale, out=self.o, lse=self.lse)
+            return self.o
+        if w.kind == "bwd":
+            fa.bwd(b[0], b[1], b[2], self.o, b[3], self.lse, causal=w.causal, scale=w.scale,
+                   dq=self.dq, dk=self.dk, dv=self.dv, workspace=self.ws)
+            return self.dq
+        fa.decode(b[0], b[1], b[2], b[3], scale=w.scale, out=self.o, lse=self.lse,
+                  workspace=self.ws)
+        return self.o
+
+    def value(self, seconds):
+        return self.work / seconds / 1e12 if self.unit == "TFLOP/s" else self.work / seconds / 1e9
+
+
+def barrier(world):
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+
+
+def max_over_ranks(x, world, dev):
+    if world == 1:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def time_device(r, steps, warmup, world, dev):
+    """Kernel-only timing: inputs resident in HBM; events around each step."""
+    stream = torch.cuda.current_stream()
+    for _ in range(warmup):
+        if r.flush is not None:
+            r.flush.zero_()
+        r.step()
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    sampler = ClockSampler(dev.index or 0)
+    sampler.start()
+    time.sleep(0.3)
+    barrier(world)
+    t0 = time.perf_counter()
+    for i in range(steps):
+        if r.flush is not None:
+            r.flush.zero_()
+        starts[i].record(stream)
+        r.step()
+        ends[i].record(stream)
+    barrier(world)
+    wall = time.perf_counter() - t0
+    clocks = sampler.stop()
+    per = [s.elapsed_time(e) * 1e-3 for s, e in zip(starts, ends)]
+    mean_s = max_over_ranks(float(np.mean(per)), world, dev)
+    return mean_s, per, wall, clocks
+
+
+def time_e2e(r, steps, warmup, world, dev):
+    """End-to-end through the public API: pinned host -> device, the call, and
+    the result back to the host, every step."""
+    host = [t.pin_memory() for t in r.host]
+    dbufs = [torch.empty_like(t, device=dev) for t in r.host]
+    h2d = sum(t.numel() * t.element_size() for t in host)
+    d2h = r.out_host.numel() * r.out_host.element_size()
+
+    def one():
+        for hb, db in zip(host, dbufs):
+            db.copy_(hb, non_blocking=True)
+        out = r.step(dbufs)
+        r.out_host.copy_(out, non_blocking=True)
+
+    for _ in range(max(1, warmup)):
+        one()
+    barrier(world)
+    st, en = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    st.record()
+    for _ in range(steps):
+        one()
+    en.record()
+    barrier(world)
+    sec = max_over_ranks(st.elapsed_time(en) * 1e-3 / steps, world, dev)
+    return sec, h2d, d2h
+
+
+# ----------------------------------------------------------------------------- reference arm
+def run_reference(args, w, total_budget=150.0, emit=True):
+    """The fp64 CPU oracle as it stands, on a bounded sample of the workload."""
+    import oracle
+    try:
+        from threadpoolctl import threadpool_info
+        cores = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
+    except Exception:
+        cores = os.cpu_count() or 1
+    host = inputs.workload_inputs(w)
+    f64 = inputs.to_f64
+    budget = total_budget / max(1, args.steps + args.warmup)  # seconds per step
+    rng = np.random.default_rng(w.seed)
+    if w.kind in ("fwd", "bwd"):
+        q, k, v = (t for t in host[:3])
+        heads = [(b, h) for b in range(w.B) for h in range(w.H)]
+        # rows per step sized from a probe so that a step stays within budget
+        b0, h0 = heads[0]
+        qh, kh, vh = f64(q[b0, h0]), f64(k[b0, h0]), f64(v[b0, h0])
+        t0 = time.perf_counter()
+        oracle.attention_forward_rows(qh, kh, vh, w.causal, w.scale, np.arange(min(64, w.N)))
+        per_row = (time.perf_counter() - t0) / min(64, w.N)
+        rows_per_step = int(max(1, min(w.N, budget / max(per_row, 1e-9))))
+        sample = f"{rows_per_step} query rows of one (batch, head) per step, rows drawn uniformly"
+        mult = 3.5 if w.kind == "bwd" else 1.0  # bwd oracle is not timed; fwd rows scaled
+
+        def step(i):
+            b, h = heads[i % len(heads)]
+            rows = np.sort(rng.integers(0, w.N, rows_per_step))
+            qh, kh, vh = f64(q[b, h]), f64(k[b, h]), f64(v[b, h])
+            t = time.perf_counter()
+            oracle.attention_forward_rows(qh, kh, vh, w.causal, w.scale, rows)
+            dt = time.perf_counter() - t
+            keys = (rows + 1).sum() if w.causal else rows.size * w.N
+            return dt, 4.0 * keys * w.d * (2.5 if w.kind == "bwd" else 1.0), mult
+        unit = "TFLOP/s"
+        scale_out = 1e12
+    else:
+        q, kc, vc, sl = host
+        sample = "one (batch, head) cache prefix per step"
+
+        def step(i):
+            b = i % w.B
+            h = (i // w.B) % w.H
+            L = int(sl[b])
+            qq, kk, vv = f64(q[b:b + 1, h:h + 1]), f64(kc[b:b + 1, h:h + 1, :L]), f64(vc[b:b + 1, h:h + 1, :L])
+            t = time.perf_counter()
+            oracle.decode_forward(qq, kk, vv, [L], w.scale)
+            return time.perf_counter() - t, float(L) * w.d * 4, 1.0
+        unit = "GB/s"
+        scale_out = 1e9
+    for i in range(args.warmup):
+        step(i)
+    tot_t, tot_w = 0.0, 0.0
+    for i in range(args.steps):
+        dt, work, mult = step(args.warmup + i)
+        tot_t += dt * mult
+        tot_w += work
+    value = tot_w / tot_t / scale_out
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": unit, "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": tot_t / args.steps * 1e3, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": w.name, "parallelism": "cpu"},
+        "cpu_baseline": {"value": value, "unit": unit, "cores": cores, "kind": "oracle",
+                         "sample": sample + (" (bwd: forward-row oracle time x3.5)" if w.kind == "bwd" else "")},
+        "e2e": {"value": value, "unit": unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    if emit:
+        print(json.dumps(line), flush=True)
+    return line
+
+
+def cpu_baseline(w, seconds=15.0):
+    """Oracle timing on the host cores for the JSON line (bounded sample)."""
+    ns = argparse.Namespace(steps=6, warmup=1, gpus=1)
+    return run_reference(ns, w, total_budget=seconds, emit=False)["cpu_baseline"]
+
+
+# ----------------------------------------------------------------------------- main
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=None)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(inputs.WORKLOADS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-extra", action="store_true", help="skip the other workloads' lines")
+    args = ap.parse_args()
+    w = inputs.WORKLOADS[args.workload]
+    default_steps = {"fwd": 4000, "bwd": 300, "decode": 800}[w.kind]
+    if w.name == "fwd_causal_B1_H32_N32768_d128":
+        default_steps = 200
+    if args.steps is None:
+        args.steps = default_steps
+    args.warmup = max(3, args.warmup)
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if args.impl == "reference":
+        if rank == 0:
+            run_reference(args, w)
+        return
+
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        from datetime import timedelta
+        torch.distributed.init_process_group("nccl", timeout=timedelta(seconds=120),
+                                             device_id=dev)
+    from io_aware_exact_35_b200 import fa
+    fa.lib()
+
+    r = Runner(w, dev)
+    mean_s, per, wall, clocks = time_device(r, args.steps, args.warmup, world, dev)
+    e2e_s, h2d, d2h = time_e2e(r, max(3, min(args.steps, 50)), 2, world, dev)
+    err = fa.get_device_error()
+    peaks, peak_src = load_peaks()
+    value = r.value(mean_s) * world
+    if r.kind_bound == "tensor":
+        peak = float(peaks["bf16_tflops"])
+        ach = r.work / mean_s / 1e12
+        traffic = profiled_traffic(r.kernel_key)
+        roof = {"bound": "tensor", "achieved": ach, "peak": peak, "unit": "TFLOP/s",
+                "frac": ach / peak, "traffic": traffic,
+                "peak_source": f"{peak_src} bf16_tflops (burst)"}
+    else:
+        peak = float(peaks["hbm_gbs"])
+        ach = r.work / mean_s / 1e9
+        traffic = profiled_traffic(r.kernel_key)
+        roof = {"bound": "hbm", "achieved": ach, "peak": peak, "unit": "GB/s",
+                "frac": ach / peak, "traffic": traffic,
+                "peak_source": f"{peak_src} hbm_gbs"}
+    line = {
+        "metric": METRIC, "value": value, "unit": r.unit, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": mean_s * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": w.name, "B": w.B, "H": w.H, "N": w.N or None, "d": w.d,
+                   "causal": w.causal, "parallelism": f"replicas{world}" if world > 1 else "single",
+                   "l2": "flushed (256 MB write) before every step" if r.flush is not None
+                   else "inputs larger than L2"},
+        "roofline": roof,
+        "e2e": {"value": r.value(e2e_s) * world, "unit": r.unit, "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h},
+        "gpu_launches": args.steps * r.launches_per_step,
+        "clocks": clocks,
+        "device_error": err,
+        "wall_s_timed_region": wall,
+    }
+    if rank == 0 and world == 1:
+        try:
+            line["cpu_baseline"] = cpu_baseline(w)
+        except Exception as e:  # the baseline is reported, not required
+            line["cpu_baseline"] = {"value": None, "error": str(e)[:200]}
+    if world > 1:
+        torch.distributed.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+if __name__ == "__main__":
+    main()

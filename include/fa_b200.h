@@ -1,0 +1,148 @@
+/*
+ * fa_b200.h - C ABI of the B200 (sm_100a) exact-attention library libfa_b200.so.
+ *
+ * Exact scaled-dot-product attention O = softmax(scale * Q K^T [+ causal mask]) V,
+ * computed tile by tile with an online softmax so that the N x N score matrix
+ * never reaches device memory ("DL101 chapter 9", handsonai.io, section 3.3
+ * FlashAttention; "Flash Attention: principle & practice", holysheep.ai,
+ * sections 2.1 Online Softmax and 2.2 Tiling).
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ *  - Tensors are contiguous, row-major, in device memory, and 16-byte aligned.
+ *    "bf16" arguments are void pointers to IEEE bfloat16 bit patterns.
+ *  - Q, K, V, O, dO, dQ, dK, dV are [B, H, N, d] (batch, head, sequence, head
+ *    dimension; the multi-head layout of "DL101 chapter 9", section 3).
+ *    LSE and D are [B, H, N] float32.
+ *  - Supported head dimensions: d = 64 and d = 128.  Any N >= 0 (ragged tails
+ *    are masked inside the kernels).
+ *  - scale multiplies Q K^T before the softmax; callers normally pass
+ *    1/sqrt(d) ("DL101 chapter 9", section 1.1).
+ *  - Causal masking keeps key j for query i iff j <= i (square, top-left
+ *    aligned, diagonal included).
+ *  - LSE is the natural-log log-sum-exp of the row's scaled, masked scores:
+ *    LSE_i = ln sum_j exp(scale * q_i . k_j).
+ *  - The caller allocates and owns every buffer, workspaces included.  The
+ *    library allocates no device memory; it keeps only per-process state
+ *    (a driver entry point, device properties and a device error word).
+ *  - All calls are asynchronous and ordered on `stream` (a cudaStream_t; NULL
+ *    is the legacy default stream).  Argument errors are reported before any
+ *    launch and leave the outputs untouched.  A failed launch returns
+ *    FA_ERR_CUDA.  A kernel whose bounded wait expired records FA_ERR_TIMEOUT
+ *    in the device error word (read it with fa_get_device_error); kernels
+ *    never trap.
+ *  - The current CUDA device must be the one that holds the buffers.
+ *  - No C++ exception crosses this interface.
+ */
+#ifndef FA_B200_H
+#define FA_B200_H
+
+#include <stddef.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st* fa_stream_t; /* same type as cudaStream_t */
+
+typedef enum {
+    FA_OK = 0,
+    FA_ERR_INVALID_ARG = 1,  /* null pointer, bad size, misaligned pointer      */
+    FA_ERR_UNSUPPORTED = 2,  /* head dimension other than 64 / 128, no sm_100   */
+    FA_ERR_WORKSPACE = 3,    /* workspace missing or smaller than required      */
+    FA_ERR_CUDA = 4,         /* a CUDA runtime / driver call failed             */
+    FA_ERR_TIMEOUT = 5       /* a kernel's bounded wait expired (device word)   */
+} fa_status;
+
+/*
+ * Forward pass.  "DL101 chapter 9", section 3.3 (tiled FlashAttention:
+ * running max m and sum l, O <- O*c + P V, final O / l) and "Flash Attention:
+ * principle & practice", section 2.1 (online softmax).
+ *   q, k, v : bf16 [B, H, N, d], read only.
+ *   o       : bf16 [B, H, N, d], written.
+ *   lse     : float32 [B, H, N], written; may be NULL when not needed.
+ *   causal  : 0 or 1.
+ * Returns FA_OK, FA_ERR_INVALID_ARG, FA_ERR_UNSUPPORTED or FA_ERR_CUDA.
+ */
+fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
+                 int B, int H, int N, int d, int causal, float scale,
+                 fa_stream_t stream);
+
+/*
+ * Bytes of device workspace fa_bwd needs: D = rowsum(dO * O) (float32
+ * [B, H, N]) followed by the float32 dQ accumulator [B, H, N, d], each
+ * region 256-byte aligned.  Returns 0 for invalid sizes.
+ */
+size_t fa_bwd_workspace_size(int B, int H, int N, int d);
+
+/*
+ * Backward pass with recomputation ("Flash Attention La Gi?", thienlv.com,
+ * Recomputation: scores are recomputed from Q, K, V and the saved LSE
+ * instead of being stored).  Gradients of sum(O * dO):
+ *   dV = P^T dO, dP = dO V^T, D = rowsum(dO * O), dS = P * (dP - D),
+ *   dQ = scale dS K, dK = scale dS^T Q.
+ *   q, k, v, o, dout : bf16 [B, H, N, d], read only (o and lse from fa_fwd).
+ *   lse              : float32 [B, H, N], read only.
+ *   dq, dk, dv       : bf16 [B, H, N, d], written.
+ *   workspace        : device buffer of at least fa_bwd_workspace_size bytes,
+ *                      256-byte aligned, owned by the caller; contents on
+ *                      entry are ignored, on exit unspecified.
+ * Returns FA_OK, FA_ERR_INVALID_ARG, FA_ERR_UNSUPPORTED, FA_ERR_WORKSPACE or
+ * FA_ERR_CUDA.
+ */
+fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o,
+                 const void* dout, const float* lse, void* dq, void* dk, void* dv,
+                 void* workspace, size_t ws_bytes,
+                 int B, int H, int N, int d, int causal, float scale,
+                 fa_stream_t stream);
+
+/*
+ * Bytes of device workspace fa_decode needs for the split-KV partials
+ * (per batch, head and split: running max, running sum and an unnormalised
+ * d-vector, float32) for caches of capacity Lmax.  Returns 0 for invalid
+ * sizes.
+ */
+size_t fa_decode_workspace_size(int B, int H, int Lmax, int d);
+
+/*
+ * KV-cache decode: one new query per (batch, head) attends the cached keys
+ * and values at positions 0 .. seqlens[b]-1 ("DL101 chapter 9", section 1.1
+ * Key/Value Caching), split over chunks of the cache whose partial softmax
+ * states are merged afterwards with the rescale-and-add rule of "Flash
+ * Attention: principle & practice", section 2.1.
+ *   q       : bf16 [B, H, d], read only.
+ *   kcache,
+ *   vcache  : bf16 [B, H, Lmax, d], read only; rows at or beyond seqlens[b]
+ *             are never read.
+ *   seqlens : int32 [B] in DEVICE memory, 0 <= seqlens[b] <= Lmax (values
+ *             outside are clamped to that range).
+ *   o       : bf16 [B, H, d], written (zeros where seqlens[b] == 0).
+ *   lse     : float32 [B, H], written (-inf where seqlens[b] == 0); may be NULL.
+ *   workspace : at least fa_decode_workspace_size(B, H, Lmax, d) bytes,
+ *             256-byte aligned, owned by the caller.
+ * Returns FA_OK, FA_ERR_INVALID_ARG, FA_ERR_UNSUPPORTED, FA_ERR_WORKSPACE or
+ * FA_ERR_CUDA.
+ */
+fa_status fa_decode(const void* q, const void* kcache, const void* vcache,
+                    const int* seqlens, void* o, float* lse,
+                    int B, int H, int Lmax, int d, float scale,
+                    void* workspace, size_t ws_bytes, fa_stream_t stream);
+
+/*
+ * Synchronises `stream`, then reads and clears the current device's error
+ * word.  Returns FA_OK, FA_ERR_TIMEOUT (a kernel gave up a bounded wait and
+ * returned without finishing) or FA_ERR_CUDA (the synchronisation failed).
+ */
+fa_status fa_get_device_error(fa_stream_t stream);
+
+/* Static, NUL-terminated description of a status code. */
+const char* fa_status_string(fa_status status);
+
+/* Library version as major * 10000 + minor * 100 + patch. */
+int fa_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FA_B200_H */

@@ -1,0 +1,186 @@
+// fa_api.cu - the C ABI declared in include/fa_b200.h: argument validation,
+// tensor-map encoding, workspace sizing and the device error word.
+#include <climits>
+#include <cstring>
+#include <mutex>
+
+#include "fa_internal.h"
+#include "sm100.cuh"
+
+namespace fa {
+
+namespace {
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(ptr);
+  });
+  return fn;
+}
+
+constexpr int kMaxDevices = 64;
+
+// 1 = sm_100 family, 0 = other, -1 = unknown (query failed).
+fa_status check_device() {
+  static int cache[kMaxDevices];
+  static std::once_flag once;
+  std::call_once(once, [] {
+    for (int i = 0; i < kMaxDevices; ++i) cache[i] = -2;
+  });
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return FA_ERR_CUDA;
+  if (dev < 0 || dev >= kMaxDevices) return FA_ERR_UNSUPPORTED;
+  if (cache[dev] == -2) {
+    int major = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess)
+      return FA_ERR_CUDA;
+    cache[dev] = (major == 10) ? 1 : 0;
+  }
+  return cache[dev] == 1 ? FA_OK : FA_ERR_UNSUPPORTED;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+bool aligned256(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 255u) == 0; }
+
+fa_status check_shape(int B, int H, int N, int d) {
+  if (B < 1 || H < 1 || N < 0) return FA_ERR_INVALID_ARG;
+  if (static_cast<long long>(B) * H > INT_MAX) return FA_ERR_INVALID_ARG;
+  if ((static_cast<long long>(N) + 127) / 128 > 65535) return FA_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
+  return FA_OK;
+}
+
+}  // namespace
+
+fa_status make_tmap_bf16_3d(CUtensorMap* map, const void* base, uint64_t d, uint64_t rows,
+                            uint64_t outer, uint32_t box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (fn == nullptr) return FA_ERR_CUDA;
+  const cuuint64_t dims[3] = {d, rows, outer};
+  const cuuint64_t strides[2] = {d * 2, rows * d * 2};  // bytes, dims 1 and 2
+  const cuuint32_t box[3] = {64u, box_rows, 1u};
+  const cuuint32_t estr[3] = {1u, 1u, 1u};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims,
+                  strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? FA_OK : FA_ERR_CUDA;
+}
+
+}  // namespace fa
+
+using namespace fa;
+
+extern "C" {
+
+const char* fa_status_string(fa_status s) {
+  switch (s) {
+    case FA_OK: return "ok";
+    case FA_ERR_INVALID_ARG: return "invalid argument";
+    case FA_ERR_UNSUPPORTED: return "unsupported head dimension or device";
+    case FA_ERR_WORKSPACE: return "workspace missing or too small";
+    case FA_ERR_CUDA: return "CUDA error";
+    case FA_ERR_TIMEOUT: return "a kernel's bounded wait expired";
+  }
+  return "unknown status";
+}
+
+int fa_version(void) { return 100; }
+
+fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
+                 int N, int d, int causal, float scale, fa_stream_t stream) {
+  fa_status st = check_shape(B, H, N, d);
+  if (st != FA_OK) return st;
+  if (!q || !k || !v || !o) return FA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o)) return FA_ERR_INVALID_ARG;
+  if (lse != nullptr && (reinterpret_cast<uintptr_t>(lse) & 3u)) return FA_ERR_INVALID_ARG;
+  if (causal != 0 && causal != 1) return FA_ERR_INVALID_ARG;
+  if (!(scale == scale)) return FA_ERR_INVALID_ARG;  // NaN
+  if ((st = check_device()) != FA_OK) return st;
+  if (N == 0) return FA_OK;
+  return launch_fwd(q, k, v, o, lse, B, H, N, d, causal, scale,
+                    reinterpret_cast<cudaStream_t>(stream));
+}
+
+size_t fa_bwd_workspace_size(int B, int H, int N, int d) {
+  if (check_shape(B, H, N, d) != FA_OK) return 0;
+  const size_t rows = static_cast<size_t>(B) * H * N;
+  return align_up(rows * sizeof(float), 256) + align_up(rows * d * sizeof(float), 256);
+}
+
+fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, const void* dout,
+                 const float* lse, void* dq, void* dk, void* dv, void* workspace,
+                 size_t ws_bytes, int B, int H, int N, int d, int causal, float scale,
+                 fa_stream_t stream) {
+  fa_status st = check_shape(B, H, N, d);
+  if (st != FA_OK) return st;
+  if (!q || !k || !v || !o || !dout || !lse || !dq || !dk || !dv) return FA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(dout) ||
+      !aligned16(dq) || !aligned16(dk) || !aligned16(dv) ||
+      (reinterpret_cast<uintptr_t>(lse) & 3u))
+    return FA_ERR_INVALID_ARG;
+  if (causal != 0 && causal != 1) return FA_ERR_INVALID_ARG;
+  if (!(scale == scale)) return FA_ERR_INVALID_ARG;
+  const size_t need = fa_bwd_workspace_size(B, H, N, d);
+  if (N > 0 && (workspace == nullptr || ws_bytes < need || !aligned256(workspace)))
+    return FA_ERR_WORKSPACE;
+  if ((st = check_device()) != FA_OK) return st;
+  if (N == 0) return FA_OK;
+  return launch_bwd(q, k, v, o, dout, lse, dq, dk, dv, workspace, B, H, N, d, causal, scale,
+                    reinterpret_cast<cudaStream_t>(stream));
+}
+
+size_t fa_decode_workspace_size(int B, int H, int Lmax, int d) {
+  if (B < 1 || H < 1 || Lmax < 0 || (d != 64 && d != 128)) return 0;
+  if (static_cast<long long>(B) * H > INT_MAX) return 0;
+  const size_t splits = static_cast<size_t>(decode_num_splits(Lmax));
+  return align_up(static_cast<size_t>(B) * H * splits * (d + 2) * sizeof(float), 256);
+}
+
+fa_status fa_decode(const void* q, const void* kcache, const void* vcache, const int* seqlens,
+                    void* o, float* lse, int B, int H, int Lmax, int d, float scale,
+                    void* workspace, size_t ws_bytes, fa_stream_t stream) {
+  if (B < 1 || H < 1 || Lmax < 0) return FA_ERR_INVALID_ARG;
+  if (static_cast<long long>(B) * H > INT_MAX) return FA_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
+  if (!q || !kcache || !vcache || !seqlens || !o) return FA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(kcache) || !aligned16(vcache) || !aligned16(o) ||
+      (reinterpret_cast<uintptr_t>(seqlens) & 3u) ||
+      (lse != nullptr && (reinterpret_cast<uintptr_t>(lse) & 3u)))
+    return FA_ERR_INVALID_ARG;
+  if (!(scale == scale)) return FA_ERR_INVALID_ARG;
+  const size_t need = fa_decode_workspace_size(B, H, Lmax, d);
+  if (need > 0 && (workspace == nullptr || ws_bytes < need || !aligned256(workspace)))
+    return FA_ERR_WORKSPACE;
+  fa_status st = check_device();
+  if (st != FA_OK) return st;
+  return launch_decode(q, kcache, vcache, seqlens, o, lse, B, H, Lmax, d, scale,
+                       static_cast<float*>(workspace), reinterpret_cast<cudaStream_t>(stream));
+}
+
+fa_status fa_get_device_error(fa_stream_t stream) {
+  if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return FA_ERR_CUDA;
+  int v = 0;
+  if (cudaMemcpyFromSymbol(&v, fa::g_device_error, sizeof(int)) != cudaSuccess)
+    return FA_ERR_CUDA;
+  if (v != 0) {
+    const int zero = 0;
+    if (cudaMemcpyToSymbol(fa::g_device_error, &zero, sizeof(int)) != cudaSuccess)
+      return FA_ERR_CUDA;
+  }
+  return v == 0 ? FA_OK : static_cast<fa_status>(v);
+}
+
+}  // extern "C"

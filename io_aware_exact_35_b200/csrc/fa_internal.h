@@ -1,0 +1,38 @@
+// fa_internal.h - host-side declarations shared by the C-ABI front end and the
+// kernel launchers.  Not part of the public interface.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cstddef>
+#include <cstdint>
+
+#include "../../include/fa_b200.h"
+
+namespace fa {
+
+// Encodes a 3-D bf16 tensor map over a [outer, rows, d] array (d innermost)
+// with a box of 64 x box_rows x 1 elements and 128-byte swizzle.  Rows beyond
+// `rows` read as zero, so a tile never spills into the next (batch, head).
+fa_status make_tmap_bf16_3d(CUtensorMap* map, const void* base, uint64_t d, uint64_t rows,
+                            uint64_t outer, uint32_t box_rows);
+
+fa_status launch_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B,
+                     int H, int N, int d, int causal, float scale, cudaStream_t stream);
+
+fa_status launch_bwd(const void* q, const void* k, const void* v, const void* o,
+                     const void* dout, const float* lse, void* dq, void* dk, void* dv,
+                     void* workspace, int B, int H, int N, int d, int causal, float scale,
+                     cudaStream_t stream);
+
+int decode_num_splits(int Lmax);
+fa_status launch_decode(const void* q, const void* kc, const void* vc, const int* seqlens,
+                        void* o, float* lse, int B, int H, int Lmax, int d, float scale,
+                        float* partials, cudaStream_t stream);
+
+inline fa_status cuda_status(cudaError_t e) { return e == cudaSuccess ? FA_OK : FA_ERR_CUDA; }
+
+inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+}  // namespace fa

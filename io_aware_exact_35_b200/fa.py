@@ -1,0 +1,192 @@
+"""Python binding of libfa_b200.so (argument marshalling only).
+
+Every function takes torch CUDA tensors, checks dtype / shape / contiguity,
+allocates outputs when none are given, and calls the C ABI of
+include/fa_b200.h with raw device pointers and the current CUDA stream.  All
+arithmetic happens in the library's sm_100a kernels; there is no fallback:
+if the library is missing or the device is unsupported, the call raises.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+from typing import Optional
+
+import torch
+
+_LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "lib", "libfa_b200.so")
+_lib = None
+
+FA_OK = 0
+STATUS_NAMES = {0: "FA_OK", 1: "FA_ERR_INVALID_ARG", 2: "FA_ERR_UNSUPPORTED",
+                3: "FA_ERR_WORKSPACE", 4: "FA_ERR_CUDA", 5: "FA_ERR_TIMEOUT"}
+
+# Public entry points and their C signatures (restype, argtypes).
+_P, _I, _F, _S = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
+SIGNATURES = {
+    "fa_fwd": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _P]),
+    "fa_bwd_workspace_size": (_S, [_I, _I, _I, _I]),
+    "fa_bwd": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _S, _I, _I, _I, _I, _I, _F, _P]),
+    "fa_decode_workspace_size": (_S, [_I, _I, _I, _I]),
+    "fa_decode": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _F, _P, _S, _P]),
+    "fa_get_device_error": (_I, [_P]),
+    "fa_status_string": (ctypes.c_char_p, [_I]),
+    "fa_version": (_I, []),
+}
+
+
+class FAError(RuntimeError):
+    def __init__(self, fn: str, status: int):
+        self.status = status
+        name = STATUS_NAMES.get(status, str(status))
+        super().__init__(f"{fn} failed: {name} ({status_string(status)})")
+
+
+def library_path() -> str:
+    return _LIB_PATH
+
+
+def lib():
+    """Load libfa_b200.so once; raise if it has not been built."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(_LIB_PATH):
+            raise RuntimeError(f"{_LIB_PATH} is missing: build it with "
+                               "`python -m io_aware_exact_35_b200.build`")
+        handle = ctypes.CDLL(_LIB_PATH)
+        for name, (res, args) in SIGNATURES.items():
+            fn = getattr(handle, name)
+            fn.restype, fn.argtypes = res, args
+        _lib = handle
+    return _lib
+
+
+def status_string(status: int) -> str:
+    return lib().fa_status_string(int(status)).decode()
+
+
+def _check(fn: str, status: int) -> None:
+    if status != FA_OK:
+        raise FAError(fn, status)
+
+
+def _stream_ptr(stream: Optional[torch.cuda.Stream]) -> int:
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return s.cuda_stream
+
+
+def _req(t: torch.Tensor, name: str, dtype: torch.dtype, ndim: int) -> None:
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if t.dim() != ndim:
+        raise ValueError(f"{name} must have {ndim} dims, got {tuple(t.shape)}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+def _ptr(t: Optional[torch.Tensor]) -> Optional[int]:
+    return None if t is None else t.data_ptr()
+
+
+def fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, causal: bool = False,
+        scale: Optional[float] = None, out: Optional[torch.Tensor] = None,
+        lse: Optional[torch.Tensor] = None, want_lse: bool = True, stream=None):
+    """Exact attention forward.  q, k, v: bf16 [B, H, N, d].  Returns (o, lse)."""
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _req(t, n, torch.bfloat16, 4)
+    if k.shape != q.shape or v.shape != q.shape:
+        raise ValueError("q, k and v must have the same shape [B, H, N, d]")
+    B, H, N, d = q.shape
+    scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
+    if out is None:
+        out = torch.empty_like(q)
+    _req(out, "out", torch.bfloat16, 4)
+    if out.shape != q.shape:
+        raise ValueError("out must match q")
+    if lse is None and want_lse:
+        lse = torch.empty((B, H, N), dtype=torch.float32, device=q.device)
+    if lse is not None:
+        _req(lse, "lse", torch.float32, 3)
+        if tuple(lse.shape) != (B, H, N):
+            raise ValueError("lse must be [B, H, N]")
+    st = lib().fa_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), _ptr(lse),
+                      B, H, N, d, int(bool(causal)), scale, _stream_ptr(stream))
+    _check("fa_fwd", st)
+    return out, lse
+
+
+def bwd_workspace_size(B: int, H: int, N: int, d: int) -> int:
+    return int(lib().fa_bwd_workspace_size(B, H, N, d))
+
+
+def bwd(q, k, v, o, do, lse, causal: bool = False, scale: Optional[float] = None,
+        dq=None, dk=None, dv=None, workspace: Optional[torch.Tensor] = None, stream=None):
+    """Backward with recomputation.  Returns (dq, dk, dv), bf16 [B, H, N, d]."""
+    for t, n in ((q, "q"), (k, "k"), (v, "v"), (o, "o"), (do, "do")):
+        _req(t, n, torch.bfloat16, 4)
+        if t.shape != q.shape:
+            raise ValueError(f"{n} must match q's shape")
+    B, H, N, d = q.shape
+    _req(lse, "lse", torch.float32, 3)
+    if tuple(lse.shape) != (B, H, N):
+        raise ValueError("lse must be [B, H, N]")
+    scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(q) if dk is None else dk
+    dv = torch.empty_like(q) if dv is None else dv
+    for t, n in ((dq, "dq"), (dk, "dk"), (dv, "dv")):
+        _req(t, n, torch.bfloat16, 4)
+    need = bwd_workspace_size(B, H, N, d)
+    if workspace is None:
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=q.device)
+    st = lib().fa_bwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), do.data_ptr(),
+                      lse.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(),
+                      workspace.data_ptr(), workspace.numel() * workspace.element_size(),
+                      B, H, N, d, int(bool(causal)), scale, _stream_ptr(stream))
+    _check("fa_bwd", st)
+    return dq, dk, dv
+
+
+def decode_workspace_size(B: int, H: int, Lmax: int, d: int) -> int:
+    return int(lib().fa_decode_workspace_size(B, H, Lmax, d))
+
+
+def decode(q, kcache, vcache, seqlens, scale: Optional[float] = None, out=None, lse=None,
+           want_lse: bool = True, workspace: Optional[torch.Tensor] = None, stream=None):
+    """Split-KV decode.  q [B,H,d], caches [B,H,Lmax,d] bf16, seqlens int32 [B]
+    on the device.  Returns (o [B,H,d] bf16, lse [B,H] fp32)."""
+    _req(q, "q", torch.bfloat16, 3)
+    _req(kcache, "kcache", torch.bfloat16, 4)
+    _req(vcache, "vcache", torch.bfloat16, 4)
+    _req(seqlens, "seqlens", torch.int32, 1)
+    B, H, d = q.shape
+    Lmax = kcache.shape[2]
+    if tuple(kcache.shape) != (B, H, Lmax, d) or vcache.shape != kcache.shape:
+        raise ValueError("caches must be [B, H, Lmax, d] matching q")
+    if seqlens.shape[0] != B:
+        raise ValueError("seqlens must have B entries")
+    scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
+    out = torch.empty_like(q) if out is None else out
+    _req(out, "out", torch.bfloat16, 3)
+    if lse is None and want_lse:
+        lse = torch.empty((B, H), dtype=torch.float32, device=q.device)
+    need = decode_workspace_size(B, H, Lmax, d)
+    if workspace is None:
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=q.device)
+    st = lib().fa_decode(q.data_ptr(), kcache.data_ptr(), vcache.data_ptr(), seqlens.data_ptr(),
+                         out.data_ptr(), _ptr(lse), B, H, Lmax, d, scale,
+                         workspace.data_ptr(), workspace.numel() * workspace.element_size(),
+                         _stream_ptr(stream))
+    _check("fa_decode", st)
+    return out, lse
+
+
+def get_device_error(stream=None) -> int:
+    """Synchronise the stream and return (and clear) the device error word."""
+    return int(lib().fa_get_device_error(_stream_ptr(stream)))

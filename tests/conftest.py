@@ -19,3 +19,12 @@ def cuda_device():
     if not torch.cuda.is_available():
         pytest.skip("no CUDA device")
     return torch.device("cuda:0")
+
+
+@pytest.fixture(scope="session")
+def fa_mod():
+    """The binding module with the in-tree library built (nvcc, sm_100a)."""
+    from io_aware_exact_35_b200 import build, fa
+    build.build()
+    fa.lib()
+    return fa

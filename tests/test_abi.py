@@ -1,0 +1,89 @@
+"""CPU checks of the C ABI: the library builds for sm_100a, loads, exports every
+entry point declared in include/*.h, and sizes workspaces / rejects bad
+arguments on the host before touching a device."""
+import ctypes
+import glob
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def declared_functions():
+    names = set()
+    for h in glob.glob(os.path.join(ROOT, "include", "*.h")):
+        text = open(h).read()
+        text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+        for m in re.finditer(r"\b(fa_\w+)\s*\(", text):
+            names.add(m.group(1))
+    return names
+
+
+def test_header_declares_the_boundary():
+    names = declared_functions()
+    for required in ("fa_fwd", "fa_bwd", "fa_decode", "fa_bwd_workspace_size",
+                     "fa_decode_workspace_size", "fa_get_device_error", "fa_status_string"):
+        assert required in names
+
+
+def test_library_exports_every_declared_symbol(fa_mod):
+    lib = ctypes.CDLL(fa_mod.library_path())
+    for name in declared_functions():
+        assert hasattr(lib, name), f"{name} declared in include/ but not exported"
+    assert set(fa_mod.SIGNATURES) <= declared_functions()
+
+
+def test_status_strings(fa_mod):
+    for code in range(6):
+        assert fa_mod.status_string(code)
+    assert fa_mod.lib().fa_version() >= 100
+
+
+def test_workspace_sizes(fa_mod):
+    B, H, N, d = 2, 16, 8192, 128
+    ws = fa_mod.bwd_workspace_size(B, H, N, d)
+    rows = B * H * N
+    assert ws >= rows * 4 + rows * d * 4
+    assert ws % 256 == 0
+    assert fa_mod.bwd_workspace_size(0, 1, 1, 128) == 0
+    assert fa_mod.bwd_workspace_size(1, 1, 1, 96) == 0
+    wd = fa_mod.decode_workspace_size(16, 32, 16384, 128)
+    assert wd >= 16 * 32 * (d + 2) * 4 and wd % 256 == 0
+    assert fa_mod.decode_workspace_size(1, 1, 0, 128) == 0
+    assert fa_mod.decode_workspace_size(1, 1, 10, 80) == 0
+
+
+def test_host_validation_rejects_bad_arguments(fa_mod):
+    lib = fa_mod.lib()
+    P = 1 << 20  # a fake, aligned address: never dereferenced on these paths
+    INVALID, UNSUPPORTED, WORKSPACE = 1, 2, 3
+    # null pointers, negative sizes, misalignment, bad flags, bad head dims
+    assert lib.fa_fwd(None, P, P, P, None, 1, 1, 8, 64, 0, 1.0, None) == INVALID
+    assert lib.fa_fwd(P, P, P, P, None, 0, 1, 8, 64, 0, 1.0, None) == INVALID
+    assert lib.fa_fwd(P, P, P, P, None, 1, 1, -1, 64, 0, 1.0, None) == INVALID
+    assert lib.fa_fwd(P + 8, P, P, P, None, 1, 1, 8, 64, 0, 1.0, None) == INVALID
+    assert lib.fa_fwd(P, P, P, P, P + 2, 1, 1, 8, 64, 0, 1.0, None) == INVALID
+    assert lib.fa_fwd(P, P, P, P, None, 1, 1, 8, 64, 2, 1.0, None) == INVALID
+    assert lib.fa_fwd(P, P, P, P, None, 1, 1, 8, 64, 0, float("nan"), None) == INVALID
+    assert lib.fa_fwd(P, P, P, P, None, 1, 1, 8, 96, 0, 1.0, None) == UNSUPPORTED
+    assert lib.fa_fwd(P, P, P, P, None, 1, 1, 128 * 65536, 64, 0, 1.0, None) == INVALID
+    # backward: workspace checks
+    args = [P] * 6 + [P, P, P]
+    assert lib.fa_bwd(*args, None, 0, 1, 1, 8, 64, 0, 1.0, None) == WORKSPACE
+    assert lib.fa_bwd(*args, P, 16, 1, 1, 8, 64, 0, 1.0, None) == WORKSPACE
+    assert lib.fa_bwd(*args, P + 16, 1 << 20, 1, 1, 8, 64, 0, 1.0, None) == WORKSPACE
+    assert lib.fa_bwd(None, *args[1:], P, 1 << 20, 1, 1, 8, 64, 0, 1.0, None) == INVALID
+    # decode
+    assert lib.fa_decode(P, P, P, P, P, None, 1, 1, 1024, 128, 1.0, None, 0, None) == WORKSPACE
+    assert lib.fa_decode(P, P, P, P + 2, P, None, 1, 1, 1024, 128, 1.0, P, 1 << 20, None) == INVALID
+    assert lib.fa_decode(P, P, P, P, P, None, 1, 1, 1024, 80, 1.0, P, 1 << 20, None) == UNSUPPORTED
+    assert lib.fa_decode(P, P, None, P, P, None, 1, 1, 1024, 128, 1.0, P, 1 << 20, None) == INVALID
+
+
+def test_binding_fails_loudly_without_cuda_tensors(fa_mod):
+    import torch
+    x = torch.zeros(1, 1, 8, 64, dtype=torch.bfloat16)
+    with pytest.raises(ValueError):
+        fa_mod.fwd(x, x, x)

@@ -1,0 +1,100 @@
+"""GPU parity of the forward kernel against the fp64 oracle (through the C ABI)."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from io_aware_exact_35_b200 import inputs
+from tests._parity import check_lse, check_o, check_o_scaled
+
+pytestmark = pytest.mark.gpu
+
+
+def _run(fa_mod, q, k, v, causal, scale):
+    dev = torch.device("cuda:0")
+    o, lse = fa_mod.fwd(q.to(dev), k.to(dev), v.to(dev), causal=causal, scale=scale)
+    torch.cuda.synchronize()
+    assert fa_mod.get_device_error() == 0
+    return o.cpu(), lse.cpu()
+
+
+SMALL = [
+    # (B, H, N, d): several tiles, ragged tails, sub-tile sizes
+    (1, 2, 1, 64), (1, 1, 7, 128), (2, 3, 64, 64), (1, 2, 128, 128), (1, 2, 129, 128),
+    (2, 2, 255, 64), (1, 3, 256, 128), (2, 1, 401, 128), (1, 1, 1000, 64), (1, 2, 1153, 128),
+]
+
+
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("shape", SMALL, ids=lambda s: "B%dH%dN%dd%d" % s)
+def test_fwd_small_shapes(fa_mod, cuda_device, shape, causal):
+    B, H, N, d = shape
+    q, k, v = inputs.fwd_inputs(B, H, N, d, seed=1000 + N + d + causal)
+    scale = 1.0 / np.sqrt(d)
+    o, lse = _run(fa_mod, q, k, v, causal, scale)
+    o_ref, lse_ref = oracle.attention_forward(inputs.to_f64(q), inputs.to_f64(k),
+                                              inputs.to_f64(v), causal, scale)
+    check_o(o, o_ref)
+    check_lse(lse, lse_ref)
+
+
+def test_fwd_large_scores_and_rescaling(fa_mod, cuda_device):
+    # Scores spanning a wide range force the running maximum to move often.
+    B, H, N, d = 1, 2, 777, 128
+    q, k, v = inputs.fwd_inputs(B, H, N, d, seed=7, std=1.0)
+    ramp = torch.linspace(0.1, 4.0, N).view(1, 1, N, 1)
+    k = (k.float() * ramp).to(torch.bfloat16)
+    for causal in (False, True):
+        o, lse = _run(fa_mod, q, k, v, causal, 0.3)
+        o_ref, lse_ref = oracle.attention_forward(inputs.to_f64(q), inputs.to_f64(k),
+                                                  inputs.to_f64(v), causal, 0.3)
+        check_o_scaled(o, o_ref)
+        check_lse(lse, lse_ref)
+
+
+def test_fwd_workload_noncausal_B1_H2_N256_d64(fa_mod, cuda_device):
+    w = inputs.WORKLOADS["fwd_noncausal_B1_H2_N256_d64"]
+    q, k, v = inputs.workload_inputs(w)
+    o, lse = _run(fa_mod, q, k, v, w.causal, w.scale)
+    o_ref, lse_ref = oracle.attention_forward(inputs.to_f64(q), inputs.to_f64(k),
+                                              inputs.to_f64(v), w.causal, w.scale)
+    check_o(o, o_ref)
+    check_lse(lse, lse_ref)
+
+
+def test_fwd_workload_causal_B4_H16_N2048_d128(fa_mod, cuda_device):
+    w = inputs.WORKLOADS["fwd_causal_B4_H16_N2048_d128"]
+    q, k, v = inputs.workload_inputs(w)
+    o, lse = _run(fa_mod, q, k, v, w.causal, w.scale)
+    o_ref, lse_ref = oracle.attention_forward(inputs.to_f64(q), inputs.to_f64(k),
+                                              inputs.to_f64(v), w.causal, w.scale)
+    check_o(o, o_ref)
+    check_lse(lse, lse_ref)
+
+
+def test_fwd_workload_causal_B1_H32_N32768_d128_sampled(fa_mod, cuda_device):
+    """Full-size long-context run; sampled rows of sampled heads vs the oracle."""
+    w = inputs.WORKLOADS["fwd_causal_B1_H32_N32768_d128"]
+    q, k, v = inputs.workload_inputs(w)
+    o, lse = _run(fa_mod, q, k, v, w.causal, w.scale)
+    assert torch.isfinite(o.float()).all() and torch.isfinite(lse).all()
+    rows = inputs.sample_rows(w.N, 96, seed=w.seed, edge=64)
+    for h in (0, 13, 31):
+        qh, kh, vh = (inputs.to_f64(t[0, h]) for t in (q, k, v))
+        o_ref, lse_ref = oracle.attention_forward_rows(qh, kh, vh, True, w.scale, rows)
+        check_o(o[0, h, rows], o_ref, f"O head {h}")
+        check_lse(lse[0, h, rows], lse_ref, f"LSE head {h}")
+
+
+def test_fwd_output_buffers_and_streams(fa_mod, cuda_device):
+    B, H, N, d = 1, 2, 300, 64
+    q, k, v = (t.cuda() for t in inputs.fwd_inputs(B, H, N, d, seed=3))
+    out = torch.full_like(q, float("nan"))
+    s = torch.cuda.Stream()
+    with torch.cuda.stream(s):
+        o, lse = fa_mod.fwd(q, k, v, causal=True, out=out, want_lse=False)
+    s.synchronize()
+    assert lse is None and o.data_ptr() == out.data_ptr()
+    o_ref, _ = oracle.attention_forward(*(inputs.to_f64(t) for t in (q, k, v)), True,
+                                        1 / np.sqrt(d))
+    check_o(o.cpu(), o_ref)
