@@ -69,9 +69,10 @@ fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* ls
                  fa_stream_t stream);
 
 /*
- * Bytes of device workspace fa_bwd needs: D = rowsum(dO * O) (float32
- * [B, H, N]) followed by the float32 dQ accumulator [B, H, N, d], each
- * region 256-byte aligned.  Returns 0 for invalid sizes.
+ * Bytes of device workspace fa_bwd needs: D = rowsum(dO * O) and
+ * log2(e) * LSE as float32 [B, H, Np] with Np = N rounded up to a multiple
+ * of 128, followed by the float32 dQ accumulator [B, H, N, d], each region
+ * 256-byte aligned.  Returns 0 for invalid sizes.
  */
 size_t fa_bwd_workspace_size(int B, int H, int N, int d);
 

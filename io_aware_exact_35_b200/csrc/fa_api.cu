@@ -78,6 +78,19 @@ fa_status make_tmap_bf16_3d(CUtensorMap* map, const void* base, uint64_t d, uint
   return r == CUDA_SUCCESS ? FA_OK : FA_ERR_CUDA;
 }
 
+fa_status make_tmap_f32_2d(CUtensorMap* map, const void* base, uint64_t n, uint64_t outer) {
+  EncodeTiledFn fn = encode_fn();
+  if (fn == nullptr) return FA_ERR_CUDA;
+  const cuuint64_t dims[2] = {n, outer};
+  const cuuint64_t strides[1] = {n * 4};
+  const cuuint32_t box[2] = {128u, 1u};
+  const cuuint32_t estr[2] = {1u, 1u};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<void*>(base), dims, strides,
+                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? FA_OK : FA_ERR_CUDA;
+}
+
 }  // namespace fa
 
 using namespace fa;
@@ -115,8 +128,11 @@ fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* ls
 
 size_t fa_bwd_workspace_size(int B, int H, int N, int d) {
   if (check_shape(B, H, N, d) != FA_OK) return 0;
-  const size_t rows = static_cast<size_t>(B) * H * N;
-  return align_up(rows * sizeof(float), 256) + align_up(rows * d * sizeof(float), 256);
+  const size_t bh = static_cast<size_t>(B) * H;
+  const size_t padded = bh * bwd_row_pad(N);
+  // D and log2(e) * LSE on 128-padded rows, then the fp32 dQ accumulator
+  return 2 * align_up(padded * sizeof(float), 256) +
+         align_up(bh * static_cast<size_t>(N) * d * sizeof(float), 256);
 }
 
 fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, const void* dout,

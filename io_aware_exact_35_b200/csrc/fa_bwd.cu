@@ -1,12 +1,503 @@
-// fa_bwd.cu - backward pass (placeholder until the sm_100a kernels land).
+// fa_bwd.cu - backward pass of exact attention on sm_100a, with recomputation.
+//
+// "Flash Attention La Gi?" (thienlv.com glossary), Recomputation: the
+// attention matrix is not stored by the forward pass; the backward pass
+// recomputes it tile by tile from Q, K and the saved log-sum-exp.  With
+// L = sum(O * dO) and S = scale Q K^T:
+//   P = exp(S - LSE),  dV = P^T dO,  dP = dO V^T,  D = rowsum(dO * O),
+//   dS = P * (dP - D),  dQ = scale dS K,  dK = scale dS^T Q.
+//
+// Three kernels:
+//   fa_bwd_preprocess  D = rowsum(dO * O) (fp32) and a zeroed fp32 dQ accumulator.
+//   fa_bwd_kernel      one CTA per 128-key tile j of one (batch, head); it keeps
+//                      dK_j and dV_j in tensor memory and loops over the query
+//                      tiles i that can see key tile j (i >= j when causal):
+//                        S^T = K_j Q_i^T, dP^T = V_j dO_i^T        (tcgen05, TMEM)
+//                        P^T, dS^T on the CUDA cores (one key row per thread)
+//                        dV += P^T dO_i, dK += dS^T Q_i            (A from TMEM)
+//                        dQ_i = dS K_j  (A = dS from shared memory) -> fp32
+//                        vector reductions into the dQ accumulator.
+//   fa_bwd_dq_convert  dQ = scale * accumulator, rounded to bf16.
+//
+// Warp roles of fa_bwd_kernel (320 threads):
+//   warps 0-3  "softmax" warpgroup: thread t owns key row t (TMEM lane t).
+//   warps 4-7  dQ warpgroup: thread t owns query row t of the dQ tile.
+//   warp 8     TMA producer: K_j, V_j once; Q_i, dO_i, LSE_i, D_i through a
+//              two-stage ring.
+//   warp 9     tensor-memory allocator and MMA issuer.
+// Tensor memory (512 columns): S^T [0,128) (P^T bf16 overwrites its first 64
+// columns), dP^T [128,256) (dS^T bf16 overwrites its first 64 columns, and
+// dQ_i lands in [128, 128+d) afterwards), dV [256, 256+d), dK [256+d, 256+2d).
 #include "fa_internal.h"
+#include "sm100.cuh"
 
 namespace fa {
 
-fa_status launch_bwd(const void*, const void*, const void*, const void*, const void*,
-                     const float*, void*, void*, void*, void*, int, int, int, int, int, float,
-                     cudaStream_t) {
-  return FA_ERR_UNSUPPORTED;
+namespace bwd {
+
+constexpr int BLOCK = 128;
+constexpr int NUM_THREADS = 320;
+constexpr int PANEL_BYTES = 128 * 128;
+constexpr uint32_t TMEM_COLS = 512;
+constexpr float LOG2E = 1.4426950408889634f;
+
+template <int D>
+struct Smem {
+  static constexpr int NPANEL = D / 64;
+  static constexpr int TILE = NPANEL * PANEL_BYTES;  // 128 rows x D bf16
+  static constexpr int K_OFF = 0;
+  static constexpr int V_OFF = TILE;
+  static constexpr int Q_OFF = 2 * TILE;               // 2 stages
+  static constexpr int DO_OFF = Q_OFF + 2 * TILE;      // 2 stages
+  static constexpr int DS_OFF = DO_OFF + 2 * TILE;     // 128 keys x 128 queries bf16
+  static constexpr int DS_BYTES = 2 * PANEL_BYTES;
+  static constexpr int LSE_OFF = DS_OFF + DS_BYTES;    // 2 stages x 128 fp32
+  static constexpr int DD_OFF = LSE_OFF + 2 * 512;     // 2 stages x 128 fp32
+  static constexpr int BAR_OFF = DD_OFF + 2 * 512;
+  // kv_full, qd_full[2], qd_empty[2], st_full, dpt_full, pds_full, dq_full,
+  // dq_free, dkv_final, mma_final
+  static constexpr int NBAR = 12;
+  static constexpr int MISC_OFF = BAR_OFF + NBAR * 8;
+  static constexpr int BYTES = MISC_OFF + 16;
+  static constexpr int ALLOC = BYTES > 118784 ? BYTES : 118784;
+};
+
+struct Params {
+  __nv_bfloat16* dk;
+  __nv_bfloat16* dv;
+  float* dqacc;
+  int N;
+  int n_tiles;
+  float scale_log2;  // scale * log2(e)
+  float scale;
+};
+
+__device__ __forceinline__ void red_add_v4(float* addr, float a, float b, float c, float d) {
+  asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(addr), "f"(a), "f"(b),
+               "f"(c), "f"(d)
+               : "memory");
+}
+
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+__device__ __forceinline__ void tma_load_2d(void* smem_dst, const void* desc, uint64_t* bar,
+                                            int c0, int c1) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3}], [%4];" ::"r"(smem_u32(smem_dst)),
+      "l"(desc), "r"(c0), "r"(c1), "r"(smem_u32(bar))
+      : "memory");
+}
+
+template <int D, bool CAUSAL>
+__global__ void __launch_bounds__(NUM_THREADS, 1)
+    fa_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                  const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
+                  const __grid_constant__ CUtensorMap tm_lse,
+                  const __grid_constant__ CUtensorMap tm_dd, const Params p) {
+  using L = Smem<D>;
+  extern __shared__ __align__(1024) uint8_t smem[];
+  // The swizzled operand tiles need 1024-byte alignment; the kernel declares
+  // no static shared memory, so the dynamic window starts aligned.
+  if ((smem_u32(smem) & 1023u) != 0) {
+    if (threadIdx.x == 0) record_error(2 /* FA_ERR_UNSUPPORTED */);
+    return;
+  }
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::BAR_OFF);
+  uint64_t* kv_full = bars + 0;
+  uint64_t* qd_full = bars + 1;   // [2]
+  uint64_t* qd_empty = bars + 3;  // [2]
+  uint64_t* st_full = bars + 5;
+  uint64_t* dpt_full = bars + 6;
+  uint64_t* pds_full = bars + 7;
+  uint64_t* dq_full = bars + 8;
+  uint64_t* dq_free = bars + 9;
+  uint64_t* dkv_final = bars + 10;
+  uint64_t* mma_final = bars + 11;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::MISC_OFF);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::MISC_OFF + 4);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int bh = blockIdx.x;
+  const int kv_tile = blockIdx.y;  // tile 0 sees the most query tiles: launched first
+  const int key0 = kv_tile * BLOCK;
+  const int i_begin = CAUSAL ? kv_tile : 0;
+  const int n_it = p.n_tiles - i_begin;
+
+  if (threadIdx.x == 0) {
+    for (int b = 0; b < L::NBAR; ++b) mbar_init(&bars[b], 1);
+    mbar_init(pds_full, BLOCK);
+    mbar_init(dq_free, BLOCK);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 9) {
+    tmem_alloc(tmem_slot, TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  const uint32_t tSt = tmem_base;
+  const uint32_t tdPt = tmem_base + 128;
+  const uint32_t tdV = tmem_base + 256;
+  const uint32_t tdK = tmem_base + 256 + D;
+
+  if (warp == 8) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      tma_prefetch_desc(&tm_q);
+      tma_prefetch_desc(&tm_do);
+      int last[2] = {-1, -1};
+      mbar_arrive_expect_tx(kv_full, 2 * L::TILE);
+      for (int pn = 0; pn < L::NPANEL; ++pn) {
+        tma_load_3d(smem + L::K_OFF + pn * PANEL_BYTES, &tm_k, kv_full, pn * 64, key0, bh);
+        tma_load_3d(smem + L::V_OFF + pn * PANEL_BYTES, &tm_v, kv_full, pn * 64, key0, bh);
+      }
+      for (int it = 0; it < n_it; ++it) {
+        const int st = it & 1;
+        const int r = it >> 1;
+        const int q0 = (i_begin + it) * BLOCK;
+        if (it >= 2 && !mbar_wait(&qd_empty[st], (r - 1) & 1, abort_flag)) break;
+        mbar_arrive_expect_tx(&qd_full[st], 2 * L::TILE + 1024);
+        for (int pn = 0; pn < L::NPANEL; ++pn) {
+          tma_load_3d(smem + L::Q_OFF + st * L::TILE + pn * PANEL_BYTES, &tm_q, &qd_full[st],
+                      pn * 64, q0, bh);
+          tma_load_3d(smem + L::DO_OFF + st * L::TILE + pn * PANEL_BYTES, &tm_do, &qd_full[st],
+                      pn * 64, q0, bh);
+        }
+        tma_load_2d(smem + L::LSE_OFF + st * 512, &tm_lse, &qd_full[st], q0, bh);
+        tma_load_2d(smem + L::DD_OFF + st * 512, &tm_dd, &qd_full[st], q0, bh);
+        last[st] = r;
+      }
+      mbar_wait_drain(kv_full, 0);
+      for (int s = 0; s < 2; ++s)
+        if (last[s] >= 0) mbar_wait_drain(&qd_full[s], last[s] & 1);
+    }
+  } else if (warp == 9) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t IDESC_SS = idesc_bf16_f32(BLOCK, BLOCK, false, false);
+      constexpr uint32_t IDESC_ACC = idesc_bf16_f32(BLOCK, D, false, true);
+      constexpr uint32_t IDESC_DQ = idesc_bf16_f32(BLOCK, D, true, true);
+      const uint32_t k_addr = smem_u32(smem + L::K_OFF);
+      const uint32_t v_addr = smem_u32(smem + L::V_OFF);
+      const uint32_t ds_addr = smem_u32(smem + L::DS_OFF);
+      bool ok = mbar_wait(kv_full, 0, abort_flag);
+      for (int it = 0; ok && it < n_it; ++it) {
+        const int st = it & 1;
+        const uint32_t q_addr = smem_u32(smem + L::Q_OFF + st * L::TILE);
+        const uint32_t do_addr = smem_u32(smem + L::DO_OFF + st * L::TILE);
+        if (!mbar_wait(&qd_full[st], (it >> 1) & 1, abort_flag)) { ok = false; break; }
+        tc_fence_after();
+        // S^T = K_j Q_i^T  (M = keys, N = queries, K = d)
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * PANEL_BYTES + (kk & 3) * 32;
+          mma_bf16_ss(tSt, sdesc_kmajor_sw128(k_addr + off), sdesc_kmajor_sw128(q_addr + off),
+                      IDESC_SS, kk > 0 ? 1u : 0u);
+        }
+        mma_commit(st_full);
+        // dP^T = V_j dO_i^T, into columns the dQ warps must have emptied.
+        if (it >= 1 && !mbar_wait(dq_free, (it - 1) & 1, abort_flag)) { ok = false; break; }
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * PANEL_BYTES + (kk & 3) * 32;
+          mma_bf16_ss(tdPt, sdesc_kmajor_sw128(v_addr + off), sdesc_kmajor_sw128(do_addr + off),
+                      IDESC_SS, kk > 0 ? 1u : 0u);
+        }
+        mma_commit(dpt_full);
+        // P^T, dS^T (tensor memory) and dS (shared memory) are ready.
+        if (!mbar_wait(pds_full, it & 1, abort_flag)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t acc = it > 0 ? 1u : 0u;
+#pragma unroll
+        for (int kk = 0; kk < BLOCK / 16; ++kk)  // dV += P^T dO_i
+          mma_bf16_ts(tdV, tSt + kk * 8, sdesc_mnmajor_sw128(do_addr + kk * 2048, PANEL_BYTES),
+                      IDESC_ACC, (acc | kk) ? 1u : 0u);
+#pragma unroll
+        for (int kk = 0; kk < BLOCK / 16; ++kk)  // dK += dS^T Q_i
+          mma_bf16_ts(tdK, tdPt + kk * 8, sdesc_mnmajor_sw128(q_addr + kk * 2048, PANEL_BYTES),
+                      IDESC_ACC, (acc | kk) ? 1u : 0u);
+#pragma unroll
+        for (int kk = 0; kk < BLOCK / 16; ++kk)  // dQ_i = dS K_j (M = queries, K = keys)
+          mma_bf16_ss(tdPt, sdesc_mnmajor_sw128(ds_addr + kk * 2048, PANEL_BYTES),
+                      sdesc_mnmajor_sw128(k_addr + kk * 2048, PANEL_BYTES), IDESC_DQ,
+                      kk > 0 ? 1u : 0u);
+        mma_commit(dq_full);
+        mma_commit(&qd_empty[st]);
+      }
+      if (ok) mma_commit(dkv_final);
+      mma_commit(mma_final);
+      mbar_wait_drain(mma_final, 0);
+    }
+  } else if (warp < 4) {
+    // ------------------------------------------------------------ P^T / dS^T
+    const int t = threadIdx.x;  // key row
+    const int key_g = key0 + t;
+    const bool key_ok = key_g < p.N;
+    const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
+    const float sl2 = p.scale_log2;
+    uint8_t* ds_row = smem + L::DS_OFF + t * 128;  // row t of each 64-query panel
+    const uint32_t sw = static_cast<uint32_t>(t & 7);
+    bool ok = true;
+    for (int it = 0; it < n_it; ++it) {
+      const int st = it & 1;
+      const int q0 = (i_begin + it) * BLOCK;
+      if (!mbar_wait_warp(st_full, it & 1, abort_flag) ||
+          !mbar_wait_warp(dpt_full, it & 1, abort_flag)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      const float* lse_s = reinterpret_cast<const float*>(smem + L::LSE_OFF + st * 512);
+      const float* dd_s = reinterpret_cast<const float*>(smem + L::DD_OFF + st * 512);
+      // Queries at or beyond N carry log2(e) * LSE = +inf in the padded table,
+      // so their P is exactly 0; causal also drops queries before the key.
+      const bool diag = CAUSAL && (q0 == key0);
+#pragma unroll 1
+      for (int c = 0; c < BLOCK; c += 32) {
+        uint32_t sr[32], dr[32];
+        tmem_ld32(tSt + lane_off + c, sr);
+        tmem_ld32(tdPt + lane_off + c, dr);
+        tmem_ld_wait();
+        uint32_t pk[16], dk[16];
+#pragma unroll
+        for (int e = 0; e < 32; e += 2) {
+          float pv[2], dv[2];
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            const int q = c + e + h;
+            const float x = fmaf(__uint_as_float(sr[e + h]), sl2, -lse_s[q]);
+            float pp = ex2_approx(x);
+            bool keep = key_ok;
+            if (diag) keep = keep && (q >= t);
+            pp = keep ? pp : 0.f;
+            pv[h] = pp;
+            dv[h] = pp * (__uint_as_float(dr[e + h]) - dd_s[q]);
+          }
+          pk[e >> 1] = pack_bf16x2(pv[0], pv[1]);
+          dk[e >> 1] = pack_bf16x2(dv[0], dv[1]);
+        }
+        tmem_st16(tSt + lane_off + (c >> 1), pk);
+        tmem_st16(tdPt + lane_off + (c >> 1), dk);
+        // dS row t, queries c..c+31: panel c/64, 16-byte chunks (c%64)/8 .. +3,
+        // 128-byte swizzle (chunk index xor row % 8).
+        uint8_t* prow = ds_row + (c >> 6) * PANEL_BYTES;
+        const uint32_t ch0 = static_cast<uint32_t>((c & 63) >> 3);
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const uint32_t ch = (ch0 + u) ^ sw;
+          *reinterpret_cast<uint4*>(prow + ch * 16) =
+              make_uint4(dk[4 * u], dk[4 * u + 1], dk[4 * u + 2], dk[4 * u + 3]);
+        }
+      }
+      fence_proxy_async_smem();
+      tmem_st_wait();
+      tc_fence_before();
+      mbar_arrive(pds_full);
+    }
+    // epilogue: dV and scale * dK, one key row per thread
+    if (ok && mbar_wait_warp(dkv_final, 0, abort_flag)) {
+      tc_fence_after();
+      const size_t rowoff = (static_cast<size_t>(bh) * p.N + key_g) * D;
+#pragma unroll 1
+      for (int which = 0; which < 2; ++which) {
+        const uint32_t tacc = which == 0 ? tdV : tdK;
+        const float mul = which == 0 ? 1.f : p.scale;
+        __nv_bfloat16* dst_row = (which == 0 ? p.dv : p.dk) + rowoff;
+#pragma unroll
+        for (int c = 0; c < D; c += 32) {
+          uint32_t r[32];
+          tmem_ld32(tacc + lane_off + c, r);
+          tmem_ld_wait();
+          uint32_t pk[16];
+#pragma unroll
+          for (int e = 0; e < 32; e += 2)
+            pk[e >> 1] = pack_bf16x2(__uint_as_float(r[e]) * mul, __uint_as_float(r[e + 1]) * mul);
+          if (key_ok) {
+            uint4* dst = reinterpret_cast<uint4*>(dst_row + c);
+#pragma unroll
+            for (int v4 = 0; v4 < 4; ++v4)
+              dst[v4] = make_uint4(pk[4 * v4], pk[4 * v4 + 1], pk[4 * v4 + 2], pk[4 * v4 + 3]);
+          }
+        }
+      }
+    }
+    tmem_ld_wait();
+    tmem_st_wait();
+  } else {
+    // ------------------------------------------------------------ dQ reduction
+    const int t = threadIdx.x - 128;  // query row of the dQ tile, TMEM lane
+    const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
+    for (int it = 0; it < n_it; ++it) {
+      const int q_g = (i_begin + it) * BLOCK + t;
+      if (!mbar_wait_warp(dq_full, it & 1, abort_flag)) break;
+      tc_fence_after();
+      float* dst = p.dqacc + (static_cast<size_t>(bh) * p.N + q_g) * D;
+#pragma unroll 1
+      for (int c = 0; c < D; c += 32) {
+        uint32_t r[32];
+        tmem_ld32(tdPt + lane_off + c, r);
+        tmem_ld_wait();
+        if (q_g < p.N) {
+#pragma unroll
+          for (int v4 = 0; v4 < 8; ++v4)
+            red_add_v4(dst + c + 4 * v4, __uint_as_float(r[4 * v4]), __uint_as_float(r[4 * v4 + 1]),
+                       __uint_as_float(r[4 * v4 + 2]), __uint_as_float(r[4 * v4 + 3]));
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(dq_free);
+    }
+    tmem_ld_wait();
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 9) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem_base, TMEM_COLS);
+  }
+}
+
+// For every padded row (bh, n), n < Np: D = sum_k dO_k O_k and
+// lse2 = log2(e) * LSE when n < N, else D = 0 and lse2 = +inf; and dQacc = 0.
+template <int D>
+__global__ void __launch_bounds__(256)
+    fa_bwd_preprocess_kernel(const __nv_bfloat16* __restrict__ o,
+                             const __nv_bfloat16* __restrict__ dout,
+                             const float* __restrict__ lse, float* __restrict__ dd,
+                             float* __restrict__ lse2, float* __restrict__ dqacc, int N, int Np,
+                             long long padded_rows) {
+  constexpr int LPR = D / 8;     // lanes per row, 16 bytes each
+  constexpr int RPW = 32 / LPR;  // rows per warp
+  const int lane = threadIdx.x & 31;
+  const long long warp_g = (static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  const long long prow = warp_g * RPW + lane / LPR;
+  const int sub = lane % LPR;
+  const long long bh = prow / Np;
+  const int n = static_cast<int>(prow - bh * Np);
+  const bool real = prow < padded_rows && n < N;
+  const long long row = bh * N + n;
+  float acc = 0.f;
+  if (real) {
+    const uint4 a = *reinterpret_cast<const uint4*>(o + row * D + sub * 8);
+    const uint4 b = *reinterpret_cast<const uint4*>(dout + row * D + sub * 8);
+    const uint32_t wa[4] = {a.x, a.y, a.z, a.w}, wb[4] = {b.x, b.y, b.z, b.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      acc = fmaf(__uint_as_float(wa[i] << 16), __uint_as_float(wb[i] << 16), acc);
+      acc = fmaf(__uint_as_float(wa[i] & 0xFFFF0000u), __uint_as_float(wb[i] & 0xFFFF0000u), acc);
+    }
+    float4* z = reinterpret_cast<float4*>(dqacc + row * D + sub * 8);
+    z[0] = make_float4(0.f, 0.f, 0.f, 0.f);
+    z[1] = make_float4(0.f, 0.f, 0.f, 0.f);
+  }
+#pragma unroll
+  for (int off = LPR / 2; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+  if (prow < padded_rows && sub == 0) {
+    dd[prow] = real ? acc : 0.f;
+    lse2[prow] = real ? lse[row] * LOG2E : INFINITY;
+  }
+}
+
+// dQ = scale * dQacc in bf16, 8 elements per thread.
+__global__ void __launch_bounds__(256)
+    fa_bwd_dq_convert_kernel(const float* __restrict__ dqacc, __nv_bfloat16* __restrict__ dq,
+                             long long n8, float scale) {
+  const long long i = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (i >= n8) return;
+  const float4 a = reinterpret_cast<const float4*>(dqacc)[2 * i];
+  const float4 b = reinterpret_cast<const float4*>(dqacc)[2 * i + 1];
+  reinterpret_cast<uint4*>(dq)[i] =
+      make_uint4(pack_bf16x2(a.x * scale, a.y * scale), pack_bf16x2(a.z * scale, a.w * scale),
+                 pack_bf16x2(b.x * scale, b.y * scale), pack_bf16x2(b.z * scale, b.w * scale));
+}
+
+template <int D, bool CAUSAL>
+fa_status launch_main(const CUtensorMap* maps, const Params& prm, int BH, cudaStream_t stream) {
+  auto kern = fa_bwd_kernel<D, CAUSAL>;
+  static bool configured = false;
+  if (!configured) {
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Smem<D>::ALLOC) !=
+        cudaSuccess)
+      return FA_ERR_CUDA;
+    configured = true;
+  }
+  dim3 grid(BH, prm.n_tiles);
+  kern<<<grid, NUM_THREADS, Smem<D>::ALLOC, stream>>>(maps[0], maps[1], maps[2], maps[3], maps[4],
+                                                      maps[5], prm);
+  return cuda_status(cudaGetLastError());
+}
+
+}  // namespace bwd
+
+fa_status launch_bwd(const void* q, const void* k, const void* v, const void* o,
+                     const void* dout, const float* lse, void* dq, void* dk, void* dv,
+                     void* workspace, int B, int H, int N, int d, int causal, float scale,
+                     cudaStream_t stream) {
+  const int BH = B * H;
+  const long long rows = static_cast<long long>(BH) * N;
+  const int Np = static_cast<int>(bwd_row_pad(N));
+  const long long prows = static_cast<long long>(BH) * Np;
+  const size_t table = align_up(static_cast<size_t>(prows) * 4, 256);
+  float* dd = static_cast<float*>(workspace);
+  float* lse2 = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + table);
+  float* dqacc = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + 2 * table);
+  // 1. D, log2(e) * LSE (padded tables) and the zeroed accumulator
+  {
+    const int rows_per_block = (256 / 32) * (32 / (d / 8));
+    const long long blocks = (prows + rows_per_block - 1) / rows_per_block;
+    if (d == 128)
+      bwd::fa_bwd_preprocess_kernel<128><<<static_cast<unsigned>(blocks), 256, 0, stream>>>(
+          static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(dout), lse, dd,
+          lse2, dqacc, N, Np, prows);
+    else
+      bwd::fa_bwd_preprocess_kernel<64><<<static_cast<unsigned>(blocks), 256, 0, stream>>>(
+          static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(dout), lse, dd,
+          lse2, dqacc, N, Np, prows);
+    if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
+  }
+  // 2. dK, dV and the dQ accumulation
+  CUtensorMap maps[6];
+  fa_status st;
+  if ((st = make_tmap_bf16_3d(&maps[0], q, d, N, BH, bwd::BLOCK)) != FA_OK) return st;
+  if ((st = make_tmap_bf16_3d(&maps[1], k, d, N, BH, bwd::BLOCK)) != FA_OK) return st;
+  if ((st = make_tmap_bf16_3d(&maps[2], v, d, N, BH, bwd::BLOCK)) != FA_OK) return st;
+  if ((st = make_tmap_bf16_3d(&maps[3], dout, d, N, BH, bwd::BLOCK)) != FA_OK) return st;
+  if ((st = make_tmap_f32_2d(&maps[4], lse2, Np, BH)) != FA_OK) return st;
+  if ((st = make_tmap_f32_2d(&maps[5], dd, Np, BH)) != FA_OK) return st;
+  bwd::Params prm;
+  prm.dk = static_cast<__nv_bfloat16*>(dk);
+  prm.dv = static_cast<__nv_bfloat16*>(dv);
+  prm.dqacc = dqacc;
+  prm.N = N;
+  prm.n_tiles = (N + bwd::BLOCK - 1) / bwd::BLOCK;
+  prm.scale_log2 = scale * bwd::LOG2E;
+  prm.scale = scale;
+  if (d == 128)
+    st = causal ? bwd::launch_main<128, true>(maps, prm, BH, stream)
+                : bwd::launch_main<128, false>(maps, prm, BH, stream);
+  else
+    st = causal ? bwd::launch_main<64, true>(maps, prm, BH, stream)
+                : bwd::launch_main<64, false>(maps, prm, BH, stream);
+  if (st != FA_OK) return st;
+  // 3. dQ = scale * accumulator
+  {
+    const long long n8 = rows * d / 8;
+    const long long blocks = (n8 + 255) / 256;
+    bwd::fa_bwd_dq_convert_kernel<<<static_cast<unsigned>(blocks), 256, 0, stream>>>(
+        dqacc, static_cast<__nv_bfloat16*>(dq), n8, scale);
+    if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
+  }
+  return FA_OK;
 }
 
 }  // namespace fa

@@ -18,6 +18,14 @@ namespace fa {
 fa_status make_tmap_bf16_3d(CUtensorMap* map, const void* base, uint64_t d, uint64_t rows,
                             uint64_t outer, uint32_t box_rows);
 
+// 2-D float32 tensor map over a [outer, n] array with a 128 x 1 box and no
+// swizzle; n * 4 must be a multiple of 16 bytes.
+fa_status make_tmap_f32_2d(CUtensorMap* map, const void* base, uint64_t n, uint64_t outer);
+
+// Row stride (elements) of the per-row float32 tables of the backward
+// workspace: N rounded up to whole 128-row tiles.
+inline size_t bwd_row_pad(int N) { return (static_cast<size_t>(N) + 127) / 128 * 128; }
+
 fa_status launch_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B,
                      int H, int N, int d, int causal, float scale, cudaStream_t stream);
 

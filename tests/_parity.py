@@ -52,18 +52,3 @@ def check_grad(got, ref, what):
     assert rl <= GRAD_REL_L2, f"{what}: relative L2 error {rl:.3e} > {GRAD_REL_L2}"
     return rl
 
-
-def check_o_scaled(got, ref, what="O"):
-    """For deliberately peaked softmax rows, where |O| reaches |v| ~ 4: the
-    bf16 output alone rounds by up to 2^-8 |O| (0.0156 at |O| = 4), and the
-    bf16 P fed to the tensor core adds about as much again.  Bound:
-    |err| <= 1e-2 * max(1, |ref| / 2) elementwise, i.e. the spec tolerance
-    for |O| <= 2 and 0.5 % relative above it.  The relative L2 criterion is
-    unchanged."""
-    g, r = as_f64(got), as_f64(ref)
-    assert np.isfinite(g).all(), f"{what}: non-finite values"
-    bound = O_MAX_ABS * np.maximum(1.0, np.abs(r) / 2.0)
-    worst = float(np.max(np.abs(g - r) / bound))
-    assert worst <= 1.0, f"{what}: error exceeds the magnitude-scaled bound by {worst:.3f}x"
-    rl = rel_l2(g, r)
-    assert rl <= O_REL_L2, f"{what}: relative L2 error {rl:.3e} > {O_REL_L2}"

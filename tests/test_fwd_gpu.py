@@ -5,7 +5,7 @@ import torch
 
 import oracle
 from io_aware_exact_35_b200 import inputs
-from tests._parity import check_lse, check_o, check_o_scaled
+from tests._parity import check_lse, check_o
 
 pytestmark = pytest.mark.gpu
 
@@ -39,16 +39,21 @@ def test_fwd_small_shapes(fa_mod, cuda_device, shape, causal):
 
 
 def test_fwd_large_scores_and_rescaling(fa_mod, cuda_device):
-    # Scores spanning a wide range force the running maximum to move often.
+    """Keys ramped from 0.1x to 4x make every row's running maximum grow by far
+    more than the 2^8 rescale threshold across the key tiles, so O and l are
+    rescaled many times.  The rows end up dominated by a few keys; V is scaled
+    by 1/4 so that |O| stays below 1 and bf16 rounding of P and of O (2^-9
+    relative each) stays inside the absolute tolerance."""
     B, H, N, d = 1, 2, 777, 128
     q, k, v = inputs.fwd_inputs(B, H, N, d, seed=7, std=1.0)
     ramp = torch.linspace(0.1, 4.0, N).view(1, 1, N, 1)
     k = (k.float() * ramp).to(torch.bfloat16)
+    v = (v.float() * 0.25).to(torch.bfloat16)
     for causal in (False, True):
         o, lse = _run(fa_mod, q, k, v, causal, 0.3)
         o_ref, lse_ref = oracle.attention_forward(inputs.to_f64(q), inputs.to_f64(k),
                                                   inputs.to_f64(v), causal, 0.3)
-        check_o_scaled(o, o_ref)
+        check_o(o, o_ref)
         check_lse(lse, lse_ref)
 
 
