@@ -364,9 +364,15 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(inputs.WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--no-extra", action="store_true", help="skip the other workloads' lines")
+    ap.add_argument("--skip-baselines", action="store_true",
+                    help="profiling runs: skip the end-to-end and CPU-oracle legs")
+    ap.add_argument("--B", type=int, default=None,
+                    help="profiling runs: override the workload's batch size")
     args = ap.parse_args()
     w = inputs.WORKLOADS[args.workload]
+    if args.B is not None:
+        import dataclasses
+        w = dataclasses.replace(w, B=args.B, name=f"{w.name}[B={args.B}]")
     default_steps = {"fwd": 4000, "bwd": 300, "decode": 800}[w.kind]
     if w.name == "fwd_causal_B1_H32_N32768_d128":
         default_steps = 200
@@ -393,7 +399,10 @@ def main():
 
     r = Runner(w, dev)
     mean_s, per, wall, clocks = time_device(r, args.steps, args.warmup, world, dev)
-    e2e_s, h2d, d2h = time_e2e(r, max(3, min(args.steps, 50)), 2, world, dev)
+    if args.skip_baselines:
+        e2e_s, h2d, d2h = float("nan"), 0, 0
+    else:
+        e2e_s, h2d, d2h = time_e2e(r, max(3, min(args.steps, 50)), 2, world, dev)
     err = fa.get_device_error()
     peaks, peak_src = load_peaks()
     value = r.value(mean_s) * world
@@ -428,7 +437,7 @@ def main():
         "device_error": err,
         "wall_s_timed_region": wall,
     }
-    if rank == 0 and world == 1:
+    if rank == 0 and world == 1 and not args.skip_baselines:
         try:
             line["cpu_baseline"] = cpu_baseline(w)
         except Exception as e:  # the baseline is reported, not required
