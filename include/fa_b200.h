@@ -130,6 +130,35 @@ fa_status fa_decode(const void* q, const void* kcache, const void* vcache,
                     void* workspace, size_t ws_bytes, fa_stream_t stream);
 
 /*
+ * Size in bytes of the device array that fa_decode_static uses as scratch
+ * (16 MiB, held by every device that loads the library until exit).
+ */
+#define FA_DECODE_STATIC_SCRATCH_BYTES (16u * 1024u * 1024u)
+
+/*
+ * fa_decode without a caller-provided workspace, for callers that cannot
+ * call cudaMalloc (a plug-in whose host program owns nearly all device memory
+ * through its own pool, or a latency-critical loop that must not trigger the
+ * device-wide synchronisation an allocation can cause).  The pages have no
+ * counterpart: this is an interface convenience, not part of the method.
+ *   Arguments, layouts, ownership and results are those of fa_decode, minus
+ *   workspace / ws_bytes.  The split-KV partials go to a library-owned device
+ *   array of FA_DECODE_STATIC_SCRATCH_BYTES bytes; a problem whose
+ *   fa_decode_workspace_size(B, H, Lmax, d) exceeds that returns
+ *   FA_ERR_WORKSPACE before any launch.  Allocates nothing.
+ *   The first call on a device looks up the array's device address (with
+ *   that device current); make it before any stream capture.  All calls
+ *   share the array: calls that overlap on the GPU race and must be
+ *   serialised by the caller.
+ * Returns FA_OK, FA_ERR_INVALID_ARG, FA_ERR_UNSUPPORTED, FA_ERR_WORKSPACE or
+ * FA_ERR_CUDA.
+ */
+fa_status fa_decode_static(const void* q, const void* kcache, const void* vcache,
+                           const int* seqlens, void* o, float* lse,
+                           int B, int H, int Lmax, int d, float scale,
+                           fa_stream_t stream);
+
+/*
  * Synchronises `stream`, then reads and clears the current device's error
  * word.  Returns FA_OK, FA_ERR_TIMEOUT (a kernel gave up a bounded wait and
  * returned without finishing) or FA_ERR_CUDA (the synchronisation failed).

@@ -5,3 +5,4 @@
 #include "fa_fwd.cu"
 #include "fa_bwd.cu"
 #include "fa_decode.cu"
+#include "fa_decode_static.cu"

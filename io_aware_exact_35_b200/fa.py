@@ -31,6 +31,7 @@ SIGNATURES = {
     "fa_bwd": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _S, _I, _I, _I, _I, _I, _F, _P]),
     "fa_decode_workspace_size": (_S, [_I, _I, _I, _I]),
     "fa_decode": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _F, _P, _S, _P]),
+    "fa_decode_static": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _F, _P]),
     "fa_get_device_error": (_I, [_P]),
     "fa_status_string": (ctypes.c_char_p, [_I]),
     "fa_version": (_I, []),
@@ -184,6 +185,40 @@ def decode(q, kcache, vcache, seqlens, scale: Optional[float] = None, out=None, 
                          workspace.data_ptr(), workspace.numel() * workspace.element_size(),
                          _stream_ptr(stream))
     _check("fa_decode", st)
+    return out, lse
+
+
+# Bytes of the library-owned scratch array behind fa_decode_static.
+DECODE_STATIC_SCRATCH_BYTES = 16 * 1024 * 1024
+
+
+def decode_static(q, kcache, vcache, seqlens, scale: Optional[float] = None, out=None,
+                  lse=None, want_lse: bool = True, stream=None):
+    """Split-KV decode that allocates nothing: the library keeps the scratch in
+    a fixed device array (see fa_decode_static in include/fa_b200.h).  For
+    callers that cannot allocate device memory, e.g. inside a host program
+    that owns all of it.  Outputs must be passed in (or are created here by
+    torch when omitted, which is an allocation of the caller's own).  Calls
+    that overlap on the GPU share the scratch and race."""
+    _req(q, "q", torch.bfloat16, 3)
+    _req(kcache, "kcache", torch.bfloat16, 4)
+    _req(vcache, "vcache", torch.bfloat16, 4)
+    _req(seqlens, "seqlens", torch.int32, 1)
+    B, H, d = q.shape
+    Lmax = kcache.shape[2]
+    if tuple(kcache.shape) != (B, H, Lmax, d) or vcache.shape != kcache.shape:
+        raise ValueError("caches must be [B, H, Lmax, d] matching q")
+    if seqlens.shape[0] != B:
+        raise ValueError("seqlens must have B entries")
+    scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
+    out = torch.empty_like(q) if out is None else out
+    _req(out, "out", torch.bfloat16, 3)
+    if lse is None and want_lse:
+        lse = torch.empty((B, H), dtype=torch.float32, device=q.device)
+    st = lib().fa_decode_static(q.data_ptr(), kcache.data_ptr(), vcache.data_ptr(),
+                                seqlens.data_ptr(), out.data_ptr(), _ptr(lse), B, H, Lmax, d,
+                                scale, _stream_ptr(stream))
+    _check("fa_decode_static", st)
     return out, lse
 
 
