@@ -52,16 +52,25 @@ def load_peaks():
     return dict(FALLBACK_PEAKS), "fallback"
 
 
-def kernel_sources_sha():
+KERNEL_SOURCES = {
+    "fwd": ("fa_fwd.cu", "sm100.cuh"),
+    "bwd": ("fa_bwd.cu", "sm100.cuh"),
+    "decode": ("fa_decode.cu", "sm100.cuh"),
+}
+
+
+def kernel_sources_sha(kind):
+    """Hash of the source files a kernel is built from (traffic figures taken
+    by ncu are only reported while this hash still matches)."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "io_aware_exact_35_b200", "csrc")
-    for name in sorted(os.listdir(csrc)):
+    for name in KERNEL_SOURCES[kind]:
         with open(os.path.join(csrc, name), "rb") as f:
             h.update(name.encode() + f.read())
     return h.hexdigest()[:16]
 
 
-def profiled_traffic(kernel_key):
+def profiled_traffic(kernel_key, kind):
     """DRAM bytes per launch from the committed ncu summary, if still current."""
     path = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(path):
@@ -69,7 +78,7 @@ def profiled_traffic(kernel_key):
     with open(path) as f:
         d = json.load(f)
     ent = d.get(kernel_key)
-    if not ent or ent.get("source_sha") != kernel_sources_sha():
+    if not ent or ent.get("source_sha") != kernel_sources_sha(kind):
         return None
     return ent.get("dram_bytes_per_launch")
 
@@ -409,14 +418,14 @@ def main():
     if r.kind_bound == "tensor":
         peak = float(peaks["bf16_tflops"])
         ach = r.work / mean_s / 1e12
-        traffic = profiled_traffic(r.kernel_key)
+        traffic = profiled_traffic(r.kernel_key, r.w.kind)
         roof = {"bound": "tensor", "achieved": ach, "peak": peak, "unit": "TFLOP/s",
                 "frac": ach / peak, "traffic": traffic,
                 "peak_source": f"{peak_src} bf16_tflops (burst)"}
     else:
         peak = float(peaks["hbm_gbs"])
         ach = r.work / mean_s / 1e9
-        traffic = profiled_traffic(r.kernel_key)
+        traffic = profiled_traffic(r.kernel_key, r.w.kind)
         roof = {"bound": "hbm", "achieved": ach, "peak": peak, "unit": "GB/s",
                 "frac": ach / peak, "traffic": traffic,
                 "peak_source": f"{peak_src} hbm_gbs"}
