@@ -57,7 +57,7 @@ bool aligned256(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 255u) 
 fa_status check_shape(int B, int H, int N, int d) {
   if (B < 1 || H < 1 || N < 0) return FA_ERR_INVALID_ARG;
   if (static_cast<long long>(B) * H > INT_MAX) return FA_ERR_INVALID_ARG;
-  if ((static_cast<long long>(N) + 127) / 128 > 65535) return FA_ERR_INVALID_ARG;
+  if ((static_cast<long long>(N) + 127) / 128 * B * H > 0x7fffffffLL) return FA_ERR_INVALID_ARG;
   if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
   return FA_OK;
 }

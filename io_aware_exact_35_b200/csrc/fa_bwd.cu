@@ -121,8 +121,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int bh = blockIdx.x;
-  const int kv_tile = blockIdx.y;  // tile 0 sees the most query tiles: launched first
+  // One-dimensional grid, head-major: the key tiles of one (batch, head) are
+  // adjacent in launch order (so resident CTAs share that head's Q and dO
+  // tiles in L2); tile 0, which sees the most query tiles, comes first.
+  const int bh = static_cast<int>(blockIdx.x) / p.n_tiles;
+  const int kv_tile = static_cast<int>(blockIdx.x) - bh * p.n_tiles;
   const int key0 = kv_tile * BLOCK;
   const int i_begin = CAUSAL ? kv_tile : 0;
   const int n_it = p.n_tiles - i_begin;
@@ -431,7 +434,7 @@ fa_status launch_main(const CUtensorMap* maps, const Params& prm, int BH, cudaSt
       return FA_ERR_CUDA;
     configured = true;
   }
-  dim3 grid(BH, prm.n_tiles);
+  dim3 grid(prm.n_tiles * BH);
   kern<<<grid, NUM_THREADS, Smem<D>::ALLOC, stream>>>(maps[0], maps[1], maps[2], maps[3], maps[4],
                                                       maps[5], prm);
   return cuda_status(cudaGetLastError());

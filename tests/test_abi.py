@@ -68,7 +68,7 @@ def test_host_validation_rejects_bad_arguments(fa_mod):
     assert lib.fa_fwd(P, P, P, P, None, 1, 1, 8, 64, 2, 1.0, None) == INVALID
     assert lib.fa_fwd(P, P, P, P, None, 1, 1, 8, 64, 0, float("nan"), None) == INVALID
     assert lib.fa_fwd(P, P, P, P, None, 1, 1, 8, 96, 0, 1.0, None) == UNSUPPORTED
-    assert lib.fa_fwd(P, P, P, P, None, 1, 1, 128 * 65536, 64, 0, 1.0, None) == INVALID
+    assert lib.fa_fwd(P, P, P, P, None, 1024, 1024, 1 << 20, 64, 0, 1.0, None) == INVALID
     # backward: workspace checks
     args = [P] * 6 + [P, P, P]
     assert lib.fa_bwd(*args, None, 0, 1, 1, 8, 64, 0, 1.0, None) == WORKSPACE
