@@ -35,6 +35,10 @@
 // and O and l are only rescaled (a tensor-memory round trip) when the maximum
 // really moves.  Both l and O always refer to the same maximum, so the final
 // O / l is unchanged.
+#include <algorithm>
+#include <cstdlib>
+#include <cstring>
+
 #include "fa_internal.h"
 #include "sm100.cuh"
 
@@ -50,6 +54,10 @@ constexpr int NUM_THREADS = 320;
 constexpr int PANEL_BYTES = 128 * 128;   // 128 rows x 64 bf16 (one swizzle panel)
 constexpr uint32_t TMEM_COLS = 512;
 constexpr float RESCALE_THRESHOLD = 8.0f;  // log2 units
+#ifndef FA_FWD_EMU_PAIRS
+#define FA_FWD_EMU_PAIRS 0
+#endif
+constexpr int EMU_PAIRS = FA_FWD_EMU_PAIRS;  // of every 4 exp pairs, on the FMA pipe
 
 template <int D>
 struct Smem {
@@ -60,9 +68,9 @@ struct Smem {
   static constexpr int K_OFF = NQ * TILE;
   static constexpr int V_OFF = K_OFF + NS * TILE;
   static constexpr int BAR_OFF = V_OFF + NS * TILE;
-  // barriers: q_full, k_full[NS], v_full[NS], k_empty[NS], v_empty[NS],
-  //           s_full[NQ], p_full[NQ], o_done[NQ], o_final[NQ], mma_final
-  static constexpr int NBAR = 1 + 4 * NS + 4 * NQ + 1;
+  // barriers: q_full, q_empty, k_full[NS], v_full[NS], k_empty[NS], v_empty[NS],
+  //           s_full[NQ], p_full[NQ], o_done[NQ], o_final[NQ], o_free[NQ], mma_final
+  static constexpr int NBAR = 2 + 4 * NS + 5 * NQ + 1;
   static constexpr int MISC_OFF = BAR_OFF + NBAR * 8;
   static constexpr int BYTES = MISC_OFF + 16;
   // at least 116 KB so that a single CTA (and its 512 tensor-memory columns)
@@ -74,9 +82,33 @@ struct Params {
   __nv_bfloat16* o;
   float* lse;
   int N;
+  int BH;
   int n_cta_tiles;   // ceil(N / 256)
+  int total_items;   // BH * n_cta_tiles
+  int lpt_order;     // 1: all heads' longest tiles first; 0: head-major
   float scale_log2;  // scale * log2(e)
 };
+
+// Work item -> (batch*head, 256-row tile).  In LPT order the longest tiles of
+// every head come first (good balance; used when all K/V fit in L2); in
+// head-major order the tiles of one head are adjacent, longest first (K/V of
+// the resident CTAs stay in L2 for long sequences).
+__device__ __forceinline__ void item_coords(const Params& p, int item, int& bh, int& tile) {
+  if (p.lpt_order) {
+    const int r = item / p.BH;
+    bh = item - r * p.BH;
+    tile = p.n_cta_tiles - 1 - r;
+  } else {
+    bh = item / p.n_cta_tiles;
+    tile = p.n_cta_tiles - 1 - (item - bh * p.n_cta_tiles);
+  }
+}
+
+// The k-th work item of CTA c out of G: rounds alternate direction so that a
+// CTA that drew a long item in one round draws a short one in the next.
+__device__ __forceinline__ int cta_item(int c, int k, int G) {
+  return k * G + ((k & 1) ? (G - 1 - c) : c);
+}
 
 template <int D, bool CAUSAL>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
@@ -95,32 +127,34 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::BAR_OFF);
   uint64_t* q_full = bars;
-  uint64_t* k_full = bars + 1;
+  uint64_t* q_empty = bars + 1;
+  uint64_t* k_full = bars + 2;
   uint64_t* v_full = k_full + NS;
   uint64_t* k_empty = v_full + NS;
   uint64_t* v_empty = k_empty + NS;
   uint64_t* s_full = v_empty + NS;  // [NQ]
   uint64_t* p_full = s_full + NQ;   // [NQ]
   uint64_t* o_done = p_full + NQ;   // [NQ] one phase per O += P V
-  uint64_t* o_final = o_done + NQ;  // [NQ] the last O += P V of the tile
-  uint64_t* mma_final = o_final + NQ;
+  uint64_t* o_final = o_done + NQ;  // [NQ] one phase per work item: its last O += P V
+  uint64_t* o_free = o_final + NQ;  // [NQ] one phase per work item: O read out
+  uint64_t* mma_final = o_free + NQ;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::MISC_OFF);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::MISC_OFF + 4);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  // One-dimensional grid, head-major: the 256-row tiles of one (batch, head)
-  // are adjacent in launch order, longest (last) tile first.
-  const int bh = static_cast<int>(blockIdx.x) / p.n_cta_tiles;
-  const int cta_tile = p.n_cta_tiles - 1 - (static_cast<int>(blockIdx.x) - bh * p.n_cta_tiles);
-  const int row_base = cta_tile * BLOCK_M;
+  const int G = static_cast<int>(gridDim.x);
+  const int cta = static_cast<int>(blockIdx.x);
   const int n_kv_total = (p.N + BLOCK_N - 1) / BLOCK_N;
-  // key tiles seen by query tile w (causal: up to its own diagonal tile)
-  const int n_kv0 = CAUSAL ? min(2 * cta_tile + 1, n_kv_total) : n_kv_total;
-  const int n_kv1 = CAUSAL ? min(2 * cta_tile + 2, n_kv_total) : n_kv_total;
+  // key tiles seen by query tile w of 256-row tile `tile` (causal: up to its
+  // own diagonal tile)
+  auto n_kv_of = [&](int tile, int w) {
+    return CAUSAL ? min(2 * tile + 1 + w, n_kv_total) : n_kv_total;
+  };
 
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
+    mbar_init(q_empty, 1);
     for (int s = 0; s < NS; ++s) {
       mbar_init(&k_full[s], 1);
       mbar_init(&v_full[s], 1);
@@ -132,6 +166,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       mbar_init(&p_full[w], TILE_M);
       mbar_init(&o_done[w], 1);
       mbar_init(&o_final[w], 1);
+      mbar_init(&o_free[w], TILE_M);
     }
     mbar_init(mma_final, 1);
     *abort_flag = 0;
@@ -154,34 +189,49 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   if (warp == 8) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
-      int last_k[NS], last_v[NS];
-      for (int s = 0; s < NS; ++s) last_k[s] = last_v[s] = -1;
-      mbar_arrive_expect_tx(q_full, NQ * L::TILE);
-      for (int w = 0; w < NQ; ++w)
-        for (int pn = 0; pn < L::NPANEL; ++pn)
-          tma_load_3d(smem + L::Q_OFF + w * L::TILE + pn * PANEL_BYTES, &tm_q, q_full, pn * 64,
-                      row_base + w * TILE_M, bh);
-      for (int j = 0; j < n_kv1; ++j) {
-        const int st = j % NS;
-        const int r = j / NS;
-        if (j >= NS && !mbar_wait(&k_empty[st], (r - 1) & 1, abort_flag)) break;
-        mbar_arrive_expect_tx(&k_full[st], L::TILE);
-        for (int pn = 0; pn < L::NPANEL; ++pn)
-          tma_load_3d(smem + L::K_OFF + st * L::TILE + pn * PANEL_BYTES, &tm_k, &k_full[st],
-                      pn * 64, j * BLOCK_N, bh);
-        last_k[st] = r;
-        if (j >= NS && !mbar_wait(&v_empty[st], (r - 1) & 1, abort_flag)) break;
-        mbar_arrive_expect_tx(&v_full[st], L::TILE);
-        for (int pn = 0; pn < L::NPANEL; ++pn)
-          tma_load_3d(smem + L::V_OFF + st * L::TILE + pn * PANEL_BYTES, &tm_v, &v_full[st],
-                      pn * 64, j * BLOCK_N, bh);
-        last_v[st] = r;
+      int kv = 0;        // K/V tiles loaded so far (all work items)
+      int n_items = 0;   // Q pairs loaded so far
+      bool ok = true;
+      for (int k = 0; ok; ++k) {
+        const int item = cta_item(cta, k, G);
+        if (item >= p.total_items) break;
+        int bh, tile;
+        item_coords(p, item, bh, tile);
+        const int n_kv1 = n_kv_of(tile, 1);
+        // the Q pair of the previous item must have been consumed by its S MMAs
+        if (k > 0 && !mbar_wait(q_empty, (k - 1) & 1, abort_flag)) break;
+        mbar_arrive_expect_tx(q_full, NQ * L::TILE);
+        for (int w = 0; w < NQ; ++w)
+          for (int pn = 0; pn < L::NPANEL; ++pn)
+            tma_load_3d(smem + L::Q_OFF + w * L::TILE + pn * PANEL_BYTES, &tm_q, q_full,
+                        pn * 64, tile * BLOCK_M + w * TILE_M, bh);
+        ++n_items;
+        for (int j = 0; j < n_kv1; ++j, ++kv) {
+          const int st = kv % NS;
+          const int r = kv / NS;
+          if (kv >= NS && !mbar_wait(&k_empty[st], (r - 1) & 1, abort_flag)) { ok = false; break; }
+          mbar_arrive_expect_tx(&k_full[st], L::TILE);
+          for (int pn = 0; pn < L::NPANEL; ++pn)
+            tma_load_3d(smem + L::K_OFF + st * L::TILE + pn * PANEL_BYTES, &tm_k, &k_full[st],
+                        pn * 64, j * BLOCK_N, bh);
+          if (kv >= NS && !mbar_wait(&v_empty[st], (r - 1) & 1, abort_flag)) {
+            // K of this tile is in flight: count it so that it is drained
+            mbar_wait_drain(&k_full[st], r & 1);
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(&v_full[st], L::TILE);
+          for (int pn = 0; pn < L::NPANEL; ++pn)
+            tma_load_3d(smem + L::V_OFF + st * L::TILE + pn * PANEL_BYTES, &tm_v, &v_full[st],
+                        pn * 64, j * BLOCK_N, bh);
+        }
       }
-      // Every copy issued must land before this CTA's shared memory is freed.
-      mbar_wait_drain(q_full, 0);
-      for (int s = 0; s < NS; ++s) {
-        if (last_k[s] >= 0) mbar_wait_drain(&k_full[s], last_k[s] & 1);
-        if (last_v[s] >= 0) mbar_wait_drain(&v_full[s], last_v[s] & 1);
+      // Every copy issued must land before this CTA's shared memory is freed:
+      // the last phase of each barrier that received copies.
+      if (n_items > 0) mbar_wait_drain(q_full, (n_items - 1) & 1);
+      for (int g = max(0, kv - NS); g < kv; ++g) {
+        mbar_wait_drain(&k_full[g % NS], (g / NS) & 1);
+        mbar_wait_drain(&v_full[g % NS], (g / NS) & 1);
       }
     }
   } else if (warp == 9) {
@@ -192,11 +242,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       const uint32_t q_addr = smem_u32(smem + L::Q_OFF);
       const uint32_t k_addr = smem_u32(smem + L::K_OFF);
       const uint32_t v_addr = smem_u32(smem + L::V_OFF);
-      const int n_kv[NQ] = {n_kv0, n_kv1};
+      int pcount[NQ] = {0, 0};  // P tiles consumed per warpgroup (all items)
 
-      // S_w = Q_w K_j^T into S buffer w (K_j already resident)
-      auto issue_s = [&](int w, int j) {
-        const uint32_t kbase = k_addr + (j % NS) * L::TILE;
+      // S_w = Q_w K^T with K in ring slot `slot`
+      auto issue_s = [&](int w, int slot) {
+        const uint32_t kbase = k_addr + slot * L::TILE;
         const uint32_t qbase = q_addr + w * L::TILE;
         const uint32_t dS = tmem_base + w * 128;
 #pragma unroll
@@ -207,47 +257,67 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         }
         mma_commit(&s_full[w]);
       };
-      // O_w += P_w V_j once warpgroup w has written P_w (V_j already resident)
-      auto issue_pv = [&](int w, int j) -> bool {
-        if (!mbar_wait(&p_full[w], j & 1, abort_flag)) return false;
+      // O_w (+)= P_w V with V in ring slot `slot`, once warpgroup w wrote P_w
+      auto issue_pv = [&](int w, int slot, bool first, bool last) -> bool {
+        if (!mbar_wait(&p_full[w], pcount[w] & 1, abort_flag)) return false;
+        ++pcount[w];
         tc_fence_after();
-        const uint32_t vbase = v_addr + (j % NS) * L::TILE;
+        const uint32_t vbase = v_addr + slot * L::TILE;
         const uint32_t tP = tmem_base + w * 128;
         const uint32_t tO = tmem_base + 256 + w * 128;
 #pragma unroll
         for (int kk = 0; kk < BLOCK_N / 16; ++kk) {
           // keys 16kk .. 16kk+15: P columns 8kk.., V rows 16kk.. (2048 bytes per step)
           const uint64_t bdesc = sdesc_mnmajor_sw128(vbase + kk * 2048, PANEL_BYTES);
-          mma_bf16_ts(tO, tP + kk * 8, bdesc, IDESC_O, (j > 0 || kk > 0) ? 1u : 0u);
+          mma_bf16_ts(tO, tP + kk * 8, bdesc, IDESC_O, (!first || kk > 0) ? 1u : 0u);
         }
         mma_commit(&o_done[w]);
-        if (j == n_kv[w] - 1) mma_commit(&o_final[w]);
+        if (last) mma_commit(&o_final[w]);
         return true;
       };
 
-      bool ok = mbar_wait(q_full, 0, abort_flag) && mbar_wait(&k_full[0], 0, abort_flag);
-      if (ok) {
+      int kv = 0;  // K/V tiles consumed so far (all work items)
+      bool ok = true;
+      for (int k = 0; ok; ++k) {
+        const int item = cta_item(cta, k, G);
+        if (item >= p.total_items) break;
+        int bh, tile;
+        item_coords(p, item, bh, tile);
+        const int n0 = n_kv_of(tile, 0);
+        const int n1 = n_kv_of(tile, 1);
+        if (!mbar_wait(q_full, k & 1, abort_flag) ||
+            !mbar_wait(&k_full[kv % NS], (kv / NS) & 1, abort_flag)) { ok = false; break; }
         tc_fence_after();
-        issue_s(0, 0);
-        issue_s(1, 0);
-        mma_commit(&k_empty[0]);
-      }
-      for (int j = 0; ok && j < n_kv1; ++j) {
-        const int st = j % NS;
-        const bool more = j + 1 < n_kv1;
-        if (!mbar_wait(&v_full[st], (j / NS) & 1, abort_flag)) { ok = false; break; }
-        if (j < n_kv0 && !issue_pv(0, j)) { ok = false; break; }
-        if (more) {
-          if (!mbar_wait(&k_full[(j + 1) % NS], ((j + 1) / NS) & 1, abort_flag)) { ok = false; break; }
-          tc_fence_after();
-          if (j + 1 < n_kv0) issue_s(0, j + 1);
+        issue_s(0, kv % NS);
+        issue_s(1, kv % NS);
+        mma_commit(&k_empty[kv % NS]);
+        if (n1 == 1) mma_commit(q_empty);
+        for (int j = 0; j < n1; ++j) {
+          const int g = kv + j;
+          const int st = g % NS;
+          const bool more = j + 1 < n1;
+          if (!mbar_wait(&v_full[st], (g / NS) & 1, abort_flag)) { ok = false; break; }
+          if (j < n0) {
+            // the first product of an item overwrites O_0: its read-out by the
+            // previous item's epilogue must be complete
+            if (j == 0 && k > 0 && !mbar_wait(&o_free[0], (k - 1) & 1, abort_flag)) { ok = false; break; }
+            if (!issue_pv(0, st, j == 0, j == n0 - 1)) { ok = false; break; }
+          }
+          if (more) {
+            if (!mbar_wait(&k_full[(g + 1) % NS], ((g + 1) / NS) & 1, abort_flag)) { ok = false; break; }
+            tc_fence_after();
+            if (j + 1 < n0) issue_s(0, (g + 1) % NS);
+          }
+          if (j == 0 && k > 0 && !mbar_wait(&o_free[1], (k - 1) & 1, abort_flag)) { ok = false; break; }
+          if (!issue_pv(1, st, j == 0, j == n1 - 1)) { ok = false; break; }
+          mma_commit(&v_empty[st]);
+          if (more) {
+            issue_s(1, (g + 1) % NS);
+            mma_commit(&k_empty[(g + 1) % NS]);
+            if (j + 2 == n1) mma_commit(q_empty);  // last S of this item issued
+          }
         }
-        if (!issue_pv(1, j)) { ok = false; break; }
-        mma_commit(&v_empty[st]);
-        if (more) {
-          issue_s(1, j + 1);
-          mma_commit(&k_empty[(j + 1) % NS]);
-        }
+        kv += n1;
       }
       // All MMAs must retire before tensor memory is released.
       mma_commit(mma_final);
@@ -257,93 +327,113 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     // ------------------------------------------------------------ softmax
     const int w = warp >> 2;                       // query tile of this warpgroup
     const int row = threadIdx.x - w * TILE_M;      // 0..127, TMEM lane
-    const int q_row0 = row_base + w * TILE_M;
-    const int row_g = q_row0 + row;
-    const int n_kv = w == 0 ? n_kv0 : n_kv1;
     const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
     const uint32_t tS = tmem_base + w * 128 + lane_off;
     const uint32_t tO = tmem_base + 256 + w * 128 + lane_off;
     const float sl2 = p.scale_log2;
-    float m = -INFINITY;  // running max of scale * log2(e) * s
-    float l = 0.f;
+    int scount = 0;   // S tiles consumed (all items)
+    int pv_base = 0;  // O += P V products of previous items
     bool ok = true;
-    for (int j = 0; j < n_kv; ++j) {
-      if (!mbar_wait_warp(&s_full[w], j & 1, abort_flag)) {
-        ok = false;
-        break;
-      }
-      tc_fence_after();
-      uint32_t sr[128];
-      tmem_ld32(tS + 0, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
-      tmem_ld32(tS + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
-      tmem_ld32(tS + 64, *reinterpret_cast<uint32_t(*)[32]>(&sr[64]));
-      tmem_ld32(tS + 96, *reinterpret_cast<uint32_t(*)[32]>(&sr[96]));
-      tmem_ld_wait();
-      const int key0 = j * BLOCK_N;
-      const bool need_mask = (key0 + BLOCK_N > p.N) || (CAUSAL && key0 + BLOCK_N - 1 > q_row0);
-      float mx0 = -INFINITY, mx1 = -INFINITY;
-      if (need_mask) {
-        const int lim = CAUSAL ? min(p.N - 1, row_g) : p.N - 1;  // last admissible key
-#pragma unroll
-        for (int c = 0; c < 128; ++c) {
-          const float s = (key0 + c <= lim) ? __uint_as_float(sr[c]) : -INFINITY;
-          sr[c] = __float_as_uint(s);
-          if (c & 1) mx1 = fmaxf(mx1, s); else mx0 = fmaxf(mx0, s);
-        }
-      } else {
-#pragma unroll
-        for (int c = 0; c < 128; c += 2) {
-          mx0 = fmaxf(mx0, __uint_as_float(sr[c]));
-          mx1 = fmaxf(mx1, __uint_as_float(sr[c + 1]));
-        }
-      }
-      // scale * log2(e) > 0, so the maximum of the scaled row is the scaled maximum
-      const float m_new = fmaxf(m, fmaxf(mx0, mx1) * sl2);
-      const bool grow = (m_new - m) > RESCALE_THRESHOLD;  // true when m = -inf
-      const bool warp_grow = __any_sync(0xffffffffu, grow);
-      const float m_use = warp_grow ? m_new : m;
-      const float m_ref = (m_use == -INFINITY) ? 0.f : m_use;
-      const float alpha = ex2_approx(m - m_ref);  // 0 when m = -inf
-      float rs0 = 0.f, rs1 = 0.f;
-#pragma unroll
-      for (int c = 0; c < 128; c += 32) {
-        uint32_t pk[16];
-#pragma unroll
-        for (int e = 0; e < 32; e += 2) {
-          const float p0 = ex2_approx(fmaf(__uint_as_float(sr[c + e]), sl2, -m_ref));
-          const float p1 = ex2_approx(fmaf(__uint_as_float(sr[c + e + 1]), sl2, -m_ref));
-          rs0 += p0;
-          rs1 += p1;
-          pk[e >> 1] = pack_bf16x2(p0, p1);
-        }
-        tmem_st16(tS + (c >> 1), pk);
-      }
-      l = l * alpha + (rs0 + rs1);
-      if (warp_grow && j > 0) {
-        // O holds P_0 V_0 + ... + P_{j-1} V_{j-1} relative to the old max.  S_w,j
-        // was issued after O_w += P_{j-1} V_{j-1}, so that product has landed
-        // (o_done[w] has completed exactly j times); the wait only confirms it.
-        if (!mbar_wait_warp(&o_done[w], (j - 1) & 1, abort_flag)) {
+    for (int k = 0; ok; ++k) {
+      const int item = cta_item(cta, k, G);
+      if (item >= p.total_items) break;
+      int bh, tile;
+      item_coords(p, item, bh, tile);
+      const int q_row0 = tile * BLOCK_M + w * TILE_M;
+      const int row_g = q_row0 + row;
+      const int n_kv = n_kv_of(tile, w);
+      float m = -INFINITY;  // running max of scale * log2(e) * s
+      float l = 0.f;
+      for (int j = 0; j < n_kv; ++j) {
+        if (!mbar_wait_warp(&s_full[w], scount & 1, abort_flag)) {
           ok = false;
           break;
         }
+        ++scount;
         tc_fence_after();
+        uint32_t sr[128];
+        tmem_ld32(tS + 0, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
+        tmem_ld32(tS + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
+        tmem_ld32(tS + 64, *reinterpret_cast<uint32_t(*)[32]>(&sr[64]));
+        tmem_ld32(tS + 96, *reinterpret_cast<uint32_t(*)[32]>(&sr[96]));
+        tmem_ld_wait();
+        const int key0 = j * BLOCK_N;
+        const bool need_mask = (key0 + BLOCK_N > p.N) || (CAUSAL && key0 + BLOCK_N - 1 > q_row0);
+        // four independent max chains (latency, not throughput, bounds this loop)
+        float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+        if (need_mask) {
+          const int lim = CAUSAL ? min(p.N - 1, row_g) : p.N - 1;  // last admissible key
 #pragma unroll
-        for (int c = 0; c < D; c += 32) {
-          uint32_t orow[32];
-          tmem_ld32(tO + c, orow);
-          tmem_ld_wait();
+          for (int c = 0; c < 128; ++c) {
+            const float s = (key0 + c <= lim) ? __uint_as_float(sr[c]) : -INFINITY;
+            sr[c] = __float_as_uint(s);
+            mx[c & 3] = fmaxf(mx[c & 3], s);
+          }
+        } else {
 #pragma unroll
-          for (int e = 0; e < 32; ++e) orow[e] = __float_as_uint(__uint_as_float(orow[e]) * alpha);
-          tmem_st32(tO + c, orow);
+          for (int c = 0; c < 128; ++c) mx[c & 3] = fmaxf(mx[c & 3], __uint_as_float(sr[c]));
         }
+        // scale * log2(e) > 0, so the maximum of the scaled row is the scaled maximum
+        const float m_new = fmaxf(m, fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])) * sl2);
+        const bool grow = (m_new - m) > RESCALE_THRESHOLD;  // true when m = -inf
+        const bool warp_grow = __any_sync(0xffffffffu, grow);
+        const float m_use = warp_grow ? m_new : m;
+        const float m_ref = (m_use == -INFINITY) ? 0.f : m_use;
+        const float alpha = ex2_approx(m - m_ref);  // 0 when m = -inf
+        float rs[4] = {0.f, 0.f, 0.f, 0.f};
+        // Exponentials: MUFU ex2; in unmasked tiles EMU_PAIRS of every 4 pairs
+        // may go to the FMA-pipe polynomial.  Masked tiles use ex2 only, so
+        // excluded keys give exactly 0.
+#pragma unroll
+        for (int c = 0; c < 128; c += 32) {
+          uint32_t pk[16];
+#pragma unroll
+          for (int e = 0; e < 32; e += 2) {
+            const float x0 = fmaf(__uint_as_float(sr[c + e]), sl2, -m_ref);
+            const float x1 = fmaf(__uint_as_float(sr[c + e + 1]), sl2, -m_ref);
+            float p0, p1;
+            if (((e >> 1) & 3) >= 4 - EMU_PAIRS && !need_mask) {
+              p0 = ex2_poly3(x0);
+              p1 = ex2_poly3(x1);
+            } else {
+              p0 = ex2_approx(x0);
+              p1 = ex2_approx(x1);
+            }
+            rs[(e >> 1) & 3] += p0 + p1;
+            pk[e >> 1] = pack_bf16x2(p0, p1);
+          }
+          tmem_st16(tS + (c >> 1), pk);
+        }
+        l = l * alpha + ((rs[0] + rs[1]) + (rs[2] + rs[3]));
+        if (warp_grow && j > 0) {
+          // O holds P_0 V_0 + ... + P_{j-1} V_{j-1} relative to the old max.
+          // S_w,j was issued after O_w += P_{j-1} V_{j-1}, so o_done[w] has
+          // completed exactly pv_base + j times; the wait only confirms it.
+          if (!mbar_wait_warp(&o_done[w], (pv_base + j - 1) & 1, abort_flag)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+#pragma unroll
+          for (int c = 0; c < D; c += 32) {
+            uint32_t orow[32];
+            tmem_ld32(tO + c, orow);
+            tmem_ld_wait();
+#pragma unroll
+            for (int e = 0; e < 32; ++e)
+              orow[e] = __float_as_uint(__uint_as_float(orow[e]) * alpha);
+            tmem_st32(tO + c, orow);
+          }
+        }
+        m = m_use;
+        tmem_st_wait();
+        tc_fence_before();
+        mbar_arrive(&p_full[w]);
       }
-      m = m_use;
-      tmem_st_wait();
-      tc_fence_before();
-      mbar_arrive(&p_full[w]);
-    }
-    if (ok && n_kv > 0 && mbar_wait_warp(&o_final[w], 0, abort_flag)) {
+      if (!ok || !mbar_wait_warp(&o_final[w], k & 1, abort_flag)) {
+        ok = false;
+        break;
+      }
       tc_fence_after();
       const float inv_l = (l > 0.f) ? 1.f / l : 0.f;
       const bool valid = row_g < p.N;
@@ -365,11 +455,15 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             dst[v4] = make_uint4(pk[4 * v4], pk[4 * v4 + 1], pk[4 * v4 + 2], pk[4 * v4 + 3]);
         }
       }
+      // O_w has been read: the next item's first O += P V may overwrite it.
+      tc_fence_before();
+      mbar_arrive(&o_free[w]);
       if (valid && p.lse != nullptr) {
         // LSE = ln(sum exp(scale * s)) = (m + log2 l) * ln 2, m in log2 units.
         const float lse = (l > 0.f) ? (m + lg2_approx(l)) * 0.6931471805599453f : -INFINITY;
         p.lse[static_cast<size_t>(bh) * p.N + row_g] = lse;
       }
+      pv_base += n_kv;
     }
     tmem_ld_wait();
     tmem_st_wait();
@@ -386,7 +480,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 
 template <int D, bool CAUSAL>
 fa_status launch(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
-                 const Params& prm, int BH, cudaStream_t stream) {
+                 const Params& prm, int grid_size, cudaStream_t stream) {
   auto kern = fa_fwd_kernel<D, CAUSAL>;
   static bool configured = false;  // per process; the attribute is per function
   if (!configured) {
@@ -395,11 +489,23 @@ fa_status launch(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap
     if (e != cudaSuccess) return FA_ERR_CUDA;
     configured = true;
   }
-  // The 256-row tiles of a head are adjacent in launch order, so the CTAs
-  // resident at one time share few heads and K/V tiles stay in L2.
-  dim3 grid(prm.n_cta_tiles * BH);
-  kern<<<grid, NUM_THREADS, Smem<D>::ALLOC, stream>>>(tq, tk, tv, prm);
+  kern<<<grid_size, NUM_THREADS, Smem<D>::ALLOC, stream>>>(tq, tk, tv, prm);
   return cuda_status(cudaGetLastError());
+}
+
+// Work distribution.  Causal problems whose K and V all fit comfortably in L2
+// run persistently (one CTA per SM, longest tiles first, alternating rounds);
+// everything else runs one CTA per 256-row tile in head-major order, so the
+// resident CTAs share their heads' K/V tiles in L2.  FA_FWD_SCHEDULE=grid or
+// =persistent forces one of the two.
+int schedule_mode() {
+  static int mode = -1;
+  if (mode < 0) {
+    const char* env = std::getenv("FA_FWD_SCHEDULE");
+    mode = (env && std::strcmp(env, "grid") == 0) ? 1
+           : (env && std::strcmp(env, "persistent") == 0) ? 2 : 0;
+  }
+  return mode;
 }
 
 }  // namespace fwd
@@ -407,24 +513,43 @@ fa_status launch(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap
 fa_status launch_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B,
                      int H, int N, int d, int causal, float scale, cudaStream_t stream) {
   const int BH = B * H;
-  if (static_cast<long long>(BH) * ((N + fwd::BLOCK_M - 1) / fwd::BLOCK_M) > 0x7fffffffLL)
-    return FA_ERR_INVALID_ARG;
+  const long long n_cta_tiles = (N + fwd::BLOCK_M - 1) / fwd::BLOCK_M;
+  const long long items = static_cast<long long>(BH) * n_cta_tiles;
+  if (items > 0x7fffffffLL) return FA_ERR_INVALID_ARG;
   CUtensorMap tq, tk, tv;
   fa_status st;
   if ((st = make_tmap_bf16_3d(&tq, q, d, N, BH, fwd::TILE_M)) != FA_OK) return st;
   if ((st = make_tmap_bf16_3d(&tk, k, d, N, BH, fwd::BLOCK_N)) != FA_OK) return st;
   if ((st = make_tmap_bf16_3d(&tv, v, d, N, BH, fwd::BLOCK_N)) != FA_OK) return st;
+  int dev = 0, sms = 148;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+    return FA_ERR_CUDA;
+  const double kv_bytes = 4.0 * BH * static_cast<double>(N) * d;
+  const int mode = fwd::schedule_mode();
+  bool persistent = causal && items > sms && kv_bytes <= 96.0 * 1024 * 1024;
+  int grid = persistent ? sms : static_cast<int>(items);
+  if (mode == 1) {
+    persistent = false;
+    grid = static_cast<int>(items);
+  } else if (mode == 2) {  // forced: about three items per CTA even for small problems
+    persistent = true;
+    grid = static_cast<int>(std::min<long long>(sms, std::max<long long>(1, items / 3)));
+  }
   fwd::Params prm;
   prm.o = static_cast<__nv_bfloat16*>(o);
   prm.lse = lse;
   prm.N = N;
-  prm.n_cta_tiles = (N + fwd::BLOCK_M - 1) / fwd::BLOCK_M;
+  prm.BH = BH;
+  prm.n_cta_tiles = static_cast<int>(n_cta_tiles);
+  prm.total_items = static_cast<int>(items);
+  prm.lpt_order = persistent ? 1 : 0;
   prm.scale_log2 = scale * 1.4426950408889634f;
   if (d == 128)
-    return causal ? fwd::launch<128, true>(tq, tk, tv, prm, BH, stream)
-                  : fwd::launch<128, false>(tq, tk, tv, prm, BH, stream);
-  return causal ? fwd::launch<64, true>(tq, tk, tv, prm, BH, stream)
-                : fwd::launch<64, false>(tq, tk, tv, prm, BH, stream);
+    return causal ? fwd::launch<128, true>(tq, tk, tv, prm, grid, stream)
+                  : fwd::launch<128, false>(tq, tk, tv, prm, grid, stream);
+  return causal ? fwd::launch<64, true>(tq, tk, tv, prm, grid, stream)
+                : fwd::launch<64, false>(tq, tk, tv, prm, grid, stream);
 }
 
 }  // namespace fa

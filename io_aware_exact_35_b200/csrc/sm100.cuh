@@ -279,6 +279,27 @@ __device__ __forceinline__ float lg2_approx(float x) {
   return y;
 }
 
+// 2^x on the FMA pipe instead of the MUFU unit.  n = round(x) is formed by
+// adding 1.5 * 2^23; f = x - n lies in [-1/2, 1/2]; 2^f is the minimax cubic
+// (relative error <= 7.5e-5) fitted by the Remez exchange in
+// io_aware_exact_35_b200/exp2_poly.py; n is then added to the exponent field.
+// x is clamped at -125 so the exponent cannot underflow: inputs below that
+// (masked scores included) give about 2^-125 instead of 0, so use it only where
+// such a value is negligible against the rest of the sum.
+constexpr float kEx2C0 = 0.99992806f;
+constexpr float kEx2C1 = 0.69326097f;
+constexpr float kEx2C2 = 0.24261113f;
+constexpr float kEx2C3 = 0.05517167f;
+__device__ __forceinline__ float ex2_poly3(float x) {
+  x = fmaxf(x, -125.f);
+  const float t = __fadd_rn(x, 12582912.f);
+  const float f = __fsub_rn(x, __fsub_rn(t, 12582912.f));
+  float p = fmaf(kEx2C3, f, kEx2C2);
+  p = fmaf(p, f, kEx2C1);
+  p = fmaf(p, f, kEx2C0);
+  return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
+}
+
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&v);

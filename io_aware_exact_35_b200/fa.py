@@ -16,7 +16,9 @@ from typing import Optional
 
 import torch
 
-_LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "lib", "libfa_b200.so")
+# The in-tree build; FA_B200_LIBRARY may point at another build of the same library.
+_LIB_PATH = os.environ.get("FA_B200_LIBRARY") or os.path.join(
+    os.path.dirname(os.path.abspath(__file__)), "lib", "libfa_b200.so")
 _lib = None
 
 FA_OK = 0

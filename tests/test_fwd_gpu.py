@@ -103,3 +103,37 @@ def test_fwd_output_buffers_and_streams(fa_mod, cuda_device):
     o_ref, _ = oracle.attention_forward(*(inputs.to_f64(t) for t in (q, k, v)), True,
                                         1 / np.sqrt(d))
     check_o(o.cpu(), o_ref)
+
+
+_SCHEDULE_SCRIPT = r"""
+import sys, numpy as np, torch
+sys.path.insert(0, {root!r})
+import oracle
+from io_aware_exact_35_b200 import fa, inputs
+from tests._parity import check_o, check_lse
+for (B, H, N, d, causal) in [(2, 3, 1000, 128, True), (1, 5, 777, 64, True), (3, 2, 513, 128, False),
+                             (2, 4, 2048, 128, True)]:
+    q, k, v = inputs.fwd_inputs(B, H, N, d, seed=N + d)
+    o, lse = fa.fwd(q.cuda(), k.cuda(), v.cuda(), causal=causal)
+    torch.cuda.synchronize()
+    assert fa.get_device_error() == 0
+    ref_o, ref_l = oracle.attention_forward(*(inputs.to_f64(t) for t in (q, k, v)), causal, 1 / np.sqrt(d))
+    check_o(o.cpu(), ref_o)
+    check_lse(lse.cpu(), ref_l)
+print("ok")
+"""
+
+
+@pytest.mark.parametrize("schedule", ["persistent", "grid"])
+def test_fwd_both_work_schedules(fa_mod, cuda_device, schedule):
+    """The forward runs either one CTA per 256-row tile or persistently (each
+    CTA loops over several tiles, barrier phases carried across them); both
+    must give the oracle's result."""
+    import os
+    import subprocess
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    env = dict(os.environ, FA_FWD_SCHEDULE=schedule)
+    r = subprocess.run([sys.executable, "-c", _SCHEDULE_SCRIPT.format(root=root)], env=env,
+                       capture_output=True, text=True, timeout=600, cwd=root)
+    assert r.returncode == 0 and r.stdout.strip().endswith("ok"), r.stdout + r.stderr
