@@ -145,6 +145,11 @@ class ClockSampler:
 
 
 # ----------------------------------------------------------------------------- workloads
+def workload_config(w, parallelism):
+    return {"workload": w.name, "B": w.B, "H": w.H, "N": w.N or None, "d": w.d,
+            "causal": w.causal, "parallelism": parallelism}
+
+
 def fwd_flops(w):
     f = 4.0 * w.B * w.H * w.N * w.N * w.d
     return f * 0.5 if w.causal else f
@@ -349,7 +354,7 @@ def run_reference(args, w, total_budget=150.0, emit=True):
         "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": tot_t / args.steps * 1e3, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": w.name, "parallelism": "cpu"},
+        "config": workload_config(w, "cpu"),
         "cpu_baseline": {"value": value, "unit": unit, "cores": cores, "kind": "oracle",
                          "sample": sample + (" (bwd: forward-row oracle time x3.5)" if w.kind == "bwd" else "")},
         "e2e": {"value": value, "unit": unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -434,10 +439,9 @@ def main():
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": mean_s * 1e3,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "bf16", "data": "synthetic",
-        "config": {"workload": w.name, "B": w.B, "H": w.H, "N": w.N or None, "d": w.d,
-                   "causal": w.causal, "parallelism": f"replicas{world}" if world > 1 else "single",
-                   "l2": "flushed (256 MB write) before every step" if r.flush is not None
-                   else "inputs larger than L2"},
+        "config": dict(workload_config(w, f"replicas{world}" if world > 1 else "single"),
+                       l2="flushed (256 MB write) before every step" if r.flush is not None
+                       else "inputs larger than L2"),
         "roofline": roof,
         "e2e": {"value": r.value(e2e_s) * world, "unit": r.unit, "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h},

@@ -91,6 +91,20 @@ fa_status make_tmap_f32_2d(CUtensorMap* map, const void* base, uint64_t n, uint6
   return r == CUDA_SUCCESS ? FA_OK : FA_ERR_CUDA;
 }
 
+fa_status make_tmap_f32_3d_sw128(CUtensorMap* map, const void* base, uint64_t d, uint64_t rows,
+                                 uint64_t outer) {
+  EncodeTiledFn fn = encode_fn();
+  if (fn == nullptr) return FA_ERR_CUDA;
+  const cuuint64_t dims[3] = {d, rows, outer};
+  const cuuint64_t strides[2] = {d * 4, rows * d * 4};
+  const cuuint32_t box[3] = {32u, 128u, 1u};
+  const cuuint32_t estr[3] = {1u, 1u, 1u};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, const_cast<void*>(base), dims, strides,
+                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? FA_OK : FA_ERR_CUDA;
+}
+
 }  // namespace fa
 
 using namespace fa;

@@ -15,19 +15,22 @@
 //                        S^T = K_j Q_i^T, dP^T = V_j dO_i^T        (tcgen05, TMEM)
 //                        P^T, dS^T on the CUDA cores (one key row per thread)
 //                        dV += P^T dO_i, dK += dS^T Q_i            (A from TMEM)
-//                        dQ_i = dS K_j  (A = dS from shared memory) -> fp32
-//                        vector reductions into the dQ accumulator.
+//                        dQ_i = dS K_j  (A = dS from shared memory), added to
+//                        an fp32 accumulator with bulk tensor reductions.
 //   fa_bwd_dq_convert  dQ = scale * accumulator, rounded to bf16.
 //
-// Warp roles of fa_bwd_kernel (320 threads):
-//   warps 0-3  "softmax" warpgroup: thread t owns key row t (TMEM lane t).
-//   warps 4-7  dQ warpgroup: thread t owns query row t of the dQ tile.
-//   warp 8     TMA producer: K_j, V_j once; Q_i, dO_i, LSE_i, D_i through a
+// Warp roles of fa_bwd_kernel (448 threads):
+//   warps 0-7  two P^T / dS^T warpgroups: thread t of warpgroup g owns key row t
+//              (TMEM lane t) for queries 64g .. 64g+63 of the tile; in the
+//              epilogue warpgroup 0 writes dV and warpgroup 1 writes dK.
+//   warps 8-11 dQ warpgroup: thread t owns query row t of the dQ tile.
+//   warp 12    TMA producer: K_j, V_j once; Q_i, dO_i, LSE_i, D_i through a
 //              two-stage ring.
-//   warp 9     tensor-memory allocator and MMA issuer.
-// Tensor memory (512 columns): S^T [0,128) (P^T bf16 overwrites its first 64
-// columns), dP^T [128,256) (dS^T bf16 overwrites its first 64 columns, and
-// dQ_i lands in [128, 128+d) afterwards), dV [256, 256+d), dK [256+d, 256+2d).
+//   warp 13    tensor-memory allocator and MMA issuer.
+// Tensor memory (512 columns): S^T [0,128), dP^T [128,256), dV [256, 256+d),
+// dK [256+d, 256+2d).  Warpgroup g overwrites columns [64g, 64g+32) of S^T
+// with P^T (bf16 pairs) and the same columns of dP^T with dS^T, i.e. only
+// scores it has already read; dQ_i lands in [128, 128+d) afterwards.
 #include "fa_internal.h"
 #include "sm100.cuh"
 
@@ -36,7 +39,7 @@ namespace fa {
 namespace bwd {
 
 constexpr int BLOCK = 128;
-constexpr int NUM_THREADS = 320;
+constexpr int NUM_THREADS = 448;
 constexpr int PANEL_BYTES = 128 * 128;
 constexpr uint32_t TMEM_COLS = 512;
 constexpr float LOG2E = 1.4426950408889634f;
@@ -55,8 +58,8 @@ struct Smem {
   static constexpr int DD_OFF = LSE_OFF + 2 * 512;     // 2 stages x 128 fp32
   static constexpr int BAR_OFF = DD_OFF + 2 * 512;
   // kv_full, qd_full[2], qd_empty[2], st_full, dpt_full, pds_full, dq_full,
-  // dq_free, dkv_final, mma_final
-  static constexpr int NBAR = 12;
+  // dq_free, dkv_final, mma_final, stg_full, stg_free
+  static constexpr int NBAR = 14;
   static constexpr int MISC_OFF = BAR_OFF + NBAR * 8;
   static constexpr int BYTES = MISC_OFF + 16;
   static constexpr int ALLOC = BYTES > 118784 ? BYTES : 118784;
@@ -72,16 +75,6 @@ struct Params {
   float scale;
 };
 
-__device__ __forceinline__ void red_add_v4(float* addr, float a, float b, float c, float d) {
-  asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(addr), "f"(a), "f"(b),
-               "f"(c), "f"(d)
-               : "memory");
-}
-
-__device__ __forceinline__ void fence_proxy_async_smem() {
-  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-}
-
 __device__ __forceinline__ void tma_load_2d(void* smem_dst, const void* desc, uint64_t* bar,
                                             int c0, int c1) {
   asm volatile(
@@ -96,7 +89,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     fa_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                   const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
                   const __grid_constant__ CUtensorMap tm_lse,
-                  const __grid_constant__ CUtensorMap tm_dd, const Params p) {
+                  const __grid_constant__ CUtensorMap tm_dd,
+                  const __grid_constant__ CUtensorMap tm_dq, const Params p) {
   using L = Smem<D>;
   extern __shared__ __align__(1024) uint8_t smem[];
   // The swizzled operand tiles need 1024-byte alignment; the kernel declares
@@ -116,6 +110,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   uint64_t* dq_free = bars + 9;
   uint64_t* dkv_final = bars + 10;
   uint64_t* mma_final = bars + 11;
+  uint64_t* stg_full = bars + 12;  // dQ staging written (128 arrivals)
+  uint64_t* stg_free = bars + 13;  // dQ staging read by the bulk reduction
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::MISC_OFF);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::MISC_OFF + 4);
 
@@ -132,12 +128,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 
   if (threadIdx.x == 0) {
     for (int b = 0; b < L::NBAR; ++b) mbar_init(&bars[b], 1);
-    mbar_init(pds_full, BLOCK);
+    mbar_init(pds_full, 2 * BLOCK);  // both P^T / dS^T warpgroups
     mbar_init(dq_free, BLOCK);
+    mbar_init(stg_full, BLOCK);
     *abort_flag = 0;
     fence_mbar_init();
   }
-  if (warp == 9) {
+  if (warp == 13) {
     tmem_alloc(tmem_slot, TMEM_COLS);
     tmem_relinquish();
   }
@@ -150,7 +147,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   const uint32_t tdV = tmem_base + 256;
   const uint32_t tdK = tmem_base + 256 + D;
 
-  if (warp == 8) {
+  if (warp == 12) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
       tma_prefetch_desc(&tm_q);
@@ -181,7 +178,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       for (int s = 0; s < 2; ++s)
         if (last[s] >= 0) mbar_wait_drain(&qd_full[s], last[s] & 1);
     }
-  } else if (warp == 9) {
+  } else if (warp == 13) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       constexpr uint32_t IDESC_SS = idesc_bf16_f32(BLOCK, BLOCK, false, false);
@@ -219,14 +216,18 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         if (!mbar_wait(pds_full, it & 1, abort_flag)) { ok = false; break; }
         tc_fence_after();
         const uint32_t acc = it > 0 ? 1u : 0u;
+        // P^T / dS^T of queries 64g .. 64g+63 sit in columns 64g .. 64g+31 of
+        // their buffer (warpgroup g wrote them over scores it had read).
 #pragma unroll
         for (int kk = 0; kk < BLOCK / 16; ++kk)  // dV += P^T dO_i
-          mma_bf16_ts(tdV, tSt + kk * 8, sdesc_mnmajor_sw128(do_addr + kk * 2048, PANEL_BYTES),
-                      IDESC_ACC, (acc | kk) ? 1u : 0u);
+          mma_bf16_ts(tdV, tSt + (kk >> 2) * 64 + (kk & 3) * 8,
+                      sdesc_mnmajor_sw128(do_addr + kk * 2048, PANEL_BYTES), IDESC_ACC,
+                      (acc | kk) ? 1u : 0u);
 #pragma unroll
         for (int kk = 0; kk < BLOCK / 16; ++kk)  // dK += dS^T Q_i
-          mma_bf16_ts(tdK, tdPt + kk * 8, sdesc_mnmajor_sw128(q_addr + kk * 2048, PANEL_BYTES),
-                      IDESC_ACC, (acc | kk) ? 1u : 0u);
+          mma_bf16_ts(tdK, tdPt + (kk >> 2) * 64 + (kk & 3) * 8,
+                      sdesc_mnmajor_sw128(q_addr + kk * 2048, PANEL_BYTES), IDESC_ACC,
+                      (acc | kk) ? 1u : 0u);
 #pragma unroll
         for (int kk = 0; kk < BLOCK / 16; ++kk)  // dQ_i = dS K_j (M = queries, K = keys)
           mma_bf16_ss(tdPt, sdesc_mnmajor_sw128(ds_addr + kk * 2048, PANEL_BYTES),
@@ -239,14 +240,16 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       mma_commit(mma_final);
       mbar_wait_drain(mma_final, 0);
     }
-  } else if (warp < 4) {
+  } else if (warp < 8) {
     // ------------------------------------------------------------ P^T / dS^T
-    const int t = threadIdx.x;  // key row
+    // Warpgroup g handles queries 64g .. 64g+63 of every key row.
+    const int g = warp >> 2;
+    const int t = threadIdx.x - g * BLOCK;  // key row, TMEM lane
     const int key_g = key0 + t;
     const bool key_ok = key_g < p.N;
-    const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
+    const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
     const float sl2 = p.scale_log2;
-    uint8_t* ds_row = smem + L::DS_OFF + t * 128;  // row t of each 64-query panel
+    uint8_t* ds_row = smem + L::DS_OFF + g * PANEL_BYTES + t * 128;  // row t of panel g
     const uint32_t sw = static_cast<uint32_t>(t & 7);
     bool ok = true;
     for (int it = 0; it < n_it; ++it) {
@@ -264,7 +267,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       // so their P is exactly 0; causal also drops queries before the key.
       const bool diag = CAUSAL && (q0 == key0);
 #pragma unroll 1
-      for (int c = 0; c < BLOCK; c += 32) {
+      for (int c = 64 * g; c < 64 * g + 64; c += 32) {
         uint32_t sr[32], dr[32];
         tmem_ld32(tSt + lane_off + c, sr);
         tmem_ld32(tdPt + lane_off + c, dr);
@@ -287,11 +290,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           pk[e >> 1] = pack_bf16x2(pv[0], pv[1]);
           dk[e >> 1] = pack_bf16x2(dv[0], dv[1]);
         }
-        tmem_st16(tSt + lane_off + (c >> 1), pk);
-        tmem_st16(tdPt + lane_off + (c >> 1), dk);
-        // dS row t, queries c..c+31: panel c/64, 16-byte chunks (c%64)/8 .. +3,
+        // columns 64g + (c - 64g)/2: inside the range this warpgroup has read
+        const uint32_t pc = static_cast<uint32_t>(64 * g + ((c - 64 * g) >> 1));
+        tmem_st16(tSt + lane_off + pc, pk);
+        tmem_st16(tdPt + lane_off + pc, dk);
+        // dS row t, queries c..c+31: panel g, 16-byte chunks (c%64)/8 .. +3,
         // 128-byte swizzle (chunk index xor row % 8).
-        uint8_t* prow = ds_row + (c >> 6) * PANEL_BYTES;
+        uint8_t* prow = ds_row;
         const uint32_t ch0 = static_cast<uint32_t>((c & 63) >> 3);
 #pragma unroll
         for (int u = 0; u < 4; ++u) {
@@ -305,12 +310,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       tc_fence_before();
       mbar_arrive(pds_full);
     }
-    // epilogue: dV and scale * dK, one key row per thread
+    // epilogue: warpgroup 0 writes dV, warpgroup 1 scale * dK, one key row per thread
     if (ok && mbar_wait_warp(dkv_final, 0, abort_flag)) {
       tc_fence_after();
       const size_t rowoff = (static_cast<size_t>(bh) * p.N + key_g) * D;
-#pragma unroll 1
-      for (int which = 0; which < 2; ++which) {
+      {
+        const int which = g;
         const uint32_t tacc = which == 0 ? tdV : tdK;
         const float mul = which == 0 ? 1.f : p.scale;
         __nv_bfloat16* dst_row = (which == 0 ? p.dv : p.dk) + rowoff;
@@ -336,34 +341,65 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     tmem_st_wait();
   } else {
     // ------------------------------------------------------------ dQ reduction
-    const int t = threadIdx.x - 128;  // query row of the dQ tile, TMEM lane
+    // dQ_i (fp32, 128 query rows x d) leaves tensor memory 64 columns at a
+    // time through the dS buffer, which the dQ MMA has finished reading: two
+    // 128 x 32 fp32 boxes with the 128-byte swizzle, then one thread adds
+    // them to the accumulator with bulk tensor reductions.  dq_free is
+    // signalled once the staging buffer has been read, which also frees it
+    // for the next tile's dS (written only after the next dP^T, which waits
+    // for dq_free).
+    const int t = threadIdx.x - 2 * BLOCK;  // query row of the dQ tile, TMEM lane
     const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
-    for (int it = 0; it < n_it; ++it) {
-      const int q_g = (i_begin + it) * BLOCK + t;
+    uint8_t* stage = smem + L::DS_OFF;      // 2 boxes of 128 rows x 128 bytes
+    const uint32_t sw = static_cast<uint32_t>(t & 7);
+    int rounds = 0;  // staging rounds so far
+    bool ok = true;
+    for (int it = 0; ok && it < n_it; ++it) {
+      const int q0 = (i_begin + it) * BLOCK;
       if (!mbar_wait_warp(dq_full, it & 1, abort_flag)) break;
       tc_fence_after();
-      float* dst = p.dqacc + (static_cast<size_t>(bh) * p.N + q_g) * D;
 #pragma unroll 1
-      for (int c = 0; c < D; c += 32) {
-        uint32_t r[32];
-        tmem_ld32(tdPt + lane_off + c, r);
+      for (int h = 0; h < D / 64; ++h, ++rounds) {
+        uint32_t r[2][32];
+        tmem_ld32(tdPt + lane_off + 64 * h, r[0]);
+        tmem_ld32(tdPt + lane_off + 64 * h + 32, r[1]);
         tmem_ld_wait();
-        if (q_g < p.N) {
 #pragma unroll
-          for (int v4 = 0; v4 < 8; ++v4)
-            red_add_v4(dst + c + 4 * v4, __uint_as_float(r[4 * v4]), __uint_as_float(r[4 * v4 + 1]),
-                       __uint_as_float(r[4 * v4 + 2]), __uint_as_float(r[4 * v4 + 3]));
+        for (int b = 0; b < 2; ++b) {
+          uint8_t* row = stage + b * PANEL_BYTES + t * 128;
+#pragma unroll
+          for (int c = 0; c < 8; ++c)
+            *reinterpret_cast<uint4*>(row + ((c ^ sw) << 4)) =
+                make_uint4(r[b][4 * c], r[b][4 * c + 1], r[b][4 * c + 2], r[b][4 * c + 3]);
+        }
+        fence_proxy_async_smem();
+        mbar_arrive(stg_full);
+        if (t == 0) {
+          if (mbar_wait(stg_full, rounds & 1, abort_flag)) {
+            tma_reduce_add_3d(&tm_dq, stage, 64 * h, q0, bh);
+            tma_reduce_add_3d(&tm_dq, stage + PANEL_BYTES, 64 * h + 32, q0, bh);
+            bulk_commit_group();
+            bulk_wait_group_read0();
+          }
+          mbar_arrive(stg_free);
+        }
+        // the staging buffer may be rewritten once the reduction has read it
+        if (!mbar_wait_warp(stg_free, rounds & 1, abort_flag)) {
+          ok = false;
+          break;
         }
       }
+      if (!ok) break;
       tc_fence_before();
       mbar_arrive(dq_free);
     }
+    if (t == 0) bulk_wait_group0();
     tmem_ld_wait();
   }
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 9) {
+  if (warp == 13) {
     __syncwarp();
     tc_fence_after();
     tmem_dealloc(tmem_base, TMEM_COLS);
@@ -436,7 +472,7 @@ fa_status launch_main(const CUtensorMap* maps, const Params& prm, int BH, cudaSt
   }
   dim3 grid(prm.n_tiles * BH);
   kern<<<grid, NUM_THREADS, Smem<D>::ALLOC, stream>>>(maps[0], maps[1], maps[2], maps[3], maps[4],
-                                                      maps[5], prm);
+                                                      maps[5], maps[6], prm);
   return cuda_status(cudaGetLastError());
 }
 
@@ -469,7 +505,7 @@ fa_status launch_bwd(const void* q, const void* k, const void* v, const void* o,
     if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
   }
   // 2. dK, dV and the dQ accumulation
-  CUtensorMap maps[6];
+  CUtensorMap maps[7];
   fa_status st;
   if ((st = make_tmap_bf16_3d(&maps[0], q, d, N, BH, bwd::BLOCK)) != FA_OK) return st;
   if ((st = make_tmap_bf16_3d(&maps[1], k, d, N, BH, bwd::BLOCK)) != FA_OK) return st;
@@ -477,6 +513,7 @@ fa_status launch_bwd(const void* q, const void* k, const void* v, const void* o,
   if ((st = make_tmap_bf16_3d(&maps[3], dout, d, N, BH, bwd::BLOCK)) != FA_OK) return st;
   if ((st = make_tmap_f32_2d(&maps[4], lse2, Np, BH)) != FA_OK) return st;
   if ((st = make_tmap_f32_2d(&maps[5], dd, Np, BH)) != FA_OK) return st;
+  if ((st = make_tmap_f32_3d_sw128(&maps[6], dqacc, d, N, BH)) != FA_OK) return st;
   bwd::Params prm;
   prm.dk = static_cast<__nv_bfloat16*>(dk);
   prm.dv = static_cast<__nv_bfloat16*>(dv);

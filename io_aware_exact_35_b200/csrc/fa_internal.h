@@ -22,6 +22,11 @@ fa_status make_tmap_bf16_3d(CUtensorMap* map, const void* base, uint64_t d, uint
 // swizzle; n * 4 must be a multiple of 16 bytes.
 fa_status make_tmap_f32_2d(CUtensorMap* map, const void* base, uint64_t n, uint64_t outer);
 
+// 3-D float32 tensor map over a [outer, rows, d] array with a 32 x 128 x 1 box
+// (128 bytes wide) and 128-byte swizzle, for bulk reductions of 128-row tiles.
+fa_status make_tmap_f32_3d_sw128(CUtensorMap* map, const void* base, uint64_t d, uint64_t rows,
+                                 uint64_t outer);
+
 // Row stride (elements) of the per-row float32 tables of the backward
 // workspace: N rounded up to whole 128-row tiles.
 inline size_t bwd_row_pad(int N) { return (static_cast<size_t>(N) + 127) / 128 * 128; }
