@@ -184,33 +184,40 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       constexpr uint32_t IDESC_SS = idesc_bf16_f32(BLOCK, BLOCK, false, false);
       constexpr uint32_t IDESC_ACC = idesc_bf16_f32(BLOCK, D, false, true);
       constexpr uint32_t IDESC_DQ = idesc_bf16_f32(BLOCK, D, true, true);
-      const uint32_t k_addr = smem_u32(smem + L::K_OFF);
-      const uint32_t v_addr = smem_u32(smem + L::V_OFF);
-      const uint32_t ds_addr = smem_u32(smem + L::DS_OFF);
+      // Descriptors are built once; a k-step adds a compile-time byte offset
+      // (>> 4) to the start-address field (no carry below 256 KB), so each MMA
+      // costs a few instructions on a scheduler shared with busy warps.
+      const uint64_t kdK = sdesc_kmajor_sw128(smem_u32(smem + L::K_OFF));
+      const uint64_t vdK = sdesc_kmajor_sw128(smem_u32(smem + L::V_OFF));
+      const uint64_t kdM = sdesc_mnmajor_sw128(smem_u32(smem + L::K_OFF), PANEL_BYTES);
+      const uint64_t dsdM = sdesc_mnmajor_sw128(smem_u32(smem + L::DS_OFF), PANEL_BYTES);
+      const uint64_t qdK0 = sdesc_kmajor_sw128(smem_u32(smem + L::Q_OFF));
+      const uint64_t dodK0 = sdesc_kmajor_sw128(smem_u32(smem + L::DO_OFF));
+      const uint64_t qdM0 = sdesc_mnmajor_sw128(smem_u32(smem + L::Q_OFF), PANEL_BYTES);
+      const uint64_t dodM0 = sdesc_mnmajor_sw128(smem_u32(smem + L::DO_OFF), PANEL_BYTES);
+      auto koff = [](int kk) {  // K-major: 16-element K slice kk of a 128-row tile
+        return static_cast<uint64_t>(((kk >> 2) * PANEL_BYTES + (kk & 3) * 32) >> 4);
+      };
+      auto moff = [](int kk) {  // MN-major: rows 16kk .. 16kk+15
+        return static_cast<uint64_t>((kk * 2048) >> 4);
+      };
       bool ok = mbar_wait(kv_full, 0, abort_flag);
       for (int it = 0; ok && it < n_it; ++it) {
         const int st = it & 1;
-        const uint32_t q_addr = smem_u32(smem + L::Q_OFF + st * L::TILE);
-        const uint32_t do_addr = smem_u32(smem + L::DO_OFF + st * L::TILE);
+        const uint64_t soff = static_cast<uint64_t>((st * L::TILE) >> 4);
         if (!mbar_wait(&qd_full[st], (it >> 1) & 1, abort_flag)) { ok = false; break; }
         tc_fence_after();
         // S^T = K_j Q_i^T  (M = keys, N = queries, K = d)
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * PANEL_BYTES + (kk & 3) * 32;
-          mma_bf16_ss(tSt, sdesc_kmajor_sw128(k_addr + off), sdesc_kmajor_sw128(q_addr + off),
-                      IDESC_SS, kk > 0 ? 1u : 0u);
-        }
+        for (int kk = 0; kk < D / 16; ++kk)
+          mma_bf16_ss(tSt, kdK + koff(kk), qdK0 + soff + koff(kk), IDESC_SS, kk > 0 ? 1u : 0u);
         mma_commit(st_full);
         // dP^T = V_j dO_i^T, into columns the dQ warps must have emptied.
         if (it >= 1 && !mbar_wait(dq_free, (it - 1) & 1, abort_flag)) { ok = false; break; }
         tc_fence_after();
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * PANEL_BYTES + (kk & 3) * 32;
-          mma_bf16_ss(tdPt, sdesc_kmajor_sw128(v_addr + off), sdesc_kmajor_sw128(do_addr + off),
-                      IDESC_SS, kk > 0 ? 1u : 0u);
-        }
+        for (int kk = 0; kk < D / 16; ++kk)
+          mma_bf16_ss(tdPt, vdK + koff(kk), dodK0 + soff + koff(kk), IDESC_SS, kk > 0 ? 1u : 0u);
         mma_commit(dpt_full);
         // P^T, dS^T (tensor memory) and dS (shared memory) are ready.
         if (!mbar_wait(pds_full, it & 1, abort_flag)) { ok = false; break; }
@@ -220,19 +227,15 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         // their buffer (warpgroup g wrote them over scores it had read).
 #pragma unroll
         for (int kk = 0; kk < BLOCK / 16; ++kk)  // dV += P^T dO_i
-          mma_bf16_ts(tdV, tSt + (kk >> 2) * 64 + (kk & 3) * 8,
-                      sdesc_mnmajor_sw128(do_addr + kk * 2048, PANEL_BYTES), IDESC_ACC,
-                      (acc | kk) ? 1u : 0u);
+          mma_bf16_ts(tdV, tSt + (kk >> 2) * 64 + (kk & 3) * 8, dodM0 + soff + moff(kk),
+                      IDESC_ACC, (acc | kk) ? 1u : 0u);
 #pragma unroll
         for (int kk = 0; kk < BLOCK / 16; ++kk)  // dK += dS^T Q_i
-          mma_bf16_ts(tdK, tdPt + (kk >> 2) * 64 + (kk & 3) * 8,
-                      sdesc_mnmajor_sw128(q_addr + kk * 2048, PANEL_BYTES), IDESC_ACC,
-                      (acc | kk) ? 1u : 0u);
+          mma_bf16_ts(tdK, tdPt + (kk >> 2) * 64 + (kk & 3) * 8, qdM0 + soff + moff(kk),
+                      IDESC_ACC, (acc | kk) ? 1u : 0u);
 #pragma unroll
         for (int kk = 0; kk < BLOCK / 16; ++kk)  // dQ_i = dS K_j (M = queries, K = keys)
-          mma_bf16_ss(tdPt, sdesc_mnmajor_sw128(ds_addr + kk * 2048, PANEL_BYTES),
-                      sdesc_mnmajor_sw128(k_addr + kk * 2048, PANEL_BYTES), IDESC_DQ,
-                      kk > 0 ? 1u : 0u);
+          mma_bf16_ss(tdPt, dsdM + moff(kk), kdM + moff(kk), IDESC_DQ, kk > 0 ? 1u : 0u);
         mma_commit(dq_full);
         mma_commit(&qd_empty[st]);
       }

@@ -19,8 +19,10 @@
 //              max m and sum l (log2 domain), writes P as bf16 into the same
 //              tensor-memory columns, rescales its O when m grows, and finally
 //              writes O / l and LSE.
-//   warp 8     TMA producer: Q_0 and Q_1 once, then K_j and V_j through an
-//              NS-stage ring shared by both query tiles.
+//   warp 8     TMA producer: the query pair of each work item, then K_j and
+//              V_j through one ring of NSLOT tile-sized slots that holds K and
+//              V tiles in the order they are consumed (K_0 V_0 K_1 V_1 ...), so
+//              loads run about two key tiles ahead of the tensor core.
 //   warp 9     tensor-memory allocator and MMA issuer (one thread).  The two
 //              query tiles ping-pong: while warpgroup 0 exponentiates S_0,j the
 //              tensor core runs O_1 += P_1 V_{j-1} and S_1,j, and vice versa:
@@ -63,14 +65,13 @@ template <int D>
 struct Smem {
   static constexpr int NPANEL = D / 64;
   static constexpr int TILE = NPANEL * PANEL_BYTES;  // 128 rows x D bf16
-  static constexpr int NS = 2;                       // K/V ring depth
+  static constexpr int NSLOT = 5;                    // K/V ring slots
   static constexpr int Q_OFF = 0;                    // NQ tiles
-  static constexpr int K_OFF = NQ * TILE;
-  static constexpr int V_OFF = K_OFF + NS * TILE;
-  static constexpr int BAR_OFF = V_OFF + NS * TILE;
-  // barriers: q_full, q_empty, k_full[NS], v_full[NS], k_empty[NS], v_empty[NS],
+  static constexpr int RING_OFF = NQ * TILE;
+  static constexpr int BAR_OFF = RING_OFF + NSLOT * TILE;
+  // barriers: q_full, q_empty, full[NSLOT], empty[NSLOT],
   //           s_full[NQ], p_full[NQ], o_done[NQ], o_final[NQ], o_free[NQ], mma_final
-  static constexpr int NBAR = 2 + 4 * NS + 5 * NQ + 1;
+  static constexpr int NBAR = 2 + 2 * NSLOT + 5 * NQ + 1;
   static constexpr int MISC_OFF = BAR_OFF + NBAR * 8;
   static constexpr int BYTES = MISC_OFF + 16;
   // at least 116 KB so that a single CTA (and its 512 tensor-memory columns)
@@ -116,7 +117,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                   const __grid_constant__ CUtensorMap tm_k,
                   const __grid_constant__ CUtensorMap tm_v, const Params p) {
   using L = Smem<D>;
-  constexpr int NS = L::NS;
+  constexpr int NSLOT = L::NSLOT;
   extern __shared__ __align__(1024) uint8_t smem[];
   // The swizzled operand tiles need 1024-byte alignment; the kernel declares
   // no static shared memory, so the dynamic window starts aligned.
@@ -128,11 +129,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::BAR_OFF);
   uint64_t* q_full = bars;
   uint64_t* q_empty = bars + 1;
-  uint64_t* k_full = bars + 2;
-  uint64_t* v_full = k_full + NS;
-  uint64_t* k_empty = v_full + NS;
-  uint64_t* v_empty = k_empty + NS;
-  uint64_t* s_full = v_empty + NS;  // [NQ]
+  uint64_t* full = bars + 2;        // [NSLOT] ring slot loaded
+  uint64_t* empty = full + NSLOT;   // [NSLOT] ring slot consumed
+  uint64_t* s_full = empty + NSLOT; // [NQ]
   uint64_t* p_full = s_full + NQ;   // [NQ]
   uint64_t* o_done = p_full + NQ;   // [NQ] one phase per O += P V
   uint64_t* o_final = o_done + NQ;  // [NQ] one phase per work item: its last O += P V
@@ -155,11 +154,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
     mbar_init(q_empty, 1);
-    for (int s = 0; s < NS; ++s) {
-      mbar_init(&k_full[s], 1);
-      mbar_init(&v_full[s], 1);
-      mbar_init(&k_empty[s], 1);
-      mbar_init(&v_empty[s], 1);
+    for (int s = 0; s < NSLOT; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
     }
     for (int w = 0; w < NQ; ++w) {
       mbar_init(&s_full[w], 1);
@@ -189,8 +186,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   if (warp == 8) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
-      int kv = 0;        // K/V tiles loaded so far (all work items)
-      int n_items = 0;   // Q pairs loaded so far
+      int kv = 0;        // key tiles loaded so far (all work items)
+      int loaded = 0;    // ring tiles (K or V) loaded so far
+      int n_items = 0;   // query pairs loaded so far
       bool ok = true;
       for (int k = 0; ok; ++k) {
         const int item = cta_item(cta, k, G);
@@ -206,33 +204,28 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             tma_load_3d(smem + L::Q_OFF + w * L::TILE + pn * PANEL_BYTES, &tm_q, q_full,
                         pn * 64, tile * BLOCK_M + w * TILE_M, bh);
         ++n_items;
-        for (int j = 0; j < n_kv1; ++j, ++kv) {
-          const int st = kv % NS;
-          const int r = kv / NS;
-          if (kv >= NS && !mbar_wait(&k_empty[st], (r - 1) & 1, abort_flag)) { ok = false; break; }
-          mbar_arrive_expect_tx(&k_full[st], L::TILE);
-          for (int pn = 0; pn < L::NPANEL; ++pn)
-            tma_load_3d(smem + L::K_OFF + st * L::TILE + pn * PANEL_BYTES, &tm_k, &k_full[st],
-                        pn * 64, j * BLOCK_N, bh);
-          if (kv >= NS && !mbar_wait(&v_empty[st], (r - 1) & 1, abort_flag)) {
-            // K of this tile is in flight: count it so that it is drained
-            mbar_wait_drain(&k_full[st], r & 1);
-            ok = false;
-            break;
+        for (int j = 0; j < n_kv1 && ok; ++j, ++kv) {
+          // K_kv is ring tile 2 kv, V_kv is ring tile 2 kv + 1
+          for (int half = 0; half < 2; ++half) {
+            const int u = 2 * kv + half;
+            const int slot = u % NSLOT;
+            if (u >= NSLOT && !mbar_wait(&empty[slot], (u / NSLOT - 1) & 1, abort_flag)) {
+              ok = false;
+              break;
+            }
+            mbar_arrive_expect_tx(&full[slot], L::TILE);
+            for (int pn = 0; pn < L::NPANEL; ++pn)
+              tma_load_3d(smem + L::RING_OFF + slot * L::TILE + pn * PANEL_BYTES,
+                          half ? &tm_v : &tm_k, &full[slot], pn * 64, j * BLOCK_N, bh);
+            ++loaded;
           }
-          mbar_arrive_expect_tx(&v_full[st], L::TILE);
-          for (int pn = 0; pn < L::NPANEL; ++pn)
-            tma_load_3d(smem + L::V_OFF + st * L::TILE + pn * PANEL_BYTES, &tm_v, &v_full[st],
-                        pn * 64, j * BLOCK_N, bh);
         }
       }
       // Every copy issued must land before this CTA's shared memory is freed:
       // the last phase of each barrier that received copies.
       if (n_items > 0) mbar_wait_drain(q_full, (n_items - 1) & 1);
-      for (int g = max(0, kv - NS); g < kv; ++g) {
-        mbar_wait_drain(&k_full[g % NS], (g / NS) & 1);
-        mbar_wait_drain(&v_full[g % NS], (g / NS) & 1);
-      }
+      for (int u = max(0, loaded - NSLOT); u < loaded; ++u)
+        mbar_wait_drain(&full[u % NSLOT], (u / NSLOT) & 1);
     }
   } else if (warp == 9) {
     // ------------------------------------------------------------ MMA issuer
@@ -240,20 +233,26 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       constexpr uint32_t IDESC_S = idesc_bf16_f32(TILE_M, BLOCK_N, false, false);
       constexpr uint32_t IDESC_O = idesc_bf16_f32(TILE_M, D, false, true);
       const uint32_t q_addr = smem_u32(smem + L::Q_OFF);
-      const uint32_t k_addr = smem_u32(smem + L::K_OFF);
-      const uint32_t v_addr = smem_u32(smem + L::V_OFF);
+      const uint32_t ring_addr = smem_u32(smem + L::RING_OFF);
       int pcount[NQ] = {0, 0};  // P tiles consumed per warpgroup (all items)
 
       // S_w = Q_w K^T with K in ring slot `slot`
+      // Shared-memory descriptors are built once; a k-step only adds a
+      // compile-time byte offset (>> 4) to the start-address field, which
+      // never carries out of its 14 bits for addresses below 256 KB.  This
+      // keeps the issue loop at a few instructions per MMA: the MMA warp
+      // shares its scheduler with two busy softmax warps.
+      const uint64_t q_desc0 = sdesc_kmajor_sw128(q_addr);
+      const uint64_t ring_kdesc0 = sdesc_kmajor_sw128(ring_addr);
+      const uint64_t ring_vdesc0 = sdesc_mnmajor_sw128(ring_addr, PANEL_BYTES);
       auto issue_s = [&](int w, int slot) {
-        const uint32_t kbase = k_addr + slot * L::TILE;
-        const uint32_t qbase = q_addr + w * L::TILE;
+        const uint64_t qd = q_desc0 + static_cast<uint64_t>((w * L::TILE) >> 4);
+        const uint64_t kd = ring_kdesc0 + static_cast<uint64_t>((slot * L::TILE) >> 4);
         const uint32_t dS = tmem_base + w * 128;
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * PANEL_BYTES + (kk & 3) * 32;
-          mma_bf16_ss(dS, sdesc_kmajor_sw128(qbase + off), sdesc_kmajor_sw128(kbase + off),
-                      IDESC_S, kk > 0 ? 1u : 0u);
+          const uint64_t off = static_cast<uint64_t>(((kk >> 2) * PANEL_BYTES + (kk & 3) * 32) >> 4);
+          mma_bf16_ss(dS, qd + off, kd + off, IDESC_S, kk > 0 ? 1u : 0u);
         }
         mma_commit(&s_full[w]);
       };
@@ -262,21 +261,25 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         if (!mbar_wait(&p_full[w], pcount[w] & 1, abort_flag)) return false;
         ++pcount[w];
         tc_fence_after();
-        const uint32_t vbase = v_addr + slot * L::TILE;
+        const uint64_t vd = ring_vdesc0 + static_cast<uint64_t>((slot * L::TILE) >> 4);
         const uint32_t tP = tmem_base + w * 128;
         const uint32_t tO = tmem_base + 256 + w * 128;
 #pragma unroll
         for (int kk = 0; kk < BLOCK_N / 16; ++kk) {
           // keys 16kk .. 16kk+15: P columns 8kk.., V rows 16kk.. (2048 bytes per step)
-          const uint64_t bdesc = sdesc_mnmajor_sw128(vbase + kk * 2048, PANEL_BYTES);
-          mma_bf16_ts(tO, tP + kk * 8, bdesc, IDESC_O, (!first || kk > 0) ? 1u : 0u);
+          mma_bf16_ts(tO, tP + kk * 8, vd + static_cast<uint64_t>((kk * 2048) >> 4), IDESC_O,
+                      (!first || kk > 0) ? 1u : 0u);
         }
         mma_commit(&o_done[w]);
         if (last) mma_commit(&o_final[w]);
         return true;
       };
 
-      int kv = 0;  // K/V tiles consumed so far (all work items)
+      int kv = 0;  // key tiles consumed so far (all work items)
+      auto kslot = [&](int g) { return (2 * g) % NSLOT; };
+      auto vslot = [&](int g) { return (2 * g + 1) % NSLOT; };
+      auto kwait = [&](int g) { return mbar_wait(&full[kslot(g)], ((2 * g) / NSLOT) & 1, abort_flag); };
+      auto vwait = [&](int g) { return mbar_wait(&full[vslot(g)], ((2 * g + 1) / NSLOT) & 1, abort_flag); };
       bool ok = true;
       for (int k = 0; ok; ++k) {
         const int item = cta_item(cta, k, G);
@@ -285,35 +288,33 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         item_coords(p, item, bh, tile);
         const int n0 = n_kv_of(tile, 0);
         const int n1 = n_kv_of(tile, 1);
-        if (!mbar_wait(q_full, k & 1, abort_flag) ||
-            !mbar_wait(&k_full[kv % NS], (kv / NS) & 1, abort_flag)) { ok = false; break; }
+        if (!mbar_wait(q_full, k & 1, abort_flag) || !kwait(kv)) { ok = false; break; }
         tc_fence_after();
-        issue_s(0, kv % NS);
-        issue_s(1, kv % NS);
-        mma_commit(&k_empty[kv % NS]);
+        issue_s(0, kslot(kv));
+        issue_s(1, kslot(kv));
+        mma_commit(&empty[kslot(kv)]);
         if (n1 == 1) mma_commit(q_empty);
         for (int j = 0; j < n1; ++j) {
           const int g = kv + j;
-          const int st = g % NS;
           const bool more = j + 1 < n1;
-          if (!mbar_wait(&v_full[st], (g / NS) & 1, abort_flag)) { ok = false; break; }
+          if (!vwait(g)) { ok = false; break; }
           if (j < n0) {
             // the first product of an item overwrites O_0: its read-out by the
             // previous item's epilogue must be complete
             if (j == 0 && k > 0 && !mbar_wait(&o_free[0], (k - 1) & 1, abort_flag)) { ok = false; break; }
-            if (!issue_pv(0, st, j == 0, j == n0 - 1)) { ok = false; break; }
+            if (!issue_pv(0, vslot(g), j == 0, j == n0 - 1)) { ok = false; break; }
           }
           if (more) {
-            if (!mbar_wait(&k_full[(g + 1) % NS], ((g + 1) / NS) & 1, abort_flag)) { ok = false; break; }
+            if (!kwait(g + 1)) { ok = false; break; }
             tc_fence_after();
-            if (j + 1 < n0) issue_s(0, (g + 1) % NS);
+            if (j + 1 < n0) issue_s(0, kslot(g + 1));
           }
           if (j == 0 && k > 0 && !mbar_wait(&o_free[1], (k - 1) & 1, abort_flag)) { ok = false; break; }
-          if (!issue_pv(1, st, j == 0, j == n1 - 1)) { ok = false; break; }
-          mma_commit(&v_empty[st]);
+          if (!issue_pv(1, vslot(g), j == 0, j == n1 - 1)) { ok = false; break; }
+          mma_commit(&empty[vslot(g)]);
           if (more) {
-            issue_s(1, (g + 1) % NS);
-            mma_commit(&k_empty[(g + 1) % NS]);
+            issue_s(1, kslot(g + 1));
+            mma_commit(&empty[kslot(g + 1)]);
             if (j + 2 == n1) mma_commit(q_empty);  // last S of this item issued
           }
         }
