@@ -51,6 +51,7 @@ import numpy as np
 
 __all__ = [
     "softmax_rows",
+    "expand_kv_heads",
     "attention_forward",
     "attention_forward_rows",
     "attention_backward",
@@ -108,17 +109,32 @@ def _row_stats(s: np.ndarray):
     return p, lse
 
 
+def expand_kv_heads(x: np.ndarray, n_heads: int) -> np.ndarray:
+    """Grouped-query attention ("DL101 chapter 9", §3.1 MQA and §3.2 GQA): the
+    query heads are split into groups of H / Hkv consecutive heads and every
+    group shares one key/value head.  Returns x [B, Hkv, L, d] repeated to
+    [B, H, L, d] (query head h reads key/value head h // (H / Hkv))."""
+    hkv = x.shape[-3]
+    if n_heads % hkv:
+        raise ValueError("the number of query heads must be a multiple of the K/V heads")
+    return np.repeat(x, n_heads // hkv, axis=-3)
+
+
 def attention_forward(q: np.ndarray, k: np.ndarray, v: np.ndarray,
                       causal: bool, scale: float):
     """O = softmax(scale * Q K^T [+ causal mask]) V and LSE, per (batch, head).
 
-    Shapes: q [..., Nq, d], k and v [..., Nk, d] (same leading dims).  Returns
+    Shapes: q [..., Nq, d], k and v [..., Nk, d] (same leading dims; with
+    [B, H, N, d] queries, k and v may carry fewer heads Hkv dividing H, which
+    grouped-query attention shares between groups of query heads).  Returns
     o [..., Nq, d] and lse [..., Nq], both float64.
 
     "Flash Attention: principle & practice", §1.2 (S = QK^T * scale,
     P = softmax(S), O = PV); "DL101 chapter 9", §1.1 (causal: K_{<=t}).
     """
     _check_f64(q, k, v)
+    if q.ndim == 4 and k.ndim == 4 and k.shape[1] != q.shape[1]:
+        k, v = expand_kv_heads(k, q.shape[1]), expand_kv_heads(v, q.shape[1])
     if causal and q.shape[-2] != k.shape[-2]:
         raise ValueError("causal attention is defined here for Nq == Nk only")
     lead = q.shape[:-2]
@@ -164,10 +180,20 @@ def attention_backward(q: np.ndarray, k: np.ndarray, v: np.ndarray,
         dS = P * (dP - D)          (zero where masked, since P is zero there)
         dQ = scale * dS K
         dK = scale * dS^T Q
-    Shapes as in ``attention_forward`` (Nq == Nk when causal).  Returns
-    (dq, dk, dv, D) with D = the row term above, float64.
+    Shapes as in ``attention_forward`` (Nq == Nk when causal).  With grouped
+    K/V heads the gradient of a shared head is the sum over its group of
+    query heads.  Returns (dq, dk, dv, D) with D = the row term above,
+    float64.
     """
     _check_f64(q, k, v, do)
+    if q.ndim == 4 and k.ndim == 4 and k.shape[1] != q.shape[1]:
+        H, hkv = q.shape[1], k.shape[1]
+        dq, dk, dv, D = attention_backward(q, expand_kv_heads(k, H), expand_kv_heads(v, H),
+                                           do, causal, scale)
+        g = H // hkv
+        dk = dk.reshape(dk.shape[0], hkv, g, *dk.shape[2:]).sum(axis=2)
+        dv = dv.reshape(dv.shape[0], hkv, g, *dv.shape[2:]).sum(axis=2)
+        return dq, dk, dv, D
     if causal and q.shape[-2] != k.shape[-2]:
         raise ValueError("causal attention is defined here for Nq == Nk only")
     lead = q.shape[:-2]
@@ -201,12 +227,16 @@ def decode_forward(q: np.ndarray, kcache: np.ndarray, vcache: np.ndarray,
 
     "DL101 chapter 9", §1.1: the newest query attends the cached keys and
     values of positions 0 .. L_b - 1 (non-causal within the prefix).
-    q [B, H, d]; kcache, vcache [B, H, Lmax, d]; seqlens [B] with
+    q [B, H, d]; kcache, vcache [B, H, Lmax, d] (or [B, Hkv, Lmax, d], key/
+    value heads shared by groups of H / Hkv query heads); seqlens [B] with
     0 <= L_b <= Lmax.  Cache rows at or beyond L_b are never read (they may
     hold anything, NaN included).  Returns o [B, H, d], lse [B, H]; a
     sequence with L_b == 0 gives o = 0, lse = -inf.
     """
     _check_f64(q, kcache, vcache)
+    if kcache.shape[1] != q.shape[1]:
+        kcache = expand_kv_heads(kcache, q.shape[1])
+        vcache = expand_kv_heads(vcache, q.shape[1])
     B, H, d = q.shape
     o = np.zeros((B, H, vcache.shape[-1]))
     lse = np.full((B, H), -np.inf)

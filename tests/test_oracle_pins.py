@@ -373,3 +373,42 @@ def _mutant_bwd(kind):
 def test_pins_reject_planted_backward_mistakes(kind):
     with pytest.raises(AssertionError):
         pin_finite_differences(_mutant_bwd(kind))
+
+
+def test_grouped_query_attention_matches_sdpa_enable_gqa():
+    """"DL101 chapter 9", §3.1-3.2 compute MQA / GQA with torch SDPA's
+    enable_gqa; the oracle's grouped heads must agree with that routine."""
+    for hkv in (1, 2, 4):
+        for causal in (False, True):
+            q = bf16_grid((2, 8, 40, 16))
+            k, v = bf16_grid((2, hkv, 40, 16)), bf16_grid((2, hkv, 40, 16))
+            o, lse = A.attention_forward(q, k, v, causal, 0.3)
+            ref = torch.nn.functional.scaled_dot_product_attention(
+                *(torch.from_numpy(x) for x in (q, k, v)), is_causal=causal, scale=0.3,
+                enable_gqa=True).numpy()
+            assert np.allclose(o, ref, atol=1e-12)
+
+
+def test_grouped_query_backward_matches_autograd():
+    for hkv in (1, 2):
+        q, do = bf16_grid((1, 4, 24, 8)), bf16_grid((1, 4, 24, 8))
+        k, v = bf16_grid((1, hkv, 24, 8)), bf16_grid((1, hkv, 24, 8))
+        tq, tk, tv = (torch.from_numpy(x).requires_grad_() for x in (q, k, v))
+        o = torch.nn.functional.scaled_dot_product_attention(tq, tk, tv, is_causal=True, scale=0.4,
+                                                             enable_gqa=True)
+        o.backward(torch.from_numpy(do))
+        dq, dk, dv, _ = A.attention_backward(q, k, v, do, True, 0.4)
+        for a, b in ((dq, tq.grad), (dk, tk.grad), (dv, tv.grad)):
+            assert a.shape == b.shape and np.allclose(a, b.numpy(), atol=1e-11)
+
+
+def test_grouped_decode_matches_expanded_cache():
+    q = bf16_grid((2, 6, 8))
+    kc, vc = bf16_grid((2, 3, 30, 8)), bf16_grid((2, 3, 30, 8))
+    o, lse = A.decode_forward(q, kc, vc, [30, 11], 0.5)
+    for b, L in enumerate([30, 11]):
+        for h in range(6):
+            ref = torch.nn.functional.scaled_dot_product_attention(
+                torch.from_numpy(q[b, h][None, None]), torch.from_numpy(kc[b, h // 2, :L][None]),
+                torch.from_numpy(vc[b, h // 2, :L][None]), scale=0.5)
+            assert np.allclose(o[b, h], ref[0, 0].numpy(), atol=1e-13)
