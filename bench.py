@@ -146,8 +146,8 @@ class ClockSampler:
 
 # ----------------------------------------------------------------------------- workloads
 def workload_config(w, parallelism):
-    return {"workload": w.name, "B": w.B, "H": w.H, "N": w.N or None, "d": w.d,
-            "causal": w.causal, "parallelism": parallelism}
+    return {"workload": w.name, "B": w.B, "H": w.H, "Hkv": w.kv_heads, "N": w.N or None,
+            "d": w.d, "causal": w.causal, "parallelism": parallelism}
 
 
 def fwd_flops(w):
@@ -156,7 +156,8 @@ def fwd_flops(w):
 
 
 def decode_bytes(w, seqlens):
-    return float(sum(int(L) for L in seqlens)) * w.H * w.d * 2 * 2
+    """Algorithmic KV bytes: every cached key and value row read once."""
+    return float(sum(int(L) for L in seqlens)) * w.kv_heads * w.d * 2 * 2
 
 
 class Runner:
@@ -179,7 +180,7 @@ class Runner:
         elif w.kind == "bwd":
             q, k, v, do = self.dbuf
             self.o, self.lse = fa.fwd(q, k, v, causal=w.causal, scale=w.scale)
-            self.dq, self.dk, self.dv = (torch.empty_like(q) for _ in range(3))
+            self.dq, self.dk, self.dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
             self.ws = torch.empty(fa.bwd_workspace_size(w.B, w.H, w.N, w.d), dtype=torch.uint8,
                                   device=dev)
             self.work = 2.5 * fwd_flops(w)
@@ -308,7 +309,7 @@ def run_reference(args, w, total_budget=150.0, emit=True):
         heads = [(b, h) for b in range(w.B) for h in range(w.H)]
         # rows per step sized from a probe so that a step stays within budget
         b0, h0 = heads[0]
-        qh, kh, vh = f64(q[b0, h0]), f64(k[b0, h0]), f64(v[b0, h0])
+        qh, kh, vh = f64(q[b0, h0]), f64(k[b0, 0]), f64(v[b0, 0])
         t0 = time.perf_counter()
         oracle.attention_forward_rows(qh, kh, vh, w.causal, w.scale, np.arange(min(64, w.N)))
         per_row = (time.perf_counter() - t0) / min(64, w.N)
@@ -316,10 +317,12 @@ def run_reference(args, w, total_budget=150.0, emit=True):
         sample = f"{rows_per_step} query rows of one (batch, head) per step, rows drawn uniformly"
         mult = 3.5 if w.kind == "bwd" else 1.0  # bwd oracle is not timed; fwd rows scaled
 
+        group = w.H // w.kv_heads
+
         def step(i):
             b, h = heads[i % len(heads)]
             rows = np.sort(rng.integers(0, w.N, rows_per_step))
-            qh, kh, vh = f64(q[b, h]), f64(k[b, h]), f64(v[b, h])
+            qh, kh, vh = f64(q[b, h]), f64(k[b, h // group]), f64(v[b, h // group])
             t = time.perf_counter()
             oracle.attention_forward_rows(qh, kh, vh, w.causal, w.scale, rows)
             dt = time.perf_counter() - t
@@ -335,7 +338,8 @@ def run_reference(args, w, total_budget=150.0, emit=True):
             b = i % w.B
             h = (i // w.B) % w.H
             L = int(sl[b])
-            qq, kk, vv = f64(q[b:b + 1, h:h + 1]), f64(kc[b:b + 1, h:h + 1, :L]), f64(vc[b:b + 1, h:h + 1, :L])
+            hk = h // (w.H // w.kv_heads)
+            qq, kk, vv = f64(q[b:b + 1, h:h + 1]), f64(kc[b:b + 1, hk:hk + 1, :L]), f64(vc[b:b + 1, hk:hk + 1, :L])
             t = time.perf_counter()
             oracle.decode_forward(qq, kk, vv, [L], w.scale)
             return time.perf_counter() - t, float(L) * w.d * 4, 1.0

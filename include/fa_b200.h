@@ -69,6 +69,16 @@ fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* ls
                  fa_stream_t stream);
 
 /*
+ * Grouped-query forward ("DL101 chapter 9", sections 3.1 MQA and 3.2 GQA):
+ * k and v are bf16 [B, Hkv, N, d] and query head h of batch b attends key /
+ * value head h / (H / Hkv) of that batch.  Hkv must divide H; Hkv = H is
+ * fa_fwd, Hkv = 1 multi-query attention.  Everything else as fa_fwd.
+ */
+fa_status fa_fwd_gqa(const void* q, const void* k, const void* v, void* o, float* lse,
+                     int B, int H, int Hkv, int N, int d, int causal, float scale,
+                     fa_stream_t stream);
+
+/*
  * Bytes of device workspace fa_bwd needs: D = rowsum(dO * O) and
  * log2(e) * LSE as float32 [B, H, Np] with Np = N rounded up to a multiple
  * of 128, followed by the float32 dQ accumulator [B, H, N, d], each region
@@ -96,6 +106,17 @@ fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o,
                  void* workspace, size_t ws_bytes,
                  int B, int H, int N, int d, int causal, float scale,
                  fa_stream_t stream);
+
+/*
+ * Grouped-query backward: k, v, dk, dv are [B, Hkv, N, d]; the gradient of a
+ * shared key / value head is the sum over its H / Hkv query heads.  The
+ * workspace is fa_bwd_workspace_size(B, H, N, d).  Everything else as fa_bwd.
+ */
+fa_status fa_bwd_gqa(const void* q, const void* k, const void* v, const void* o,
+                     const void* dout, const float* lse, void* dq, void* dk, void* dv,
+                     void* workspace, size_t ws_bytes,
+                     int B, int H, int Hkv, int N, int d, int causal, float scale,
+                     fa_stream_t stream);
 
 /*
  * Bytes of device workspace fa_decode needs for the split-KV partials
@@ -128,6 +149,16 @@ fa_status fa_decode(const void* q, const void* kcache, const void* vcache,
                     const int* seqlens, void* o, float* lse,
                     int B, int H, int Lmax, int d, float scale,
                     void* workspace, size_t ws_bytes, fa_stream_t stream);
+
+/*
+ * Grouped-query decode: kcache and vcache are [B, Hkv, Lmax, d] and query
+ * head h reads cache head h / (H / Hkv).  The workspace is
+ * fa_decode_workspace_size(B, H, Lmax, d).  Everything else as fa_decode.
+ */
+fa_status fa_decode_gqa(const void* q, const void* kcache, const void* vcache,
+                        const int* seqlens, void* o, float* lse,
+                        int B, int H, int Hkv, int Lmax, int d, float scale,
+                        void* workspace, size_t ws_bytes, fa_stream_t stream);
 
 /*
  * Size in bytes of the device array that fa_decode_static uses as scratch

@@ -127,8 +127,14 @@ int fa_version(void) { return 100; }
 
 fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
                  int N, int d, int causal, float scale, fa_stream_t stream) {
+  return fa_fwd_gqa(q, k, v, o, lse, B, H, H, N, d, causal, scale, stream);
+}
+
+fa_status fa_fwd_gqa(const void* q, const void* k, const void* v, void* o, float* lse, int B,
+                     int H, int Hkv, int N, int d, int causal, float scale, fa_stream_t stream) {
   fa_status st = check_shape(B, H, N, d);
   if (st != FA_OK) return st;
+  if (Hkv < 1 || H % Hkv != 0) return FA_ERR_INVALID_ARG;
   if (!q || !k || !v || !o) return FA_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o)) return FA_ERR_INVALID_ARG;
   if (lse != nullptr && (reinterpret_cast<uintptr_t>(lse) & 3u)) return FA_ERR_INVALID_ARG;
@@ -136,7 +142,7 @@ fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* ls
   if (!(scale == scale)) return FA_ERR_INVALID_ARG;  // NaN
   if ((st = check_device()) != FA_OK) return st;
   if (N == 0) return FA_OK;
-  return launch_fwd(q, k, v, o, lse, B, H, N, d, causal, scale,
+  return launch_fwd(q, k, v, o, lse, B, H, Hkv, N, d, causal, scale,
                     reinterpret_cast<cudaStream_t>(stream));
 }
 
@@ -153,8 +159,17 @@ fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, con
                  const float* lse, void* dq, void* dk, void* dv, void* workspace,
                  size_t ws_bytes, int B, int H, int N, int d, int causal, float scale,
                  fa_stream_t stream) {
+  return fa_bwd_gqa(q, k, v, o, dout, lse, dq, dk, dv, workspace, ws_bytes, B, H, H, N, d, causal,
+                    scale, stream);
+}
+
+fa_status fa_bwd_gqa(const void* q, const void* k, const void* v, const void* o,
+                     const void* dout, const float* lse, void* dq, void* dk, void* dv,
+                     void* workspace, size_t ws_bytes, int B, int H, int Hkv, int N, int d,
+                     int causal, float scale, fa_stream_t stream) {
   fa_status st = check_shape(B, H, N, d);
   if (st != FA_OK) return st;
+  if (Hkv < 1 || H % Hkv != 0) return FA_ERR_INVALID_ARG;
   if (!q || !k || !v || !o || !dout || !lse || !dq || !dk || !dv) return FA_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(dout) ||
       !aligned16(dq) || !aligned16(dk) || !aligned16(dv) ||
@@ -167,7 +182,7 @@ fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, con
     return FA_ERR_WORKSPACE;
   if ((st = check_device()) != FA_OK) return st;
   if (N == 0) return FA_OK;
-  return launch_bwd(q, k, v, o, dout, lse, dq, dk, dv, workspace, B, H, N, d, causal, scale,
+  return launch_bwd(q, k, v, o, dout, lse, dq, dk, dv, workspace, B, H, Hkv, N, d, causal, scale,
                     reinterpret_cast<cudaStream_t>(stream));
 }
 
@@ -181,7 +196,15 @@ size_t fa_decode_workspace_size(int B, int H, int Lmax, int d) {
 fa_status fa_decode(const void* q, const void* kcache, const void* vcache, const int* seqlens,
                     void* o, float* lse, int B, int H, int Lmax, int d, float scale,
                     void* workspace, size_t ws_bytes, fa_stream_t stream) {
+  return fa_decode_gqa(q, kcache, vcache, seqlens, o, lse, B, H, H, Lmax, d, scale, workspace,
+                       ws_bytes, stream);
+}
+
+fa_status fa_decode_gqa(const void* q, const void* kcache, const void* vcache, const int* seqlens,
+                        void* o, float* lse, int B, int H, int Hkv, int Lmax, int d, float scale,
+                        void* workspace, size_t ws_bytes, fa_stream_t stream) {
   if (B < 1 || H < 1 || Lmax < 0) return FA_ERR_INVALID_ARG;
+  if (Hkv < 1 || H % Hkv != 0) return FA_ERR_INVALID_ARG;
   if (static_cast<long long>(B) * H > INT_MAX) return FA_ERR_INVALID_ARG;
   if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
   if (!q || !kcache || !vcache || !seqlens || !o) return FA_ERR_INVALID_ARG;
@@ -195,7 +218,7 @@ fa_status fa_decode(const void* q, const void* kcache, const void* vcache, const
     return FA_ERR_WORKSPACE;
   fa_status st = check_device();
   if (st != FA_OK) return st;
-  return launch_decode(q, kcache, vcache, seqlens, o, lse, B, H, Lmax, d, scale,
+  return launch_decode(q, kcache, vcache, seqlens, o, lse, B, H, Hkv, Lmax, d, scale,
                        static_cast<float*>(workspace), reinterpret_cast<cudaStream_t>(stream));
 }
 

@@ -71,6 +71,7 @@ struct Params {
   float* dqacc;
   int N;
   int n_tiles;
+  int group;         // query heads per key/value head (1 without grouping)
   float scale_log2;  // scale * log2(e)
   float scale;
 };
@@ -120,11 +121,17 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   // One-dimensional grid, head-major: the key tiles of one (batch, head) are
   // adjacent in launch order (so resident CTAs share that head's Q and dO
   // tiles in L2); tile 0, which sees the most query tiles, comes first.
-  const int bh = static_cast<int>(blockIdx.x) / p.n_tiles;
-  const int kv_tile = static_cast<int>(blockIdx.x) - bh * p.n_tiles;
+  // bkv indexes key/value heads; the CTA accumulates dK, dV of key tile
+  // kv_tile over the query tiles of all `group` query heads sharing it.
+  const int bkv = static_cast<int>(blockIdx.x) / p.n_tiles;
+  const int kv_tile = static_cast<int>(blockIdx.x) - bkv * p.n_tiles;
   const int key0 = kv_tile * BLOCK;
   const int i_begin = CAUSAL ? kv_tile : 0;
-  const int n_it = p.n_tiles - i_begin;
+  const int n_per = p.n_tiles - i_begin;  // query tiles per query head
+  const int n_it = n_per * p.group;
+  // iteration it -> (query head, first row of its query tile)
+  auto it_head = [&](int it) { return bkv * p.group + it / n_per; };
+  auto it_q0 = [&](int it) { return (i_begin + it % n_per) * BLOCK; };
 
   if (threadIdx.x == 0) {
     for (int b = 0; b < L::NBAR; ++b) mbar_init(&bars[b], 1);
@@ -155,13 +162,14 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       int last[2] = {-1, -1};
       mbar_arrive_expect_tx(kv_full, 2 * L::TILE);
       for (int pn = 0; pn < L::NPANEL; ++pn) {
-        tma_load_3d(smem + L::K_OFF + pn * PANEL_BYTES, &tm_k, kv_full, pn * 64, key0, bh);
-        tma_load_3d(smem + L::V_OFF + pn * PANEL_BYTES, &tm_v, kv_full, pn * 64, key0, bh);
+        tma_load_3d(smem + L::K_OFF + pn * PANEL_BYTES, &tm_k, kv_full, pn * 64, key0, bkv);
+        tma_load_3d(smem + L::V_OFF + pn * PANEL_BYTES, &tm_v, kv_full, pn * 64, key0, bkv);
       }
       for (int it = 0; it < n_it; ++it) {
         const int st = it & 1;
         const int r = it >> 1;
-        const int q0 = (i_begin + it) * BLOCK;
+        const int q0 = it_q0(it);
+        const int bh = it_head(it);
         if (it >= 2 && !mbar_wait(&qd_empty[st], (r - 1) & 1, abort_flag)) break;
         mbar_arrive_expect_tx(&qd_full[st], 2 * L::TILE + 1024);
         for (int pn = 0; pn < L::NPANEL; ++pn) {
@@ -257,7 +265,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     bool ok = true;
     for (int it = 0; it < n_it; ++it) {
       const int st = it & 1;
-      const int q0 = (i_begin + it) * BLOCK;
+      const int q0 = it_q0(it);
       if (!mbar_wait_warp(st_full, it & 1, abort_flag) ||
           !mbar_wait_warp(dpt_full, it & 1, abort_flag)) {
         ok = false;
@@ -316,7 +324,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     // epilogue: warpgroup 0 writes dV, warpgroup 1 scale * dK, one key row per thread
     if (ok && mbar_wait_warp(dkv_final, 0, abort_flag)) {
       tc_fence_after();
-      const size_t rowoff = (static_cast<size_t>(bh) * p.N + key_g) * D;
+      const size_t rowoff = (static_cast<size_t>(bkv) * p.N + key_g) * D;
       {
         const int which = g;
         const uint32_t tacc = which == 0 ? tdV : tdK;
@@ -358,7 +366,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     int rounds = 0;  // staging rounds so far
     bool ok = true;
     for (int it = 0; ok && it < n_it; ++it) {
-      const int q0 = (i_begin + it) * BLOCK;
+      const int q0 = it_q0(it);
+      const int bh = it_head(it);
       if (!mbar_wait_warp(dq_full, it & 1, abort_flag)) break;
       tc_fence_after();
 #pragma unroll 1
@@ -483,9 +492,10 @@ fa_status launch_main(const CUtensorMap* maps, const Params& prm, int BH, cudaSt
 
 fa_status launch_bwd(const void* q, const void* k, const void* v, const void* o,
                      const void* dout, const float* lse, void* dq, void* dk, void* dv,
-                     void* workspace, int B, int H, int N, int d, int causal, float scale,
-                     cudaStream_t stream) {
+                     void* workspace, int B, int H, int Hkv, int N, int d, int causal,
+                     float scale, cudaStream_t stream) {
   const int BH = B * H;
+  const int BHkv = B * Hkv;
   const long long rows = static_cast<long long>(BH) * N;
   const int Np = static_cast<int>(bwd_row_pad(N));
   const long long prows = static_cast<long long>(BH) * Np;
@@ -511,8 +521,8 @@ fa_status launch_bwd(const void* q, const void* k, const void* v, const void* o,
   CUtensorMap maps[7];
   fa_status st;
   if ((st = make_tmap_bf16_3d(&maps[0], q, d, N, BH, bwd::BLOCK)) != FA_OK) return st;
-  if ((st = make_tmap_bf16_3d(&maps[1], k, d, N, BH, bwd::BLOCK)) != FA_OK) return st;
-  if ((st = make_tmap_bf16_3d(&maps[2], v, d, N, BH, bwd::BLOCK)) != FA_OK) return st;
+  if ((st = make_tmap_bf16_3d(&maps[1], k, d, N, BHkv, bwd::BLOCK)) != FA_OK) return st;
+  if ((st = make_tmap_bf16_3d(&maps[2], v, d, N, BHkv, bwd::BLOCK)) != FA_OK) return st;
   if ((st = make_tmap_bf16_3d(&maps[3], dout, d, N, BH, bwd::BLOCK)) != FA_OK) return st;
   if ((st = make_tmap_f32_2d(&maps[4], lse2, Np, BH)) != FA_OK) return st;
   if ((st = make_tmap_f32_2d(&maps[5], dd, Np, BH)) != FA_OK) return st;
@@ -523,14 +533,15 @@ fa_status launch_bwd(const void* q, const void* k, const void* v, const void* o,
   prm.dqacc = dqacc;
   prm.N = N;
   prm.n_tiles = (N + bwd::BLOCK - 1) / bwd::BLOCK;
+  prm.group = H / Hkv;
   prm.scale_log2 = scale * bwd::LOG2E;
   prm.scale = scale;
   if (d == 128)
-    st = causal ? bwd::launch_main<128, true>(maps, prm, BH, stream)
-                : bwd::launch_main<128, false>(maps, prm, BH, stream);
+    st = causal ? bwd::launch_main<128, true>(maps, prm, BHkv, stream)
+                : bwd::launch_main<128, false>(maps, prm, BHkv, stream);
   else
-    st = causal ? bwd::launch_main<64, true>(maps, prm, BH, stream)
-                : bwd::launch_main<64, false>(maps, prm, BH, stream);
+    st = causal ? bwd::launch_main<64, true>(maps, prm, BHkv, stream)
+                : bwd::launch_main<64, false>(maps, prm, BHkv, stream);
   if (st != FA_OK) return st;
   // 3. dQ = scale * accumulator
   {

@@ -49,7 +49,8 @@ __global__ void __launch_bounds__(THREADS)
     fa_decode_split_kernel(const __nv_bfloat16* __restrict__ q,
                            const __nv_bfloat16* __restrict__ kc,
                            const __nv_bfloat16* __restrict__ vc, const int* __restrict__ seqlens,
-                           float* __restrict__ part, int H, int Lmax, int S, float scale_log2) {
+                           float* __restrict__ part, int H, int group, int Lmax, int S,
+                           float scale_log2) {
   constexpr int LPK = D / 8;         // lanes per key
   constexpr int KPW = 32 / LPK;      // keys per warp step
   constexpr int HW = WARPS * KPW;    // key groups per CTA
@@ -75,8 +76,10 @@ __global__ void __launch_bounds__(THREADS)
 #pragma unroll
     for (int e = 0; e < 8; ++e) qf[e] *= scale_log2;
   }
-  const __nv_bfloat16* kbase = kc + bh * static_cast<size_t>(Lmax) * D + sub * 8;
-  const __nv_bfloat16* vbase = vc + bh * static_cast<size_t>(Lmax) * D + sub * 8;
+  // query head bh reads key/value head bh / group (grouped-query attention)
+  const size_t bkv = bh / static_cast<size_t>(group);
+  const __nv_bfloat16* kbase = kc + bkv * static_cast<size_t>(Lmax) * D + sub * 8;
+  const __nv_bfloat16* vbase = vc + bkv * static_cast<size_t>(Lmax) * D + sub * 8;
 
   float m = -INFINITY, l = 0.f, acc[8];
 #pragma unroll
@@ -187,14 +190,14 @@ __global__ void __launch_bounds__(D)
 
 template <int D>
 fa_status launch(const void* q, const void* kc, const void* vc, const int* seqlens, void* o,
-                 float* lse, int B, int H, int Lmax, float scale, float* part,
+                 float* lse, int B, int H, int group, int Lmax, float scale, float* part,
                  cudaStream_t stream) {
   const int S = decode_num_splits(Lmax);
   if (S > 0) {
     dim3 grid(S, H, B);
     fa_decode_split_kernel<D><<<grid, THREADS, 0, stream>>>(
         static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(kc),
-        static_cast<const __nv_bfloat16*>(vc), seqlens, part, H, Lmax, S,
+        static_cast<const __nv_bfloat16*>(vc), seqlens, part, H, group, Lmax, S,
         scale * 1.4426950408889634f);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return FA_ERR_CUDA;
@@ -210,12 +213,13 @@ fa_status launch(const void* q, const void* kc, const void* vc, const int* seqle
 int decode_num_splits(int Lmax) { return (Lmax + dec::CHUNK - 1) / dec::CHUNK; }
 
 fa_status launch_decode(const void* q, const void* kc, const void* vc, const int* seqlens,
-                        void* o, float* lse, int B, int H, int Lmax, int d, float scale,
-                        float* partials, cudaStream_t stream) {
+                        void* o, float* lse, int B, int H, int Hkv, int Lmax, int d,
+                        float scale, float* partials, cudaStream_t stream) {
   if (H > 65535 || B > 65535) return FA_ERR_INVALID_ARG;
+  const int group = H / Hkv;
   if (d == 128)
-    return dec::launch<128>(q, kc, vc, seqlens, o, lse, B, H, Lmax, scale, partials, stream);
-  return dec::launch<64>(q, kc, vc, seqlens, o, lse, B, H, Lmax, scale, partials, stream);
+    return dec::launch<128>(q, kc, vc, seqlens, o, lse, B, H, group, Lmax, scale, partials, stream);
+  return dec::launch<64>(q, kc, vc, seqlens, o, lse, B, H, group, Lmax, scale, partials, stream);
 }
 
 }  // namespace fa

@@ -82,6 +82,6 @@ extern "C" fa_status fa_decode_static(const void* q, const void* kcache, const v
   float* scratch = nullptr;
   const fa_status st = static_scratch(&scratch);
   if (st != FA_OK) return st;
-  return launch_decode(q, kcache, vcache, seqlens, o, lse, B, H, Lmax, d, scale, scratch,
+  return launch_decode(q, kcache, vcache, seqlens, o, lse, B, H, H, Lmax, d, scale, scratch,
                        reinterpret_cast<cudaStream_t>(stream));
 }

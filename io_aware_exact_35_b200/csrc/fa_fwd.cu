@@ -84,6 +84,7 @@ struct Params {
   float* lse;
   int N;
   int BH;
+  int group;         // query heads per key/value head (1 without grouping)
   int n_cta_tiles;   // ceil(N / 256)
   int total_items;   // BH * n_cta_tiles
   int lpt_order;     // 1: all heads' longest tiles first; 0: head-major
@@ -216,7 +217,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             mbar_arrive_expect_tx(&full[slot], L::TILE);
             for (int pn = 0; pn < L::NPANEL; ++pn)
               tma_load_3d(smem + L::RING_OFF + slot * L::TILE + pn * PANEL_BYTES,
-                          half ? &tm_v : &tm_k, &full[slot], pn * 64, j * BLOCK_N, bh);
+                          half ? &tm_v : &tm_k, &full[slot], pn * 64, j * BLOCK_N,
+                          bh / p.group);
             ++loaded;
           }
         }
@@ -512,7 +514,7 @@ int schedule_mode() {
 }  // namespace fwd
 
 fa_status launch_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B,
-                     int H, int N, int d, int causal, float scale, cudaStream_t stream) {
+                     int H, int Hkv, int N, int d, int causal, float scale, cudaStream_t stream) {
   const int BH = B * H;
   const long long n_cta_tiles = (N + fwd::BLOCK_M - 1) / fwd::BLOCK_M;
   const long long items = static_cast<long long>(BH) * n_cta_tiles;
@@ -520,13 +522,16 @@ fa_status launch_fwd(const void* q, const void* k, const void* v, void* o, float
   CUtensorMap tq, tk, tv;
   fa_status st;
   if ((st = make_tmap_bf16_3d(&tq, q, d, N, BH, fwd::TILE_M)) != FA_OK) return st;
-  if ((st = make_tmap_bf16_3d(&tk, k, d, N, BH, fwd::BLOCK_N)) != FA_OK) return st;
-  if ((st = make_tmap_bf16_3d(&tv, v, d, N, BH, fwd::BLOCK_N)) != FA_OK) return st;
+  // K and V carry B * Hkv heads; query head bh reads key/value head bh / (H / Hkv)
+  if ((st = make_tmap_bf16_3d(&tk, k, d, N, static_cast<uint64_t>(B) * Hkv, fwd::BLOCK_N)) != FA_OK)
+    return st;
+  if ((st = make_tmap_bf16_3d(&tv, v, d, N, static_cast<uint64_t>(B) * Hkv, fwd::BLOCK_N)) != FA_OK)
+    return st;
   int dev = 0, sms = 148;
   if (cudaGetDevice(&dev) != cudaSuccess ||
       cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
     return FA_ERR_CUDA;
-  const double kv_bytes = 4.0 * BH * static_cast<double>(N) * d;
+  const double kv_bytes = 4.0 * B * Hkv * static_cast<double>(N) * d;
   const int mode = fwd::schedule_mode();
   bool persistent = causal && items > sms && kv_bytes <= 96.0 * 1024 * 1024;
   int grid = persistent ? sms : static_cast<int>(items);
@@ -542,6 +547,7 @@ fa_status launch_fwd(const void* q, const void* k, const void* v, void* o, float
   prm.lse = lse;
   prm.N = N;
   prm.BH = BH;
+  prm.group = H / Hkv;
   prm.n_cta_tiles = static_cast<int>(n_cta_tiles);
   prm.total_items = static_cast<int>(items);
   prm.lpt_order = persistent ? 1 : 0;

@@ -31,18 +31,19 @@ fa_status make_tmap_f32_3d_sw128(CUtensorMap* map, const void* base, uint64_t d,
 // workspace: N rounded up to whole 128-row tiles.
 inline size_t bwd_row_pad(int N) { return (static_cast<size_t>(N) + 127) / 128 * 128; }
 
+// Hkv = number of key/value heads; H (query heads) is a multiple of it.
 fa_status launch_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B,
-                     int H, int N, int d, int causal, float scale, cudaStream_t stream);
+                     int H, int Hkv, int N, int d, int causal, float scale, cudaStream_t stream);
 
 fa_status launch_bwd(const void* q, const void* k, const void* v, const void* o,
                      const void* dout, const float* lse, void* dq, void* dk, void* dv,
-                     void* workspace, int B, int H, int N, int d, int causal, float scale,
-                     cudaStream_t stream);
+                     void* workspace, int B, int H, int Hkv, int N, int d, int causal,
+                     float scale, cudaStream_t stream);
 
 int decode_num_splits(int Lmax);
 fa_status launch_decode(const void* q, const void* kc, const void* vc, const int* seqlens,
-                        void* o, float* lse, int B, int H, int Lmax, int d, float scale,
-                        float* partials, cudaStream_t stream);
+                        void* o, float* lse, int B, int H, int Hkv, int Lmax, int d,
+                        float scale, float* partials, cudaStream_t stream);
 
 inline fa_status cuda_status(cudaError_t e) { return e == cudaSuccess ? FA_OK : FA_ERR_CUDA; }
 

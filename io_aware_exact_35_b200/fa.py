@@ -29,10 +29,14 @@ STATUS_NAMES = {0: "FA_OK", 1: "FA_ERR_INVALID_ARG", 2: "FA_ERR_UNSUPPORTED",
 _P, _I, _F, _S = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
 SIGNATURES = {
     "fa_fwd": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _P]),
+    "fa_fwd_gqa": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _P]),
     "fa_bwd_workspace_size": (_S, [_I, _I, _I, _I]),
     "fa_bwd": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _S, _I, _I, _I, _I, _I, _F, _P]),
+    "fa_bwd_gqa": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _S, _I, _I, _I, _I, _I, _I, _F,
+                        _P]),
     "fa_decode_workspace_size": (_S, [_I, _I, _I, _I]),
     "fa_decode": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _F, _P, _S, _P]),
+    "fa_decode_gqa": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _P, _S, _P]),
     "fa_decode_static": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _F, _P]),
     "fa_get_device_error": (_I, [_P]),
     "fa_status_string": (ctypes.c_char_p, [_I]),
@@ -100,12 +104,14 @@ def _ptr(t: Optional[torch.Tensor]) -> Optional[int]:
 def fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, causal: bool = False,
         scale: Optional[float] = None, out: Optional[torch.Tensor] = None,
         lse: Optional[torch.Tensor] = None, want_lse: bool = True, stream=None):
-    """Exact attention forward.  q, k, v: bf16 [B, H, N, d].  Returns (o, lse)."""
+    """Exact attention forward.  q: bf16 [B, H, N, d]; k, v: bf16 [B, Hkv, N, d]
+    with Hkv dividing H (Hkv < H: grouped-query attention).  Returns (o, lse)."""
     for t, n in ((q, "q"), (k, "k"), (v, "v")):
         _req(t, n, torch.bfloat16, 4)
-    if k.shape != q.shape or v.shape != q.shape:
-        raise ValueError("q, k and v must have the same shape [B, H, N, d]")
     B, H, N, d = q.shape
+    Hkv = k.shape[1]
+    if (tuple(k.shape) != (B, Hkv, N, d) or v.shape != k.shape or Hkv < 1 or H % Hkv):
+        raise ValueError("k and v must be [B, Hkv, N, d] with Hkv dividing q's H")
     scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
     if out is None:
         out = torch.empty_like(q)
@@ -118,9 +124,9 @@ def fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, causal: bool = False,
         _req(lse, "lse", torch.float32, 3)
         if tuple(lse.shape) != (B, H, N):
             raise ValueError("lse must be [B, H, N]")
-    st = lib().fa_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), _ptr(lse),
-                      B, H, N, d, int(bool(causal)), scale, _stream_ptr(stream))
-    _check("fa_fwd", st)
+    st = lib().fa_fwd_gqa(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), _ptr(lse),
+                          B, H, Hkv, N, d, int(bool(causal)), scale, _stream_ptr(stream))
+    _check("fa_fwd_gqa", st)
     return out, lse
 
 
@@ -130,29 +136,35 @@ def bwd_workspace_size(B: int, H: int, N: int, d: int) -> int:
 
 def bwd(q, k, v, o, do, lse, causal: bool = False, scale: Optional[float] = None,
         dq=None, dk=None, dv=None, workspace: Optional[torch.Tensor] = None, stream=None):
-    """Backward with recomputation.  Returns (dq, dk, dv), bf16 [B, H, N, d]."""
+    """Backward with recomputation.  Returns (dq, dk, dv); dk and dv have k's
+    shape [B, Hkv, N, d] (grouped heads accumulate over their query heads)."""
     for t, n in ((q, "q"), (k, "k"), (v, "v"), (o, "o"), (do, "do")):
         _req(t, n, torch.bfloat16, 4)
-        if t.shape != q.shape:
-            raise ValueError(f"{n} must match q's shape")
     B, H, N, d = q.shape
+    Hkv = k.shape[1]
+    if o.shape != q.shape or do.shape != q.shape:
+        raise ValueError("o and do must match q's shape")
+    if tuple(k.shape) != (B, Hkv, N, d) or v.shape != k.shape or H % Hkv:
+        raise ValueError("k and v must be [B, Hkv, N, d] with Hkv dividing q's H")
     _req(lse, "lse", torch.float32, 3)
     if tuple(lse.shape) != (B, H, N):
         raise ValueError("lse must be [B, H, N]")
     scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
     dq = torch.empty_like(q) if dq is None else dq
-    dk = torch.empty_like(q) if dk is None else dk
-    dv = torch.empty_like(q) if dv is None else dv
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
     for t, n in ((dq, "dq"), (dk, "dk"), (dv, "dv")):
         _req(t, n, torch.bfloat16, 4)
     need = bwd_workspace_size(B, H, N, d)
     if workspace is None:
         workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=q.device)
-    st = lib().fa_bwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), do.data_ptr(),
-                      lse.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(),
-                      workspace.data_ptr(), workspace.numel() * workspace.element_size(),
-                      B, H, N, d, int(bool(causal)), scale, _stream_ptr(stream))
-    _check("fa_bwd", st)
+    if dq.shape != q.shape or dk.shape != k.shape or dv.shape != v.shape:
+        raise ValueError("gradient buffers must match q, k, v")
+    st = lib().fa_bwd_gqa(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), do.data_ptr(),
+                          lse.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(),
+                          workspace.data_ptr(), workspace.numel() * workspace.element_size(),
+                          B, H, Hkv, N, d, int(bool(causal)), scale, _stream_ptr(stream))
+    _check("fa_bwd_gqa", st)
     return dq, dk, dv
 
 
@@ -169,9 +181,9 @@ def decode(q, kcache, vcache, seqlens, scale: Optional[float] = None, out=None, 
     _req(vcache, "vcache", torch.bfloat16, 4)
     _req(seqlens, "seqlens", torch.int32, 1)
     B, H, d = q.shape
-    Lmax = kcache.shape[2]
-    if tuple(kcache.shape) != (B, H, Lmax, d) or vcache.shape != kcache.shape:
-        raise ValueError("caches must be [B, H, Lmax, d] matching q")
+    Hkv, Lmax = kcache.shape[1], kcache.shape[2]
+    if tuple(kcache.shape) != (B, Hkv, Lmax, d) or vcache.shape != kcache.shape or H % Hkv:
+        raise ValueError("caches must be [B, Hkv, Lmax, d] with Hkv dividing q's H")
     if seqlens.shape[0] != B:
         raise ValueError("seqlens must have B entries")
     scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
@@ -182,11 +194,11 @@ def decode(q, kcache, vcache, seqlens, scale: Optional[float] = None, out=None, 
     need = decode_workspace_size(B, H, Lmax, d)
     if workspace is None:
         workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=q.device)
-    st = lib().fa_decode(q.data_ptr(), kcache.data_ptr(), vcache.data_ptr(), seqlens.data_ptr(),
-                         out.data_ptr(), _ptr(lse), B, H, Lmax, d, scale,
-                         workspace.data_ptr(), workspace.numel() * workspace.element_size(),
-                         _stream_ptr(stream))
-    _check("fa_decode", st)
+    st = lib().fa_decode_gqa(q.data_ptr(), kcache.data_ptr(), vcache.data_ptr(),
+                             seqlens.data_ptr(), out.data_ptr(), _ptr(lse), B, H, Hkv, Lmax, d,
+                             scale, workspace.data_ptr(),
+                             workspace.numel() * workspace.element_size(), _stream_ptr(stream))
+    _check("fa_decode_gqa", st)
     return out, lse
 
 

@@ -38,6 +38,11 @@ class Workload:
     Lmin: int = 0        # decode: cache length range, inclusive
     Lmax: int = 0
     seed: int = BASE_SEED
+    Hkv: int = 0         # key/value heads (0: same as H; fewer: grouped-query attention)
+
+    @property
+    def kv_heads(self) -> int:
+        return self.Hkv or self.H
 
     @property
     def scale(self) -> float:
@@ -59,6 +64,13 @@ WORKLOADS = {
                  causal=True, seed=BASE_SEED + 3),
         Workload("decode_B16_H32_d128_L4096-16384", "decode", 16, 32, 128,
                  Lmin=4096, Lmax=16384, seed=BASE_SEED + 4),
+        # grouped-query variants (8 key/value heads shared by 32 query heads)
+        Workload("fwd_causal_gqa_B4_H32_Hkv8_N2048_d128", "fwd", 4, 32, 128, N=2048,
+                 causal=True, seed=BASE_SEED + 5, Hkv=8),
+        Workload("bwd_causal_gqa_B2_H32_Hkv8_N4096_d128", "bwd", 2, 32, 128, N=4096,
+                 causal=True, seed=BASE_SEED + 6, Hkv=8),
+        Workload("decode_gqa_B16_H32_Hkv8_d128_L4096-16384", "decode", 16, 32, 128,
+                 Lmin=4096, Lmax=16384, seed=BASE_SEED + 7, Hkv=8),
     )
 }
 
@@ -74,21 +86,30 @@ def _randn_bf16(g: torch.Generator, shape, std: float = 1.0) -> torch.Tensor:
     return x.to(torch.bfloat16)
 
 
-def fwd_inputs(B: int, H: int, N: int, d: int, seed: int, std: float = 1.0):
-    """q, k, v as contiguous bf16 CPU tensors [B, H, N, d]."""
+def fwd_inputs(B: int, H: int, N: int, d: int, seed: int, std: float = 1.0,
+               Hkv: int | None = None):
+    """q [B, H, N, d] and k, v [B, Hkv, N, d] (Hkv defaults to H) as contiguous
+    bf16 CPU tensors."""
     g = _gen(seed)
-    return tuple(_randn_bf16(g, (B, H, N, d), std) for _ in range(3))
+    hk = Hkv or H
+    return (_randn_bf16(g, (B, H, N, d), std), _randn_bf16(g, (B, hk, N, d), std),
+            _randn_bf16(g, (B, hk, N, d), std))
 
 
-def bwd_inputs(B: int, H: int, N: int, d: int, seed: int, std: float = 1.0):
-    """q, k, v, dO as contiguous bf16 CPU tensors [B, H, N, d]."""
+def bwd_inputs(B: int, H: int, N: int, d: int, seed: int, std: float = 1.0,
+               Hkv: int | None = None):
+    """q, k, v, dO as contiguous bf16 CPU tensors (k, v with Hkv heads)."""
     g = _gen(seed)
-    return tuple(_randn_bf16(g, (B, H, N, d), std) for _ in range(4))
+    hk = Hkv or H
+    return (_randn_bf16(g, (B, H, N, d), std), _randn_bf16(g, (B, hk, N, d), std),
+            _randn_bf16(g, (B, hk, N, d), std), _randn_bf16(g, (B, H, N, d), std))
 
 
 def decode_inputs(B: int, H: int, d: int, Lmin: int, Lmax: int, seed: int,
-                  Lcap: int | None = None, seqlens=None, poison: bool = True):
-    """q [B,H,d], kcache/vcache [B,H,Lcap,d] bf16, seqlens int32 [B].
+                  Lcap: int | None = None, seqlens=None, poison: bool = True,
+                  Hkv: int | None = None):
+    """q [B,H,d], kcache/vcache [B,Hkv,Lcap,d] bf16 (Hkv defaults to H),
+    seqlens int32 [B].
 
     ``seqlens`` may be given explicitly (edge-case tests); otherwise it is
     drawn first from the generator.  ``Lcap`` (the cache capacity) defaults
@@ -100,22 +121,23 @@ def decode_inputs(B: int, H: int, d: int, Lmin: int, Lmax: int, seed: int,
     seqlens = torch.as_tensor(seqlens, dtype=torch.int64)
     Lcap = int(Lcap if Lcap is not None else max(Lmax, int(seqlens.max().item()) if B else 0))
     q = _randn_bf16(g, (B, H, d))
+    hk = Hkv or H
     fill = float("nan") if poison else 0.0
-    kc = torch.full((B, H, Lcap, d), fill, dtype=torch.bfloat16)
-    vc = torch.full((B, H, Lcap, d), fill, dtype=torch.bfloat16)
+    kc = torch.full((B, hk, Lcap, d), fill, dtype=torch.bfloat16)
+    vc = torch.full((B, hk, Lcap, d), fill, dtype=torch.bfloat16)
     for b in range(B):
         L = int(seqlens[b])
-        kc[b, :, :L] = _randn_bf16(g, (H, L, d))
-        vc[b, :, :L] = _randn_bf16(g, (H, L, d))
+        kc[b, :, :L] = _randn_bf16(g, (hk, L, d))
+        vc[b, :, :L] = _randn_bf16(g, (hk, L, d))
     return q, kc, vc, seqlens.to(torch.int32)
 
 
 def workload_inputs(w: Workload):
     if w.kind == "fwd":
-        return fwd_inputs(w.B, w.H, w.N, w.d, w.seed, w.std)
+        return fwd_inputs(w.B, w.H, w.N, w.d, w.seed, w.std, Hkv=w.kv_heads)
     if w.kind == "bwd":
-        return bwd_inputs(w.B, w.H, w.N, w.d, w.seed, w.std)
-    return decode_inputs(w.B, w.H, w.d, w.Lmin, w.Lmax, w.seed)
+        return bwd_inputs(w.B, w.H, w.N, w.d, w.seed, w.std, Hkv=w.kv_heads)
+    return decode_inputs(w.B, w.H, w.d, w.Lmin, w.Lmax, w.seed, Hkv=w.kv_heads)
 
 
 def sample_rows(N: int, n_random: int, seed: int, edge: int = 128) -> np.ndarray:

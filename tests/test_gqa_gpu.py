@@ -1,0 +1,72 @@
+"""GPU parity of grouped-query attention (K/V heads shared by groups of query
+heads, "DL101 chapter 9" sections 3.1-3.2) in the forward, backward and
+decode kernels, against the fp64 oracle."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from io_aware_exact_35_b200 import inputs
+from tests._parity import check_grad, check_lse, check_o
+
+pytestmark = pytest.mark.gpu
+
+SHAPES = [(1, 4, 1, 300, 128), (2, 6, 2, 257, 64), (1, 8, 2, 1024, 128), (2, 4, 4, 129, 128)]
+
+
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("shape", SHAPES, ids=lambda s: "B%dH%dHkv%dN%dd%d" % s)
+def test_gqa_forward(fa_mod, cuda_device, shape, causal):
+    B, H, Hkv, N, d = shape
+    q, k, v = inputs.fwd_inputs(B, H, N, d, seed=300 + N + Hkv, Hkv=Hkv)
+    o, lse = fa_mod.fwd(q.cuda(), k.cuda(), v.cuda(), causal=causal)
+    torch.cuda.synchronize()
+    assert fa_mod.get_device_error() == 0
+    ref_o, ref_l = oracle.attention_forward(*(inputs.to_f64(t) for t in (q, k, v)), causal,
+                                            1 / np.sqrt(d))
+    check_o(o.cpu(), ref_o)
+    check_lse(lse.cpu(), ref_l)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("shape", SHAPES, ids=lambda s: "B%dH%dHkv%dN%dd%d" % s)
+def test_gqa_backward(fa_mod, cuda_device, shape, causal):
+    B, H, Hkv, N, d = shape
+    q, k, v, do = inputs.bwd_inputs(B, H, N, d, seed=400 + N + Hkv, Hkv=Hkv)
+    qd, kd, vd, dod = (t.cuda() for t in (q, k, v, do))
+    o, lse = fa_mod.fwd(qd, kd, vd, causal=causal)
+    dq, dk, dv = fa_mod.bwd(qd, kd, vd, o, dod, lse, causal=causal)
+    torch.cuda.synchronize()
+    assert fa_mod.get_device_error() == 0
+    assert dk.shape == k.shape and dv.shape == v.shape
+    rq, rk, rv, _ = oracle.attention_backward(*(inputs.to_f64(t) for t in (q, k, v, do)), causal,
+                                              1 / np.sqrt(d))
+    check_grad(dq.cpu(), rq, "dQ")
+    check_grad(dk.cpu(), rk, "dK")
+    check_grad(dv.cpu(), rv, "dV")
+
+
+@pytest.mark.parametrize("Hkv", [1, 4, 8])
+def test_gqa_decode(fa_mod, cuda_device, Hkv):
+    q, kc, vc, sl = inputs.decode_inputs(3, 8, 128, 1, 2100, seed=500 + Hkv, Hkv=Hkv,
+                                         seqlens=[0, 700, 2100], Lcap=2100)
+    o, lse = fa_mod.decode(q.cuda(), kc.cuda(), vc.cuda(), sl.cuda())
+    torch.cuda.synchronize()
+    assert fa_mod.get_device_error() == 0
+    ref_o, ref_l = oracle.decode_forward(inputs.to_f64(q), inputs.to_f64(kc), inputs.to_f64(vc),
+                                         sl.tolist(), 1 / np.sqrt(128))
+    check_o(o.cpu(), ref_o)
+    check_lse(lse.cpu(), ref_l)
+
+
+def test_gqa_workload_forward_B4_H32_Hkv8_N2048_sampled(fa_mod, cuda_device):
+    w = inputs.WORKLOADS["fwd_causal_gqa_B4_H32_Hkv8_N2048_d128"]
+    q, k, v = inputs.workload_inputs(w)
+    o, lse = fa_mod.fwd(q.cuda(), k.cuda(), v.cuda(), causal=True)
+    torch.cuda.synchronize()
+    rows = inputs.sample_rows(w.N, 64, seed=w.seed)
+    for b, h in ((0, 0), (3, 31), (1, 9)):
+        ro, rl = oracle.attention_forward_rows(inputs.to_f64(q[b, h]), inputs.to_f64(k[b, h // 4]),
+                                               inputs.to_f64(v[b, h // 4]), True, w.scale, rows)
+        check_o(o[b, h, rows].cpu(), ro)
+        check_lse(lse[b, h, rows].cpu(), rl)
