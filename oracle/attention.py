@@ -31,7 +31,10 @@ Readings taken where the pages are silent or inconsistent:
   logarithm of the row's softmax denominator over the *scaled* scores:
   LSE_i = m_i + ln(sum_j exp(s_ij - m_i)).
 * Causal masking keeps keys j <= i (token t attends K_{<=t}); the diagonal is
-  included, top-left aligned, and requires Nq == Nk.
+  included.  With Nq != Nk the queries are read as the last Nq positions of
+  the Nk-token sequence (a chunk of new tokens over a cache): query i attends
+  keys j <= i + Nk - Nq (bottom-right alignment); queries that see no key
+  get O = 0 and LSE = -inf.
 * A row with no admissible key (decode with seqlen 0) has O = 0, LSE = -inf.
 * The tiled page-1 code divides O by l inside the loop and resets l to the
   block sum; that is only right for one key block.  The tiled routine here
@@ -87,12 +90,13 @@ def softmax_rows(s: np.ndarray) -> np.ndarray:
 
 
 def _scores(q_rows: np.ndarray, k: np.ndarray, scale: float,
-            row_index: np.ndarray | None, causal: bool) -> np.ndarray:
-    """Scaled scores s_ij = scale * q_i . k_j, masked to -inf where j > i."""
+            row_index: np.ndarray | None, causal: bool, offset: int = 0) -> np.ndarray:
+    """Scaled scores s_ij = scale * q_i . k_j, masked to -inf where j > i + offset
+    (offset = Nk - Nq: query i sits at position i + offset of the key sequence)."""
     s = scale * (q_rows @ k.T)
     if causal:
         cols = np.arange(k.shape[0])[None, :]
-        s = np.where(cols > row_index[:, None], -np.inf, s)
+        s = np.where(cols > row_index[:, None] + offset, -np.inf, s)
     return s
 
 
@@ -135,8 +139,7 @@ def attention_forward(q: np.ndarray, k: np.ndarray, v: np.ndarray,
     _check_f64(q, k, v)
     if q.ndim == 4 and k.ndim == 4 and k.shape[1] != q.shape[1]:
         k, v = expand_kv_heads(k, q.shape[1]), expand_kv_heads(v, q.shape[1])
-    if causal and q.shape[-2] != k.shape[-2]:
-        raise ValueError("causal attention is defined here for Nq == Nk only")
+    offset = k.shape[-2] - q.shape[-2]
     lead = q.shape[:-2]
     nq, d = q.shape[-2:]
     qf = q.reshape((-1, nq, d))
@@ -147,7 +150,7 @@ def attention_forward(q: np.ndarray, k: np.ndarray, v: np.ndarray,
     for bh in range(qf.shape[0]):
         for r0 in range(0, nq, _ROW_BLOCK):
             rows = np.arange(r0, min(nq, r0 + _ROW_BLOCK))
-            s = _scores(qf[bh, rows], kf[bh], scale, rows, causal)
+            s = _scores(qf[bh, rows], kf[bh], scale, rows, causal, offset)
             p, lse_blk = _row_stats(s)
             o[bh, rows] = p @ vf[bh]
             lse[bh, rows] = lse_blk
@@ -163,7 +166,7 @@ def attention_forward_rows(q: np.ndarray, k: np.ndarray, v: np.ndarray,
     """
     _check_f64(q, k, v)
     rows = np.asarray(rows, dtype=np.int64)
-    s = _scores(q[rows], k, scale, rows, causal)
+    s = _scores(q[rows], k, scale, rows, causal, k.shape[0] - q.shape[0])
     p, lse = _row_stats(s)
     return p @ v, lse
 
@@ -194,8 +197,6 @@ def attention_backward(q: np.ndarray, k: np.ndarray, v: np.ndarray,
         dk = dk.reshape(dk.shape[0], hkv, g, *dk.shape[2:]).sum(axis=2)
         dv = dv.reshape(dv.shape[0], hkv, g, *dv.shape[2:]).sum(axis=2)
         return dq, dk, dv, D
-    if causal and q.shape[-2] != k.shape[-2]:
-        raise ValueError("causal attention is defined here for Nq == Nk only")
     lead = q.shape[:-2]
     nq, d = q.shape[-2:]
     nk = k.shape[-2]
@@ -207,7 +208,7 @@ def attention_backward(q: np.ndarray, k: np.ndarray, v: np.ndarray,
     dD = np.zeros((qf.shape[0], nq))
     rows = np.arange(nq)
     for bh in range(qf.shape[0]):
-        s = _scores(qf[bh], kf[bh], scale, rows, causal)
+        s = _scores(qf[bh], kf[bh], scale, rows, causal, nk - nq)
         p, _ = _row_stats(s)
         dv[bh] = p.T @ dof[bh]
         dp = dof[bh] @ vf[bh].T

@@ -412,3 +412,41 @@ def test_grouped_decode_matches_expanded_cache():
                 torch.from_numpy(q[b, h][None, None]), torch.from_numpy(kc[b, h // 2, :L][None]),
                 torch.from_numpy(vc[b, h // 2, :L][None]), scale=0.5)
             assert np.allclose(o[b, h], ref[0, 0].numpy(), atol=1e-13)
+
+
+def test_unequal_lengths_match_sdpa_with_bottom_right_mask():
+    """Nq != Nk: non-causal against plain SDPA (the DL101 chapter 9 section 3.3
+    example uses Lq = 1280, Lk = 1152); causal against SDPA with an explicit
+    bottom-right mask tril(Nk - Nq)."""
+    for (nq, nk) in ((40, 29), (17, 50), (1, 33)):
+        q = bf16_grid((1, 2, nq, 16))
+        k, v = bf16_grid((1, 2, nk, 16)), bf16_grid((1, 2, nk, 16))
+        for causal in (False, True):
+            o, lse = A.attention_forward(q, k, v, causal, 0.25)
+            mask = torch.ones(nq, nk, dtype=torch.bool)
+            if causal:
+                mask = mask.tril(nk - nq)
+            tq, tk, tv = (torch.from_numpy(x) for x in (q, k, v))
+            ref = torch.nn.functional.scaled_dot_product_attention(tq, tk, tv, attn_mask=mask,
+                                                                   scale=0.25).numpy()
+            empty = ~mask.any(dim=1).numpy()  # rows with no admissible key
+            assert np.allclose(o[..., ~empty, :], ref[..., ~empty, :], atol=1e-12)
+            assert np.all(o[..., empty, :] == 0) and np.all(np.isneginf(lse[..., empty]))
+            s = 0.25 * (tq @ tk.transpose(-1, -2))
+            ref_lse = torch.logsumexp(s.masked_fill(~mask, -math.inf), -1).numpy()
+            assert np.allclose(lse[..., ~empty], ref_lse[..., ~empty], atol=1e-12)
+
+
+def test_unequal_lengths_backward_matches_autograd():
+    for (nq, nk) in ((24, 40), (40, 24)):
+        q, do = bf16_grid((1, 2, nq, 8)), bf16_grid((1, 2, nq, 8))
+        k, v = bf16_grid((1, 2, nk, 8)), bf16_grid((1, 2, nk, 8))
+        mask = torch.ones(nq, nk, dtype=torch.bool).tril(nk - nq)
+        keep = mask.any(dim=1)
+        tq, tk, tv = (torch.from_numpy(x).requires_grad_() for x in (q, k, v))
+        o = torch.nn.functional.scaled_dot_product_attention(tq, tk, tv, attn_mask=mask, scale=0.4)
+        # rows without keys are NaN in SDPA; the definition gives them O = 0
+        (o[..., keep, :] * torch.from_numpy(do)[..., keep, :]).sum().backward()
+        dq, dk, dv, _ = A.attention_backward(q, k, v, do, True, 0.4)
+        assert np.allclose(dq[..., keep.numpy(), :], tq.grad.numpy()[..., keep.numpy(), :], atol=1e-11)
+        assert np.allclose(dk, tk.grad.numpy(), atol=1e-11) and np.allclose(dv, tv.grad.numpy(), atol=1e-11)
