@@ -146,8 +146,11 @@ class ClockSampler:
 
 # ----------------------------------------------------------------------------- workloads
 def workload_config(w, parallelism):
-    return {"workload": w.name, "B": w.B, "H": w.H, "Hkv": w.kv_heads, "N": w.N or None,
-            "d": w.d, "causal": w.causal, "parallelism": parallelism}
+    cfg = {"workload": w.name, "B": w.B, "H": w.H, "Hkv": w.kv_heads, "N": w.N or None,
+           "d": w.d, "causal": w.causal, "parallelism": parallelism}
+    if w.page:
+        cfg["page_size"] = w.page
+    return cfg
 
 
 def fwd_flops(w):
@@ -190,14 +193,26 @@ class Runner:
             self.out_host = torch.empty(self.dq.shape, dtype=torch.bfloat16).pin_memory()
         else:
             q, kc, vc, sl = self.dbuf
+            lcap = kc.shape[2]
+            if w.page:
+                # paged cache: pools and page table replace the contiguous caches
+                kp, vp, table = inputs.page_cache(*self.host[1:3], self.host[3], w.page,
+                                                  w.seed + 1)
+                self.host = [self.host[0], kp, vp, table, self.host[3]]
+                self.dbuf = [t.to(dev) for t in self.host]
+                q = self.dbuf[0]
+                lcap = table.shape[1] * w.page
             self.o = torch.empty_like(q)
             self.lse = torch.empty(q.shape[:2], dtype=torch.float32, device=dev)
-            self.ws = torch.empty(fa.decode_workspace_size(w.B, w.H, kc.shape[2], w.d),
+            self.ws = torch.empty(fa.decode_workspace_size(w.B, w.H, lcap, w.d),
                                   dtype=torch.uint8, device=dev)
-            self.work = decode_bytes(w, self.host[3].tolist())
+            self.work = decode_bytes(w, self.host[-1].tolist())
             self.unit, self.kind_bound = "GB/s", "hbm"
             self.launches_per_step = 2
-            self.kernel_key = f"fa_decode_split_kernel<{w.d}>"
+            group = w.H // w.kv_heads
+            paged = ",paged" if w.page else ""
+            self.kernel_key = (f"fa_decode_group_split_kernel<{w.d},{group}{paged}>"
+                               if group in (2, 4, 8) else f"fa_decode_split_kernel<{w.d}{paged}>")
             self.out_host = torch.empty(self.o.shape, dtype=torch.bfloat16).pin_memory()
         self.working_set = sum(t.numel() * t.element_size() for t in self.dbuf)
         self.flush = None
@@ -214,6 +229,10 @@ class Runner:
             fa.bwd(b[0], b[1], b[2], self.o, b[3], self.lse, causal=w.causal, scale=w.scale,
                    dq=self.dq, dk=self.dk, dv=self.dv, workspace=self.ws)
             return self.dq
+        if w.page:
+            fa.decode_paged(b[0], b[1], b[2], b[3], b[4], scale=w.scale, out=self.o,
+                            lse=self.lse, workspace=self.ws)
+            return self.o
         fa.decode(b[0], b[1], b[2], b[3], scale=w.scale, out=self.o, lse=self.lse,
                   workspace=self.ws)
         return self.o

@@ -18,8 +18,12 @@
  *    are masked inside the kernels).
  *  - scale multiplies Q K^T before the softmax; callers normally pass
  *    1/sqrt(d) ("DL101 chapter 9", section 1.1).
- *  - Causal masking keeps key j for query i iff j <= i (square, top-left
- *    aligned, diagonal included).
+ *  - Causal masking keeps key j for query i iff j <= i + Nk - Nq (diagonal
+ *    included; with Nq = Nk = N simply j <= i).  With Nq != Nk (the _ext
+ *    entry points) the Nq queries are the last Nq positions of the Nk-token
+ *    sequence, i.e. a chunk of new tokens over a cache ("DL101 chapter 9",
+ *    section 1.1: token t attends K_{<=t}).  A query that sees no key
+ *    (only when Nq > Nk) gets O = 0 and LSE = -inf.
  *  - LSE is the natural-log log-sum-exp of the row's scaled, masked scores:
  *    LSE_i = ln sum_j exp(scale * q_i . k_j).
  *  - The caller allocates and owns every buffer, workspaces included.  The
@@ -79,6 +83,22 @@ fa_status fa_fwd_gqa(const void* q, const void* k, const void* v, void* o, float
                      fa_stream_t stream);
 
 /*
+ * Forward with separate query and key lengths, grouped heads allowed (the
+ * non-square Lq x Lk problem of "DL101 chapter 9", section 3.3):
+ *   q       : bf16 [B, H, Nq, d], read only.
+ *   k, v    : bf16 [B, Hkv, Nk, d], read only.
+ *   o       : bf16 [B, H, Nq, d], written.
+ *   lse     : float32 [B, H, Nq], written; may be NULL.
+ * Nq, Nk >= 0 with Nq + Nk < 2^31.  Causal masking is bottom-right aligned
+ * (see the conventions above).  Nk = 0 writes O = 0 and LSE = -inf.
+ * Pointers to arrays of zero size may be NULL.
+ * fa_fwd_gqa(..., N, ...) is fa_fwd_ext(..., N, N, ...).  Returns as fa_fwd.
+ */
+fa_status fa_fwd_ext(const void* q, const void* k, const void* v, void* o, float* lse,
+                     int B, int H, int Hkv, int Nq, int Nk, int d, int causal, float scale,
+                     fa_stream_t stream);
+
+/*
  * Bytes of device workspace fa_bwd needs: D = rowsum(dO * O) and
  * log2(e) * LSE as float32 [B, H, Np] with Np = N rounded up to a multiple
  * of 128, followed by the float32 dQ accumulator [B, H, N, d], each region
@@ -116,6 +136,24 @@ fa_status fa_bwd_gqa(const void* q, const void* k, const void* v, const void* o,
                      const void* dout, const float* lse, void* dq, void* dk, void* dv,
                      void* workspace, size_t ws_bytes,
                      int B, int H, int Hkv, int N, int d, int causal, float scale,
+                     fa_stream_t stream);
+
+/*
+ * Backward with separate query and key lengths (the inverse of fa_fwd_ext):
+ *   q, o, dout : bf16 [B, H, Nq, d], read only;  lse : float32 [B, H, Nq].
+ *   k, v       : bf16 [B, Hkv, Nk, d], read only.
+ *   dq         : bf16 [B, H, Nq, d], written.
+ *   dk, dv     : bf16 [B, Hkv, Nk, d], written.
+ *   workspace  : fa_bwd_workspace_size(B, H, Nq, d) bytes (not needed when
+ *                Nq or Nk is 0).
+ * Queries with LSE = -inf (they saw no key) contribute nothing.  Nq = 0
+ * writes dK = dV = 0; Nk = 0 writes dQ = 0.  Pointers to arrays of zero size
+ * may be NULL.  Returns as fa_bwd.
+ */
+fa_status fa_bwd_ext(const void* q, const void* k, const void* v, const void* o,
+                     const void* dout, const float* lse, void* dq, void* dk, void* dv,
+                     void* workspace, size_t ws_bytes,
+                     int B, int H, int Hkv, int Nq, int Nk, int d, int causal, float scale,
                      fa_stream_t stream);
 
 /*
@@ -159,6 +197,36 @@ fa_status fa_decode_gqa(const void* q, const void* kcache, const void* vcache,
                         const int* seqlens, void* o, float* lse,
                         int B, int H, int Hkv, int Lmax, int d, float scale,
                         void* workspace, size_t ws_bytes, fa_stream_t stream);
+
+/*
+ * Decode over a paged KV cache.  The pages name PagedAttention without
+ * describing it; this is the addressing it implies: the cache of every
+ * sequence is a list of fixed-size pages drawn from one pool, so sequences
+ * grow without reserving Lmax rows each.  The arithmetic is fa_decode's
+ * ("DL101 chapter 9", section 1.1; split-KV merge of "Flash Attention:
+ * principle & practice", section 2.1).
+ *   kpages,
+ *   vpages      : bf16 [num_pages, Hkv, page_size, d], read only; row r of
+ *                 head h of pool page p holds the key / value of one position.
+ *   block_table : int32 [B, pages_per_seq] in DEVICE memory: position j of
+ *                 sequence b lives in row j % page_size of pool page
+ *                 block_table[b][j / page_size].  Entries past a sequence's
+ *                 last page are never read.  An entry outside
+ *                 [0, num_pages) is never dereferenced: its positions count
+ *                 as masked and FA_ERR_INVALID_ARG is recorded in the device
+ *                 error word (read it with fa_get_device_error).
+ *   seqlens     : int32 [B], device; clamped to [0, pages_per_seq * page_size].
+ *   page_size   : a power of two from 1 to 65536.
+ *   workspace   : fa_decode_workspace_size(B, H, pages_per_seq * page_size, d).
+ * q, o, lse, scale and the grouping Hkv as fa_decode_gqa.  Returns
+ * FA_OK, FA_ERR_INVALID_ARG, FA_ERR_UNSUPPORTED, FA_ERR_WORKSPACE or
+ * FA_ERR_CUDA.
+ */
+fa_status fa_decode_paged(const void* q, const void* kpages, const void* vpages,
+                          const int* block_table, const int* seqlens, void* o, float* lse,
+                          int B, int H, int Hkv, int page_size, int pages_per_seq,
+                          int num_pages, int d, float scale,
+                          void* workspace, size_t ws_bytes, fa_stream_t stream);
 
 /*
  * Size in bytes of the device array that fa_decode_static uses as scratch

@@ -4,4 +4,4 @@ split-KV decode, behind the C-ABI library ``libfa_b200.so``.
 Importing the package loads nothing; ``io_aware_exact_35_b200.fa`` loads the
 compiled library on first use and raises if it is missing.
 """
-__all__ = ["fa", "inputs"]
+__all__ = ["fa", "inputs", "autograd"]

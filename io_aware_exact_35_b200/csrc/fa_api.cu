@@ -132,17 +132,26 @@ fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* ls
 
 fa_status fa_fwd_gqa(const void* q, const void* k, const void* v, void* o, float* lse, int B,
                      int H, int Hkv, int N, int d, int causal, float scale, fa_stream_t stream) {
-  fa_status st = check_shape(B, H, N, d);
+  return fa_fwd_ext(q, k, v, o, lse, B, H, Hkv, N, N, d, causal, scale, stream);
+}
+
+fa_status fa_fwd_ext(const void* q, const void* k, const void* v, void* o, float* lse, int B,
+                     int H, int Hkv, int Nq, int Nk, int d, int causal, float scale,
+                     fa_stream_t stream) {
+  fa_status st = check_shape(B, H, Nq, d);
   if (st != FA_OK) return st;
+  if ((st = check_shape(B, Hkv, Nk, d)) != FA_OK) return st;
+  if (static_cast<long long>(Nq) + Nk > INT_MAX) return FA_ERR_INVALID_ARG;
   if (Hkv < 1 || H % Hkv != 0) return FA_ERR_INVALID_ARG;
-  if (!q || !k || !v || !o) return FA_ERR_INVALID_ARG;
+  // arrays of zero size may be null
+  if (Nq > 0 && (!q || !o || (Nk > 0 && (!k || !v)))) return FA_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o)) return FA_ERR_INVALID_ARG;
   if (lse != nullptr && (reinterpret_cast<uintptr_t>(lse) & 3u)) return FA_ERR_INVALID_ARG;
   if (causal != 0 && causal != 1) return FA_ERR_INVALID_ARG;
   if (!(scale == scale)) return FA_ERR_INVALID_ARG;  // NaN
   if ((st = check_device()) != FA_OK) return st;
-  if (N == 0) return FA_OK;
-  return launch_fwd(q, k, v, o, lse, B, H, Hkv, N, d, causal, scale,
+  if (Nq == 0) return FA_OK;
+  return launch_fwd(q, k, v, o, lse, B, H, Hkv, Nq, Nk, d, causal, scale,
                     reinterpret_cast<cudaStream_t>(stream));
 }
 
@@ -167,23 +176,35 @@ fa_status fa_bwd_gqa(const void* q, const void* k, const void* v, const void* o,
                      const void* dout, const float* lse, void* dq, void* dk, void* dv,
                      void* workspace, size_t ws_bytes, int B, int H, int Hkv, int N, int d,
                      int causal, float scale, fa_stream_t stream) {
-  fa_status st = check_shape(B, H, N, d);
+  return fa_bwd_ext(q, k, v, o, dout, lse, dq, dk, dv, workspace, ws_bytes, B, H, Hkv, N, N, d,
+                    causal, scale, stream);
+}
+
+fa_status fa_bwd_ext(const void* q, const void* k, const void* v, const void* o,
+                     const void* dout, const float* lse, void* dq, void* dk, void* dv,
+                     void* workspace, size_t ws_bytes, int B, int H, int Hkv, int Nq, int Nk,
+                     int d, int causal, float scale, fa_stream_t stream) {
+  fa_status st = check_shape(B, H, Nq, d);
   if (st != FA_OK) return st;
+  if ((st = check_shape(B, Hkv, Nk, d)) != FA_OK) return st;
+  if (static_cast<long long>(Nq) + Nk > INT_MAX) return FA_ERR_INVALID_ARG;
   if (Hkv < 1 || H % Hkv != 0) return FA_ERR_INVALID_ARG;
-  if (!q || !k || !v || !o || !dout || !lse || !dq || !dk || !dv) return FA_ERR_INVALID_ARG;
+  // arrays of zero size may be null
+  if (Nq > 0 && (!q || !o || !dout || !lse || !dq)) return FA_ERR_INVALID_ARG;
+  if (Nk > 0 && (!dk || !dv || (Nq > 0 && (!k || !v)))) return FA_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(dout) ||
       !aligned16(dq) || !aligned16(dk) || !aligned16(dv) ||
       (reinterpret_cast<uintptr_t>(lse) & 3u))
     return FA_ERR_INVALID_ARG;
   if (causal != 0 && causal != 1) return FA_ERR_INVALID_ARG;
   if (!(scale == scale)) return FA_ERR_INVALID_ARG;
-  const size_t need = fa_bwd_workspace_size(B, H, N, d);
-  if (N > 0 && (workspace == nullptr || ws_bytes < need || !aligned256(workspace)))
+  const size_t need = fa_bwd_workspace_size(B, H, Nq, d);
+  if (Nq > 0 && Nk > 0 && (workspace == nullptr || ws_bytes < need || !aligned256(workspace)))
     return FA_ERR_WORKSPACE;
   if ((st = check_device()) != FA_OK) return st;
-  if (N == 0) return FA_OK;
-  return launch_bwd(q, k, v, o, dout, lse, dq, dk, dv, workspace, B, H, Hkv, N, d, causal, scale,
-                    reinterpret_cast<cudaStream_t>(stream));
+  if (Nq == 0 && Nk == 0) return FA_OK;
+  return launch_bwd(q, k, v, o, dout, lse, dq, dk, dv, workspace, B, H, Hkv, Nq, Nk, d, causal,
+                    scale, reinterpret_cast<cudaStream_t>(stream));
 }
 
 size_t fa_decode_workspace_size(int B, int H, int Lmax, int d) {
@@ -220,6 +241,49 @@ fa_status fa_decode_gqa(const void* q, const void* kcache, const void* vcache, c
   if (st != FA_OK) return st;
   return launch_decode(q, kcache, vcache, seqlens, o, lse, B, H, Hkv, Lmax, d, scale,
                        static_cast<float*>(workspace), reinterpret_cast<cudaStream_t>(stream));
+}
+
+fa_status fa_decode_paged(const void* q, const void* kpages, const void* vpages,
+                          const int* block_table, const int* seqlens, void* o, float* lse, int B,
+                          int H, int Hkv, int page_size, int pages_per_seq, int num_pages, int d,
+                          float scale, void* workspace, size_t ws_bytes, fa_stream_t stream) {
+  if (B < 1 || H < 1 || pages_per_seq < 0 || num_pages < 0) return FA_ERR_INVALID_ARG;
+  if (Hkv < 1 || H % Hkv != 0) return FA_ERR_INVALID_ARG;
+  if (static_cast<long long>(B) * H > INT_MAX) return FA_ERR_INVALID_ARG;
+  // rows per page: a power of two from 1 to 65536
+  if (page_size < 1 || page_size > 65536 || (page_size & (page_size - 1)) != 0)
+    return FA_ERR_INVALID_ARG;
+  const long long lmax = static_cast<long long>(page_size) * pages_per_seq;
+  if (lmax > INT_MAX) return FA_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
+  if (!q || !seqlens || !o || (pages_per_seq > 0 && !block_table) ||
+      (num_pages > 0 && (!kpages || !vpages)))
+    return FA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(kpages) || !aligned16(vpages) || !aligned16(o) ||
+      (reinterpret_cast<uintptr_t>(seqlens) & 3u) ||
+      (reinterpret_cast<uintptr_t>(block_table) & 3u) ||
+      (lse != nullptr && (reinterpret_cast<uintptr_t>(lse) & 3u)))
+    return FA_ERR_INVALID_ARG;
+  if (!(scale == scale)) return FA_ERR_INVALID_ARG;
+  const int Lmax = static_cast<int>(lmax);
+  const size_t need = fa_decode_workspace_size(B, H, Lmax, d);
+  if (need > 0 && (workspace == nullptr || ws_bytes < need || !aligned256(workspace)))
+    return FA_ERR_WORKSPACE;
+  fa_status st = check_device();
+  if (st != FA_OK) return st;
+  int log2_page = 0;
+  while ((1 << log2_page) < page_size) ++log2_page;
+  // a table of no pages (or a pool of none) leaves every sequence empty
+  const int* table = (pages_per_seq > 0 && num_pages > 0) ? block_table : nullptr;
+  if (table == nullptr) {
+    // O = 0, LSE = -inf for every (b, h): the combine kernel alone with
+    // zero splits does exactly that (no partial is read)
+    return launch_decode(q, kpages, vpages, seqlens, o, lse, B, H, Hkv, 0, d, scale,
+                         static_cast<float*>(workspace), reinterpret_cast<cudaStream_t>(stream));
+  }
+  return launch_decode(q, kpages, vpages, seqlens, o, lse, B, H, Hkv, Lmax, d, scale,
+                       static_cast<float*>(workspace), reinterpret_cast<cudaStream_t>(stream),
+                       table, pages_per_seq, log2_page, num_pages);
 }
 
 fa_status fa_get_device_error(fa_stream_t stream) {

@@ -11,7 +11,8 @@
 //   fa_bwd_preprocess  D = rowsum(dO * O) (fp32) and a zeroed fp32 dQ accumulator.
 //   fa_bwd_kernel      one CTA per 128-key tile j of one (batch, head); it keeps
 //                      dK_j and dV_j in tensor memory and loops over the query
-//                      tiles i that can see key tile j (i >= j when causal):
+//                      tiles i that can see key tile j (causal: those holding a
+//                      query at or after key j's position):
 //                        S^T = K_j Q_i^T, dP^T = V_j dO_i^T        (tcgen05, TMEM)
 //                        P^T, dS^T on the CUDA cores (one key row per thread)
 //                        dV += P^T dO_i, dK += dS^T Q_i            (A from TMEM)
@@ -21,16 +22,26 @@
 //
 // Warp roles of fa_bwd_kernel (448 threads):
 //   warps 0-7  two P^T / dS^T warpgroups: thread t of warpgroup g owns key row t
-//              (TMEM lane t) for queries 64g .. 64g+63 of the tile; in the
-//              epilogue warpgroup 0 writes dV and warpgroup 1 writes dK.
+//              (TMEM lane t) for queries 64g .. 64g+63 of the tile, in two
+//              phases: P^T as soon as S^T is ready (dV can start), then dS^T
+//              once dP^T is ready.  In the epilogue warpgroup 0 writes dV and
+//              warpgroup 1 writes dK.
 //   warps 8-11 dQ warpgroup: thread t owns query row t of the dQ tile.
 //   warp 12    TMA producer: K_j, V_j once; Q_i, dO_i, LSE_i, D_i through a
 //              two-stage ring.
-//   warp 13    tensor-memory allocator and MMA issuer.
+//   warp 13    tensor-memory allocator and MMA issuer, in the order
+//                S^T(i) dP^T(i) | dV(i) | dK(i) dQ(i) | S^T(i+1) ...
+//              where "|" waits for the P^T phase, the dS^T phase, and (before
+//              the next dP^T) for dQ(i) to have left tensor memory.
 // Tensor memory (512 columns): S^T [0,128), dP^T [128,256), dV [256, 256+d),
 // dK [256+d, 256+2d).  Warpgroup g overwrites columns [64g, 64g+32) of S^T
 // with P^T (bf16 pairs) and the same columns of dP^T with dS^T, i.e. only
 // scores it has already read; dQ_i lands in [128, 128+d) afterwards.
+// dQ_i leaves tensor memory into the Q_i / dO_i stage it was computed from
+// (free once dQ_i is complete), so the dS buffer is never shared with it.
+#include <cstdlib>
+#include <cstring>
+
 #include "fa_internal.h"
 #include "sm100.cuh"
 
@@ -57,8 +68,8 @@ struct Smem {
   static constexpr int LSE_OFF = DS_OFF + DS_BYTES;    // 2 stages x 128 fp32
   static constexpr int DD_OFF = LSE_OFF + 2 * 512;     // 2 stages x 128 fp32
   static constexpr int BAR_OFF = DD_OFF + 2 * 512;
-  // kv_full, qd_full[2], qd_empty[2], st_full, dpt_full, pds_full, dq_full,
-  // dq_free, dkv_final, mma_final, stg_full, stg_free
+  // kv_full, qd_full[2], qd_empty[2], st_full, dpt_full, ds_full, dq_full,
+  // dq_free, dkv_final, mma_final, stg_full, p_full
   static constexpr int NBAR = 14;
   static constexpr int MISC_OFF = BAR_OFF + NBAR * 8;
   static constexpr int BYTES = MISC_OFF + 16;
@@ -69,9 +80,14 @@ struct Params {
   __nv_bfloat16* dk;
   __nv_bfloat16* dv;
   float* dqacc;
-  int N;
-  int n_tiles;
+  int Nq;            // query rows per head
+  int Nk;            // key / value rows per head
+  int causal_off;    // Nk - Nq: query i sits at key position i + causal_off
+  int n_qt;          // query tiles per head, ceil(Nq / 128)
+  int n_kt;          // key tiles per head, ceil(Nk / 128)
   int group;         // query heads per key/value head (1 without grouping)
+  int BHkv;          // batch x key/value heads
+  int lpt_order;     // 1: key tile 0 of every head first; 0: head-major
   float scale_log2;  // scale * log2(e)
   float scale;
 };
@@ -106,13 +122,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   uint64_t* qd_empty = bars + 3;  // [2]
   uint64_t* st_full = bars + 5;
   uint64_t* dpt_full = bars + 6;
-  uint64_t* pds_full = bars + 7;
+  uint64_t* ds_full = bars + 7;    // dS^T (TMEM) and dS (shared) written
   uint64_t* dq_full = bars + 8;
-  uint64_t* dq_free = bars + 9;
+  uint64_t* dq_free = bars + 9;    // dQ read out of tensor memory
   uint64_t* dkv_final = bars + 10;
   uint64_t* mma_final = bars + 11;
   uint64_t* stg_full = bars + 12;  // dQ staging written (128 arrivals)
-  uint64_t* stg_free = bars + 13;  // dQ staging read by the bulk reduction
+  uint64_t* p_full = bars + 13;    // P^T written (both warpgroups)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::MISC_OFF);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::MISC_OFF + 4);
 
@@ -123,19 +139,25 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   // tiles in L2); tile 0, which sees the most query tiles, comes first.
   // bkv indexes key/value heads; the CTA accumulates dK, dV of key tile
   // kv_tile over the query tiles of all `group` query heads sharing it.
-  const int bkv = static_cast<int>(blockIdx.x) / p.n_tiles;
-  const int kv_tile = static_cast<int>(blockIdx.x) - bkv * p.n_tiles;
+  // Head-major order keeps one head's Q / dO tiles shared in L2 by its
+  // resident CTAs; longest-first order (key tile 0, which sees every query
+  // tile, of all heads first) balances few long CTAs.
+  const int bx = static_cast<int>(blockIdx.x);
+  const int kv_tile = p.lpt_order ? bx / p.BHkv : bx % p.n_kt;
+  const int bkv = p.lpt_order ? bx - kv_tile * p.BHkv : bx / p.n_kt;
   const int key0 = kv_tile * BLOCK;
-  const int i_begin = CAUSAL ? kv_tile : 0;
-  const int n_per = p.n_tiles - i_begin;  // query tiles per query head
-  const int n_it = n_per * p.group;
+  // causal: the first query that sees key key0 is row key0 - causal_off
+  const int i_begin = CAUSAL ? max(0, key0 - p.causal_off) / BLOCK : 0;
+  const int n_per = max(0, p.n_qt - i_begin);  // query tiles per query head
+  const int n_it = n_per * p.group;            // 0: dK = dV = 0
   // iteration it -> (query head, first row of its query tile)
   auto it_head = [&](int it) { return bkv * p.group + it / n_per; };
   auto it_q0 = [&](int it) { return (i_begin + it % n_per) * BLOCK; };
 
   if (threadIdx.x == 0) {
     for (int b = 0; b < L::NBAR; ++b) mbar_init(&bars[b], 1);
-    mbar_init(pds_full, 2 * BLOCK);  // both P^T / dS^T warpgroups
+    mbar_init(p_full, 2 * BLOCK);   // both P^T / dS^T warpgroups
+    mbar_init(ds_full, 2 * BLOCK);
     mbar_init(dq_free, BLOCK);
     mbar_init(stg_full, BLOCK);
     *abort_flag = 0;
@@ -227,16 +249,18 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         for (int kk = 0; kk < D / 16; ++kk)
           mma_bf16_ss(tdPt, vdK + koff(kk), dodK0 + soff + koff(kk), IDESC_SS, kk > 0 ? 1u : 0u);
         mma_commit(dpt_full);
-        // P^T, dS^T (tensor memory) and dS (shared memory) are ready.
-        if (!mbar_wait(pds_full, it & 1, abort_flag)) { ok = false; break; }
-        tc_fence_after();
         const uint32_t acc = it > 0 ? 1u : 0u;
         // P^T / dS^T of queries 64g .. 64g+63 sit in columns 64g .. 64g+31 of
         // their buffer (warpgroup g wrote them over scores it had read).
+        if (!mbar_wait(p_full, it & 1, abort_flag)) { ok = false; break; }
+        tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < BLOCK / 16; ++kk)  // dV += P^T dO_i
           mma_bf16_ts(tdV, tSt + (kk >> 2) * 64 + (kk & 3) * 8, dodM0 + soff + moff(kk),
                       IDESC_ACC, (acc | kk) ? 1u : 0u);
+        // dS^T (tensor memory) and dS (shared memory) are ready.
+        if (!mbar_wait(ds_full, it & 1, abort_flag)) { ok = false; break; }
+        tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < BLOCK / 16; ++kk)  // dK += dS^T Q_i
           mma_bf16_ts(tdK, tdPt + (kk >> 2) * 64 + (kk & 3) * 8, qdM0 + soff + moff(kk),
@@ -244,8 +268,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 #pragma unroll
         for (int kk = 0; kk < BLOCK / 16; ++kk)  // dQ_i = dS K_j (M = queries, K = keys)
           mma_bf16_ss(tdPt, dsdM + moff(kk), kdM + moff(kk), IDESC_DQ, kk > 0 ? 1u : 0u);
+        // Q_i / dO_i (stage st) are released by the dQ warps, which stage
+        // dQ_i there once it is complete.
         mma_commit(dq_full);
-        mma_commit(&qd_empty[st]);
       }
       if (ok) mma_commit(dkv_final);
       mma_commit(mma_final);
@@ -257,7 +282,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     const int g = warp >> 2;
     const int t = threadIdx.x - g * BLOCK;  // key row, TMEM lane
     const int key_g = key0 + t;
-    const bool key_ok = key_g < p.N;
+    const bool key_ok = key_g < p.Nk;
     const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
     const float sl2 = p.scale_log2;
     uint8_t* ds_row = smem + L::DS_OFF + g * PANEL_BYTES + t * 128;  // row t of panel g
@@ -266,68 +291,96 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     for (int it = 0; it < n_it; ++it) {
       const int st = it & 1;
       const int q0 = it_q0(it);
-      if (!mbar_wait_warp(st_full, it & 1, abort_flag) ||
-          !mbar_wait_warp(dpt_full, it & 1, abort_flag)) {
+      const float* lse_s = reinterpret_cast<const float*>(smem + L::LSE_OFF + st * 512);
+      const float* dd_s = reinterpret_cast<const float*>(smem + L::DD_OFF + st * 512);
+      // Queries at or beyond Nq, and queries that see no key at all, carry
+      // log2(e) * LSE = +inf in the padded table, so their P is exactly 0.
+      // Causal: key row t is kept for query q of the tile iff
+      // key0 + t <= q0 + q + causal_off, i.e. q >= t + delta; tiles with
+      // delta <= -(BLOCK - 1) keep everything.
+      const int delta = key0 - q0 - p.causal_off;
+      const bool diag = CAUSAL && (delta > -(BLOCK - 1));
+      // Phase 1: P^T = exp2(scale log2(e) S^T - log2(e) LSE) as bf16 pairs,
+      // over the score columns already read; kept in registers for phase 2.
+      if (!mbar_wait_warp(st_full, it & 1, abort_flag)) {
         ok = false;
         break;
       }
       tc_fence_after();
-      const float* lse_s = reinterpret_cast<const float*>(smem + L::LSE_OFF + st * 512);
-      const float* dd_s = reinterpret_cast<const float*>(smem + L::DD_OFF + st * 512);
-      // Queries at or beyond N carry log2(e) * LSE = +inf in the padded table,
-      // so their P is exactly 0; causal also drops queries before the key.
-      const bool diag = CAUSAL && (q0 == key0);
-#pragma unroll 1
-      for (int c = 64 * g; c < 64 * g + 64; c += 32) {
-        uint32_t sr[32], dr[32];
+      uint32_t pk[32];  // P^T row t, queries 64g .. 64g+63
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const int c = 64 * g + 32 * h;
+        uint32_t sr[32];
         tmem_ld32(tSt + lane_off + c, sr);
-        tmem_ld32(tdPt + lane_off + c, dr);
         tmem_ld_wait();
-        uint32_t pk[16], dk[16];
 #pragma unroll
         for (int e = 0; e < 32; e += 2) {
-          float pv[2], dv[2];
+          float pv[2];
 #pragma unroll
-          for (int h = 0; h < 2; ++h) {
-            const int q = c + e + h;
-            const float x = fmaf(__uint_as_float(sr[e + h]), sl2, -lse_s[q]);
-            float pp = ex2_approx(x);
-            bool keep = key_ok;
-            if (diag) keep = keep && (q >= t);
-            pp = keep ? pp : 0.f;
-            pv[h] = pp;
-            dv[h] = pp * (__uint_as_float(dr[e + h]) - dd_s[q]);
+          for (int u = 0; u < 2; ++u) {
+            const int q = c + e + u;
+            const float pp = ex2_approx(fmaf(__uint_as_float(sr[e + u]), sl2, -lse_s[q]));
+            const bool keep = key_ok && (!diag || q >= t + delta);
+            pv[u] = keep ? pp : 0.f;
           }
-          pk[e >> 1] = pack_bf16x2(pv[0], pv[1]);
-          dk[e >> 1] = pack_bf16x2(dv[0], dv[1]);
+          pk[16 * h + (e >> 1)] = pack_bf16x2(pv[0], pv[1]);
         }
-        // columns 64g + (c - 64g)/2: inside the range this warpgroup has read
-        const uint32_t pc = static_cast<uint32_t>(64 * g + ((c - 64 * g) >> 1));
-        tmem_st16(tSt + lane_off + pc, pk);
-        tmem_st16(tdPt + lane_off + pc, dk);
+        // columns 64g + 16h ..: inside the range this warpgroup has read
+        tmem_st16(tSt + lane_off + 64 * g + 16 * h, &pk[16 * h]);
+      }
+      tmem_st_wait();
+      tc_fence_before();
+      mbar_arrive(p_full);
+      // Phase 2: dS^T = P^T * (dP^T - D), into tensor memory over the dP^T
+      // columns already read and, transposed back, into the swizzled dS
+      // buffer for the dQ product.
+      if (!mbar_wait_warp(dpt_full, it & 1, abort_flag)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const int c = 64 * g + 32 * h;
+        uint32_t dr[32];
+        tmem_ld32(tdPt + lane_off + c, dr);
+        tmem_ld_wait();
+        uint32_t dk[16];
+#pragma unroll
+        for (int e = 0; e < 32; e += 2) {
+          const uint32_t w = pk[16 * h + (e >> 1)];
+          const float d0 = __uint_as_float(w << 16) * (__uint_as_float(dr[e]) - dd_s[c + e]);
+          const float d1 =
+              __uint_as_float(w & 0xFFFF0000u) * (__uint_as_float(dr[e + 1]) - dd_s[c + e + 1]);
+          dk[e >> 1] = pack_bf16x2(d0, d1);
+        }
+        tmem_st16(tdPt + lane_off + 64 * g + 16 * h, dk);
         // dS row t, queries c..c+31: panel g, 16-byte chunks (c%64)/8 .. +3,
         // 128-byte swizzle (chunk index xor row % 8).
-        uint8_t* prow = ds_row;
         const uint32_t ch0 = static_cast<uint32_t>((c & 63) >> 3);
 #pragma unroll
         for (int u = 0; u < 4; ++u) {
           const uint32_t ch = (ch0 + u) ^ sw;
-          *reinterpret_cast<uint4*>(prow + ch * 16) =
+          *reinterpret_cast<uint4*>(ds_row + ch * 16) =
               make_uint4(dk[4 * u], dk[4 * u + 1], dk[4 * u + 2], dk[4 * u + 3]);
         }
       }
       fence_proxy_async_smem();
       tmem_st_wait();
       tc_fence_before();
-      mbar_arrive(pds_full);
+      mbar_arrive(ds_full);
     }
-    // epilogue: warpgroup 0 writes dV, warpgroup 1 scale * dK, one key row per thread
+    // epilogue: warpgroup 0 writes dV, warpgroup 1 scale * dK, one key row per
+    // thread.  A key tile that no query sees (n_it = 0) never wrote its
+    // accumulators: it stores zeros.
     if (ok && mbar_wait_warp(dkv_final, 0, abort_flag)) {
       tc_fence_after();
-      const size_t rowoff = (static_cast<size_t>(bkv) * p.N + key_g) * D;
+      const size_t rowoff = (static_cast<size_t>(bkv) * p.Nk + key_g) * D;
       {
         const int which = g;
         const uint32_t tacc = which == 0 ? tdV : tdK;
+        const bool seen = n_it > 0;
         const float mul = which == 0 ? 1.f : p.scale;
         __nv_bfloat16* dst_row = (which == 0 ? p.dv : p.dk) + rowoff;
 #pragma unroll
@@ -338,7 +391,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           uint32_t pk[16];
 #pragma unroll
           for (int e = 0; e < 32; e += 2)
-            pk[e >> 1] = pack_bf16x2(__uint_as_float(r[e]) * mul, __uint_as_float(r[e + 1]) * mul);
+            pk[e >> 1] = seen ? pack_bf16x2(__uint_as_float(r[e]) * mul,
+                                            __uint_as_float(r[e + 1]) * mul)
+                              : 0u;
           if (key_ok) {
             uint4* dst = reinterpret_cast<uint4*>(dst_row + c);
 #pragma unroll
@@ -352,58 +407,61 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     tmem_st_wait();
   } else {
     // ------------------------------------------------------------ dQ reduction
-    // dQ_i (fp32, 128 query rows x d) leaves tensor memory 64 columns at a
-    // time through the dS buffer, which the dQ MMA has finished reading: two
-    // 128 x 32 fp32 boxes with the 128-byte swizzle, then one thread adds
-    // them to the accumulator with bulk tensor reductions.  dq_free is
-    // signalled once the staging buffer has been read, which also frees it
-    // for the next tile's dS (written only after the next dP^T, which waits
-    // for dq_free).
+    // dQ_i (fp32, 128 query rows x d) leaves tensor memory into the shared
+    // memory of the Q_i / dO_i stage it was computed from: every MMA that
+    // reads Q_i or dO_i precedes dQ_i, so the stage is free once dQ_i is
+    // complete.  It is written as d/32 boxes of 128 rows x 128 bytes with the
+    // 128-byte swizzle (boxes 0 .. d/64-1 over Q_i's panels, the rest over
+    // dO_i's), and one thread adds them to the fp32 accumulator with bulk
+    // tensor reductions (performed in L2).  dq_free is signalled as soon as
+    // the tensor-memory reads are done; the stage goes back to the producer
+    // (qd_empty) once the reductions have read it.
     const int t = threadIdx.x - 2 * BLOCK;  // query row of the dQ tile, TMEM lane
     const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
-    uint8_t* stage = smem + L::DS_OFF;      // 2 boxes of 128 rows x 128 bytes
     const uint32_t sw = static_cast<uint32_t>(t & 7);
-    int rounds = 0;  // staging rounds so far
-    bool ok = true;
-    for (int it = 0; ok && it < n_it; ++it) {
+    constexpr int NBOX = D / 32;
+    auto box_addr = [&](int st, int b) {
+      return b < L::NPANEL ? smem + L::Q_OFF + st * L::TILE + b * PANEL_BYTES
+                           : smem + L::DO_OFF + st * L::TILE + (b - L::NPANEL) * PANEL_BYTES;
+    };
+    for (int it = 0; it < n_it; ++it) {
+      const int st = it & 1;
       const int q0 = it_q0(it);
       const int bh = it_head(it);
       if (!mbar_wait_warp(dq_full, it & 1, abort_flag)) break;
       tc_fence_after();
-#pragma unroll 1
-      for (int h = 0; h < D / 64; ++h, ++rounds) {
-        uint32_t r[2][32];
-        tmem_ld32(tdPt + lane_off + 64 * h, r[0]);
-        tmem_ld32(tdPt + lane_off + 64 * h + 32, r[1]);
-        tmem_ld_wait();
 #pragma unroll
-        for (int b = 0; b < 2; ++b) {
-          uint8_t* row = stage + b * PANEL_BYTES + t * 128;
+      for (int b2 = 0; b2 < NBOX; b2 += 2) {
+        uint32_t r[2][32];
+        tmem_ld32(tdPt + lane_off + 32 * b2, r[0]);
+        tmem_ld32(tdPt + lane_off + 32 * b2 + 32, r[1]);
+        tmem_ld_wait();
+        if (b2 + 2 == NBOX) {
+          // all of dQ_i is in registers or shared memory: the next dP^T may
+          // overwrite these columns
+          tc_fence_before();
+          mbar_arrive(dq_free);
+        }
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+          uint8_t* row = box_addr(st, b2 + u) + t * 128;
 #pragma unroll
           for (int c = 0; c < 8; ++c)
             *reinterpret_cast<uint4*>(row + ((c ^ sw) << 4)) =
-                make_uint4(r[b][4 * c], r[b][4 * c + 1], r[b][4 * c + 2], r[b][4 * c + 3]);
-        }
-        fence_proxy_async_smem();
-        mbar_arrive(stg_full);
-        if (t == 0) {
-          if (mbar_wait(stg_full, rounds & 1, abort_flag)) {
-            tma_reduce_add_3d(&tm_dq, stage, 64 * h, q0, bh);
-            tma_reduce_add_3d(&tm_dq, stage + PANEL_BYTES, 64 * h + 32, q0, bh);
-            bulk_commit_group();
-            bulk_wait_group_read0();
-          }
-          mbar_arrive(stg_free);
-        }
-        // the staging buffer may be rewritten once the reduction has read it
-        if (!mbar_wait_warp(stg_free, rounds & 1, abort_flag)) {
-          ok = false;
-          break;
+                make_uint4(r[u][4 * c], r[u][4 * c + 1], r[u][4 * c + 2], r[u][4 * c + 3]);
         }
       }
-      if (!ok) break;
-      tc_fence_before();
-      mbar_arrive(dq_free);
+      fence_proxy_async_smem();
+      mbar_arrive(stg_full);
+      if (t == 0) {
+        if (!mbar_wait(stg_full, it & 1, abort_flag)) break;
+#pragma unroll
+        for (int b = 0; b < NBOX; ++b) tma_reduce_add_3d(&tm_dq, box_addr(st, b), 32 * b, q0, bh);
+        bulk_commit_group();
+        bulk_wait_group_read0();
+        // Q_i / dO_i (stage st) may be reloaded
+        mbar_arrive(&qd_empty[st]);
+      }
     }
     if (t == 0) bulk_wait_group0();
     tmem_ld_wait();
@@ -420,6 +478,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 
 // For every padded row (bh, n), n < Np: D = sum_k dO_k O_k and
 // lse2 = log2(e) * LSE when n < N, else D = 0 and lse2 = +inf; and dQacc = 0.
+// A row whose LSE is -inf saw no key; its lse2 is +inf as well, so that every
+// P of it is exactly 0.
 template <int D>
 __global__ void __launch_bounds__(256)
     fa_bwd_preprocess_kernel(const __nv_bfloat16* __restrict__ o,
@@ -455,7 +515,8 @@ __global__ void __launch_bounds__(256)
   for (int off = LPR / 2; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
   if (prow < padded_rows && sub == 0) {
     dd[prow] = real ? acc : 0.f;
-    lse2[prow] = real ? lse[row] * LOG2E : INFINITY;
+    const float l = real ? lse[row] : INFINITY;
+    lse2[prow] = (l == -INFINITY) ? INFINITY : l * LOG2E;
   }
 }
 
@@ -482,7 +543,7 @@ fa_status launch_main(const CUtensorMap* maps, const Params& prm, int BH, cudaSt
       return FA_ERR_CUDA;
     configured = true;
   }
-  dim3 grid(prm.n_tiles * BH);
+  dim3 grid(prm.n_kt * BH);
   kern<<<grid, NUM_THREADS, Smem<D>::ALLOC, stream>>>(maps[0], maps[1], maps[2], maps[3], maps[4],
                                                       maps[5], maps[6], prm);
   return cuda_status(cudaGetLastError());
@@ -492,12 +553,25 @@ fa_status launch_main(const CUtensorMap* maps, const Params& prm, int BH, cudaSt
 
 fa_status launch_bwd(const void* q, const void* k, const void* v, const void* o,
                      const void* dout, const float* lse, void* dq, void* dk, void* dv,
-                     void* workspace, int B, int H, int Hkv, int N, int d, int causal,
+                     void* workspace, int B, int H, int Hkv, int Nq, int Nk, int d, int causal,
                      float scale, cudaStream_t stream) {
   const int BH = B * H;
   const int BHkv = B * Hkv;
-  const long long rows = static_cast<long long>(BH) * N;
-  const int Np = static_cast<int>(bwd_row_pad(N));
+  // No queries: no gradient reaches K or V.  No keys: O was 0 whatever Q was.
+  if (Nq == 0 || Nk == 0) {
+    if (Nq == 0 && Nk > 0) {
+      const size_t kv = static_cast<size_t>(BHkv) * Nk * d * 2;
+      if (cudaMemsetAsync(dk, 0, kv, stream) != cudaSuccess ||
+          cudaMemsetAsync(dv, 0, kv, stream) != cudaSuccess)
+        return FA_ERR_CUDA;
+    }
+    if (Nk == 0 && Nq > 0 &&
+        cudaMemsetAsync(dq, 0, static_cast<size_t>(BH) * Nq * d * 2, stream) != cudaSuccess)
+      return FA_ERR_CUDA;
+    return FA_OK;
+  }
+  const long long rows = static_cast<long long>(BH) * Nq;
+  const int Np = static_cast<int>(bwd_row_pad(Nq));
   const long long prows = static_cast<long long>(BH) * Np;
   const size_t table = align_up(static_cast<size_t>(prows) * 4, 256);
   float* dd = static_cast<float*>(workspace);
@@ -510,30 +584,50 @@ fa_status launch_bwd(const void* q, const void* k, const void* v, const void* o,
     if (d == 128)
       bwd::fa_bwd_preprocess_kernel<128><<<static_cast<unsigned>(blocks), 256, 0, stream>>>(
           static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(dout), lse, dd,
-          lse2, dqacc, N, Np, prows);
+          lse2, dqacc, Nq, Np, prows);
     else
       bwd::fa_bwd_preprocess_kernel<64><<<static_cast<unsigned>(blocks), 256, 0, stream>>>(
           static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(dout), lse, dd,
-          lse2, dqacc, N, Np, prows);
+          lse2, dqacc, Nq, Np, prows);
     if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
   }
   // 2. dK, dV and the dQ accumulation
   CUtensorMap maps[7];
   fa_status st;
-  if ((st = make_tmap_bf16_3d(&maps[0], q, d, N, BH, bwd::BLOCK)) != FA_OK) return st;
-  if ((st = make_tmap_bf16_3d(&maps[1], k, d, N, BHkv, bwd::BLOCK)) != FA_OK) return st;
-  if ((st = make_tmap_bf16_3d(&maps[2], v, d, N, BHkv, bwd::BLOCK)) != FA_OK) return st;
-  if ((st = make_tmap_bf16_3d(&maps[3], dout, d, N, BH, bwd::BLOCK)) != FA_OK) return st;
+  if ((st = make_tmap_bf16_3d(&maps[0], q, d, Nq, BH, bwd::BLOCK)) != FA_OK) return st;
+  if ((st = make_tmap_bf16_3d(&maps[1], k, d, Nk, BHkv, bwd::BLOCK)) != FA_OK) return st;
+  if ((st = make_tmap_bf16_3d(&maps[2], v, d, Nk, BHkv, bwd::BLOCK)) != FA_OK) return st;
+  if ((st = make_tmap_bf16_3d(&maps[3], dout, d, Nq, BH, bwd::BLOCK)) != FA_OK) return st;
   if ((st = make_tmap_f32_2d(&maps[4], lse2, Np, BH)) != FA_OK) return st;
   if ((st = make_tmap_f32_2d(&maps[5], dd, Np, BH)) != FA_OK) return st;
-  if ((st = make_tmap_f32_3d_sw128(&maps[6], dqacc, d, N, BH)) != FA_OK) return st;
+  if ((st = make_tmap_f32_3d_sw128(&maps[6], dqacc, d, Nq, BH)) != FA_OK) return st;
   bwd::Params prm;
   prm.dk = static_cast<__nv_bfloat16*>(dk);
   prm.dv = static_cast<__nv_bfloat16*>(dv);
   prm.dqacc = dqacc;
-  prm.N = N;
-  prm.n_tiles = (N + bwd::BLOCK - 1) / bwd::BLOCK;
+  prm.Nq = Nq;
+  prm.Nk = Nk;
+  prm.causal_off = Nk - Nq;
+  prm.n_qt = (Nq + bwd::BLOCK - 1) / bwd::BLOCK;
+  prm.n_kt = (Nk + bwd::BLOCK - 1) / bwd::BLOCK;
   prm.group = H / Hkv;
+  prm.BHkv = BHkv;
+  {
+    // Causal CTAs differ in length (later key tiles see fewer query tiles);
+    // when there are only a few waves of them, launching the longest first
+    // shortens the tail.  FA_BWD_ORDER=head|lpt forces one.
+    static int mode = -1;
+    if (mode < 0) {
+      const char* env = std::getenv("FA_BWD_ORDER");
+      mode = (env && std::strcmp(env, "head") == 0) ? 1 : (env && std::strcmp(env, "lpt") == 0) ? 2 : 0;
+    }
+    int dev = 0, sms = 148;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+      return FA_ERR_CUDA;
+    const long long ctas = static_cast<long long>(prm.n_kt) * BHkv;
+    prm.lpt_order = (mode == 2 || (mode == 0 && causal && ctas < 8LL * sms)) ? 1 : 0;
+  }
   prm.scale_log2 = scale * bwd::LOG2E;
   prm.scale = scale;
   if (d == 128)

@@ -82,10 +82,12 @@ struct Smem {
 struct Params {
   __nv_bfloat16* o;
   float* lse;
-  int N;
+  int Nq;            // query rows per head
+  int Nk;            // key / value rows per head
+  int causal_off;    // Nk - Nq: query i sits at key position i + causal_off
   int BH;
   int group;         // query heads per key/value head (1 without grouping)
-  int n_cta_tiles;   // ceil(N / 256)
+  int n_cta_tiles;   // ceil(Nq / 256)
   int total_items;   // BH * n_cta_tiles
   int lpt_order;     // 1: all heads' longest tiles first; 0: head-major
   float scale_log2;  // scale * log2(e)
@@ -145,11 +147,15 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   const int lane = threadIdx.x & 31;
   const int G = static_cast<int>(gridDim.x);
   const int cta = static_cast<int>(blockIdx.x);
-  const int n_kv_total = (p.N + BLOCK_N - 1) / BLOCK_N;
-  // key tiles seen by query tile w of 256-row tile `tile` (causal: up to its
-  // own diagonal tile)
+  const int n_kv_total = (p.Nk + BLOCK_N - 1) / BLOCK_N;  // >= 1
+  // Key tiles seen by query tile w of 256-row tile `tile`; causal: up to the
+  // tile holding the last admissible key of its last row.  At least one, so
+  // that a tile whose rows see no key at all (only when Nq > Nk) still runs
+  // the pipeline once and comes out fully masked: O = 0, LSE = -inf.
   auto n_kv_of = [&](int tile, int w) {
-    return CAUSAL ? min(2 * tile + 1 + w, n_kv_total) : n_kv_total;
+    if (!CAUSAL) return n_kv_total;
+    const int last_key = tile * BLOCK_M + w * TILE_M + TILE_M - 1 + p.causal_off;
+    return last_key < 0 ? 1 : min(last_key / BLOCK_N + 1, n_kv_total);
   };
 
   if (threadIdx.x == 0) {
@@ -361,11 +367,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         tmem_ld32(tS + 96, *reinterpret_cast<uint32_t(*)[32]>(&sr[96]));
         tmem_ld_wait();
         const int key0 = j * BLOCK_N;
-        const bool need_mask = (key0 + BLOCK_N > p.N) || (CAUSAL && key0 + BLOCK_N - 1 > q_row0);
+        const bool need_mask = (key0 + BLOCK_N > p.Nk) ||
+                               (CAUSAL && key0 + BLOCK_N - 1 > q_row0 + p.causal_off);
         // four independent max chains (latency, not throughput, bounds this loop)
         float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
         if (need_mask) {
-          const int lim = CAUSAL ? min(p.N - 1, row_g) : p.N - 1;  // last admissible key
+          // last admissible key (below 0: none, the row stays at -inf)
+          const int lim = CAUSAL ? min(p.Nk - 1, row_g + p.causal_off) : p.Nk - 1;
 #pragma unroll
           for (int c = 0; c < 128; ++c) {
             const float s = (key0 + c <= lim) ? __uint_as_float(sr[c]) : -INFINITY;
@@ -378,7 +386,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         }
         // scale * log2(e) > 0, so the maximum of the scaled row is the scaled maximum
         const float m_new = fmaxf(m, fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])) * sl2);
-        const bool grow = (m_new - m) > RESCALE_THRESHOLD;  // true when m = -inf
+        // true when m = -inf < m_new; false while the whole row is masked
+        const bool grow = (m_new - m) > RESCALE_THRESHOLD;
         const bool warp_grow = __any_sync(0xffffffffu, grow);
         const float m_use = warp_grow ? m_new : m;
         const float m_ref = (m_use == -INFINITY) ? 0.f : m_use;
@@ -439,8 +448,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       }
       tc_fence_after();
       const float inv_l = (l > 0.f) ? 1.f / l : 0.f;
-      const bool valid = row_g < p.N;
-      __nv_bfloat16* orow_g = p.o + (static_cast<size_t>(bh) * p.N + row_g) * D;
+      const bool valid = row_g < p.Nq;
+      __nv_bfloat16* orow_g = p.o + (static_cast<size_t>(bh) * p.Nq + row_g) * D;
 #pragma unroll
       for (int c = 0; c < D; c += 32) {
         uint32_t orow[32];
@@ -464,7 +473,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       if (valid && p.lse != nullptr) {
         // LSE = ln(sum exp(scale * s)) = (m + log2 l) * ln 2, m in log2 units.
         const float lse = (l > 0.f) ? (m + lg2_approx(l)) * 0.6931471805599453f : -INFINITY;
-        p.lse[static_cast<size_t>(bh) * p.N + row_g] = lse;
+        p.lse[static_cast<size_t>(bh) * p.Nq + row_g] = lse;
       }
       pv_base += n_kv;
     }
@@ -511,27 +520,47 @@ int schedule_mode() {
   return mode;
 }
 
+// Rows with no key at all (Nk = 0): O = 0, LSE = -inf, the same values the
+// main kernel gives a fully masked row.
+__global__ void fa_fwd_no_keys_kernel(__nv_bfloat16* o, float* lse, size_t rows, int d) {
+  const size_t stride = static_cast<size_t>(gridDim.x) * blockDim.x;
+  const size_t n_o = rows * static_cast<size_t>(d) / 8;  // uint4 = 8 bf16
+  for (size_t i = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; i < n_o; i += stride)
+    reinterpret_cast<uint4*>(o)[i] = make_uint4(0u, 0u, 0u, 0u);
+  if (lse != nullptr)
+    for (size_t i = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; i < rows;
+         i += stride)
+      lse[i] = -INFINITY;
+}
+
 }  // namespace fwd
 
 fa_status launch_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B,
-                     int H, int Hkv, int N, int d, int causal, float scale, cudaStream_t stream) {
+                     int H, int Hkv, int Nq, int Nk, int d, int causal, float scale,
+                     cudaStream_t stream) {
   const int BH = B * H;
-  const long long n_cta_tiles = (N + fwd::BLOCK_M - 1) / fwd::BLOCK_M;
-  const long long items = static_cast<long long>(BH) * n_cta_tiles;
-  if (items > 0x7fffffffLL) return FA_ERR_INVALID_ARG;
-  CUtensorMap tq, tk, tv;
-  fa_status st;
-  if ((st = make_tmap_bf16_3d(&tq, q, d, N, BH, fwd::TILE_M)) != FA_OK) return st;
-  // K and V carry B * Hkv heads; query head bh reads key/value head bh / (H / Hkv)
-  if ((st = make_tmap_bf16_3d(&tk, k, d, N, static_cast<uint64_t>(B) * Hkv, fwd::BLOCK_N)) != FA_OK)
-    return st;
-  if ((st = make_tmap_bf16_3d(&tv, v, d, N, static_cast<uint64_t>(B) * Hkv, fwd::BLOCK_N)) != FA_OK)
-    return st;
+  if (Nq == 0) return FA_OK;
   int dev = 0, sms = 148;
   if (cudaGetDevice(&dev) != cudaSuccess ||
       cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
     return FA_ERR_CUDA;
-  const double kv_bytes = 4.0 * B * Hkv * static_cast<double>(N) * d;
+  if (Nk == 0) {
+    fwd::fa_fwd_no_keys_kernel<<<4 * sms, 256, 0, stream>>>(
+        static_cast<__nv_bfloat16*>(o), lse, static_cast<size_t>(BH) * Nq, d);
+    return cuda_status(cudaGetLastError());
+  }
+  const long long n_cta_tiles = (Nq + fwd::BLOCK_M - 1) / fwd::BLOCK_M;
+  const long long items = static_cast<long long>(BH) * n_cta_tiles;
+  if (items > 0x7fffffffLL) return FA_ERR_INVALID_ARG;
+  CUtensorMap tq, tk, tv;
+  fa_status st;
+  if ((st = make_tmap_bf16_3d(&tq, q, d, Nq, BH, fwd::TILE_M)) != FA_OK) return st;
+  // K and V carry B * Hkv heads of Nk rows; query head bh reads key/value head
+  // bh / (H / Hkv)
+  const uint64_t BHkv = static_cast<uint64_t>(B) * Hkv;
+  if ((st = make_tmap_bf16_3d(&tk, k, d, Nk, BHkv, fwd::BLOCK_N)) != FA_OK) return st;
+  if ((st = make_tmap_bf16_3d(&tv, v, d, Nk, BHkv, fwd::BLOCK_N)) != FA_OK) return st;
+  const double kv_bytes = 4.0 * B * Hkv * static_cast<double>(Nk) * d;
   const int mode = fwd::schedule_mode();
   bool persistent = causal && items > sms && kv_bytes <= 96.0 * 1024 * 1024;
   int grid = persistent ? sms : static_cast<int>(items);
@@ -545,7 +574,9 @@ fa_status launch_fwd(const void* q, const void* k, const void* v, void* o, float
   fwd::Params prm;
   prm.o = static_cast<__nv_bfloat16*>(o);
   prm.lse = lse;
-  prm.N = N;
+  prm.Nq = Nq;
+  prm.Nk = Nk;
+  prm.causal_off = Nk - Nq;
   prm.BH = BH;
   prm.group = H / Hkv;
   prm.n_cta_tiles = static_cast<int>(n_cta_tiles);

@@ -32,18 +32,25 @@ fa_status make_tmap_f32_3d_sw128(CUtensorMap* map, const void* base, uint64_t d,
 inline size_t bwd_row_pad(int N) { return (static_cast<size_t>(N) + 127) / 128 * 128; }
 
 // Hkv = number of key/value heads; H (query heads) is a multiple of it.
+// Nq query rows, Nk key rows per head; causal masking keeps j <= i + Nk - Nq.
 fa_status launch_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B,
-                     int H, int Hkv, int N, int d, int causal, float scale, cudaStream_t stream);
+                     int H, int Hkv, int Nq, int Nk, int d, int causal, float scale,
+                     cudaStream_t stream);
 
 fa_status launch_bwd(const void* q, const void* k, const void* v, const void* o,
                      const void* dout, const float* lse, void* dq, void* dk, void* dv,
-                     void* workspace, int B, int H, int Hkv, int N, int d, int causal,
+                     void* workspace, int B, int H, int Hkv, int Nq, int Nk, int d, int causal,
                      float scale, cudaStream_t stream);
 
 int decode_num_splits(int Lmax);
+// page_table == nullptr: contiguous caches [B, Hkv, Lmax, d].  Otherwise paged
+// pools [num_pages, Hkv, 1 << log2_page, d] addressed through
+// page_table[B, pages_per_seq], with Lmax = pages_per_seq << log2_page.
 fa_status launch_decode(const void* q, const void* kc, const void* vc, const int* seqlens,
                         void* o, float* lse, int B, int H, int Hkv, int Lmax, int d,
-                        float scale, float* partials, cudaStream_t stream);
+                        float scale, float* partials, cudaStream_t stream,
+                        const int* page_table = nullptr, int pages_per_seq = 0,
+                        int log2_page = 0, int num_pages = 0);
 
 inline fa_status cuda_status(cudaError_t e) { return e == cudaSuccess ? FA_OK : FA_ERR_CUDA; }
 

@@ -30,14 +30,19 @@ _P, _I, _F, _S = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
 SIGNATURES = {
     "fa_fwd": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _P]),
     "fa_fwd_gqa": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _P]),
+    "fa_fwd_ext": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _F, _P]),
     "fa_bwd_workspace_size": (_S, [_I, _I, _I, _I]),
     "fa_bwd": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _S, _I, _I, _I, _I, _I, _F, _P]),
     "fa_bwd_gqa": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _S, _I, _I, _I, _I, _I, _I, _F,
                         _P]),
+    "fa_bwd_ext": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _S, _I, _I, _I, _I, _I, _I, _I,
+                        _F, _P]),
     "fa_decode_workspace_size": (_S, [_I, _I, _I, _I]),
     "fa_decode": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _F, _P, _S, _P]),
     "fa_decode_gqa": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _P, _S, _P]),
     "fa_decode_static": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _F, _P]),
+    "fa_decode_paged": (_I, [_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _F, _P, _S,
+                             _P]),
     "fa_get_device_error": (_I, [_P]),
     "fa_status_string": (ctypes.c_char_p, [_I]),
     "fa_version": (_I, []),
@@ -104,14 +109,16 @@ def _ptr(t: Optional[torch.Tensor]) -> Optional[int]:
 def fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, causal: bool = False,
         scale: Optional[float] = None, out: Optional[torch.Tensor] = None,
         lse: Optional[torch.Tensor] = None, want_lse: bool = True, stream=None):
-    """Exact attention forward.  q: bf16 [B, H, N, d]; k, v: bf16 [B, Hkv, N, d]
-    with Hkv dividing H (Hkv < H: grouped-query attention).  Returns (o, lse)."""
+    """Exact attention forward.  q: bf16 [B, H, Nq, d]; k, v: bf16 [B, Hkv, Nk, d]
+    with Hkv dividing H (Hkv < H: grouped-query attention).  With Nq != Nk the
+    queries are the last Nq positions of the key sequence (causal mask
+    j <= i + Nk - Nq).  Returns (o [B, H, Nq, d], lse [B, H, Nq])."""
     for t, n in ((q, "q"), (k, "k"), (v, "v")):
         _req(t, n, torch.bfloat16, 4)
     B, H, N, d = q.shape
-    Hkv = k.shape[1]
-    if (tuple(k.shape) != (B, Hkv, N, d) or v.shape != k.shape or Hkv < 1 or H % Hkv):
-        raise ValueError("k and v must be [B, Hkv, N, d] with Hkv dividing q's H")
+    Hkv, Nk = k.shape[1], k.shape[2]
+    if (tuple(k.shape) != (B, Hkv, Nk, d) or v.shape != k.shape or Hkv < 1 or H % Hkv):
+        raise ValueError("k and v must be [B, Hkv, Nk, d] with Hkv dividing q's H")
     scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
     if out is None:
         out = torch.empty_like(q)
@@ -124,9 +131,9 @@ def fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, causal: bool = False,
         _req(lse, "lse", torch.float32, 3)
         if tuple(lse.shape) != (B, H, N):
             raise ValueError("lse must be [B, H, N]")
-    st = lib().fa_fwd_gqa(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), _ptr(lse),
-                          B, H, Hkv, N, d, int(bool(causal)), scale, _stream_ptr(stream))
-    _check("fa_fwd_gqa", st)
+    st = lib().fa_fwd_ext(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), _ptr(lse),
+                          B, H, Hkv, N, Nk, d, int(bool(causal)), scale, _stream_ptr(stream))
+    _check("fa_fwd_ext", st)
     return out, lse
 
 
@@ -137,15 +144,15 @@ def bwd_workspace_size(B: int, H: int, N: int, d: int) -> int:
 def bwd(q, k, v, o, do, lse, causal: bool = False, scale: Optional[float] = None,
         dq=None, dk=None, dv=None, workspace: Optional[torch.Tensor] = None, stream=None):
     """Backward with recomputation.  Returns (dq, dk, dv); dk and dv have k's
-    shape [B, Hkv, N, d] (grouped heads accumulate over their query heads)."""
+    shape [B, Hkv, Nk, d] (grouped heads accumulate over their query heads)."""
     for t, n in ((q, "q"), (k, "k"), (v, "v"), (o, "o"), (do, "do")):
         _req(t, n, torch.bfloat16, 4)
     B, H, N, d = q.shape
-    Hkv = k.shape[1]
+    Hkv, Nk = k.shape[1], k.shape[2]
     if o.shape != q.shape or do.shape != q.shape:
         raise ValueError("o and do must match q's shape")
-    if tuple(k.shape) != (B, Hkv, N, d) or v.shape != k.shape or H % Hkv:
-        raise ValueError("k and v must be [B, Hkv, N, d] with Hkv dividing q's H")
+    if tuple(k.shape) != (B, Hkv, Nk, d) or v.shape != k.shape or H % Hkv:
+        raise ValueError("k and v must be [B, Hkv, Nk, d] with Hkv dividing q's H")
     _req(lse, "lse", torch.float32, 3)
     if tuple(lse.shape) != (B, H, N):
         raise ValueError("lse must be [B, H, N]")
@@ -160,11 +167,11 @@ def bwd(q, k, v, o, do, lse, causal: bool = False, scale: Optional[float] = None
         workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=q.device)
     if dq.shape != q.shape or dk.shape != k.shape or dv.shape != v.shape:
         raise ValueError("gradient buffers must match q, k, v")
-    st = lib().fa_bwd_gqa(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), do.data_ptr(),
+    st = lib().fa_bwd_ext(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), do.data_ptr(),
                           lse.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(),
                           workspace.data_ptr(), workspace.numel() * workspace.element_size(),
-                          B, H, Hkv, N, d, int(bool(causal)), scale, _stream_ptr(stream))
-    _check("fa_bwd_gqa", st)
+                          B, H, Hkv, N, Nk, d, int(bool(causal)), scale, _stream_ptr(stream))
+    _check("fa_bwd_ext", st)
     return dq, dk, dv
 
 
@@ -199,6 +206,42 @@ def decode(q, kcache, vcache, seqlens, scale: Optional[float] = None, out=None, 
                              scale, workspace.data_ptr(),
                              workspace.numel() * workspace.element_size(), _stream_ptr(stream))
     _check("fa_decode_gqa", st)
+    return out, lse
+
+
+def decode_paged(q, kpages, vpages, block_table, seqlens, scale: Optional[float] = None,
+                 out=None, lse=None, want_lse: bool = True,
+                 workspace: Optional[torch.Tensor] = None, stream=None):
+    """Decode over a paged cache.  q [B,H,d] bf16; kpages/vpages
+    [num_pages, Hkv, page_size, d] bf16; block_table int32 [B, pages_per_seq]
+    and seqlens int32 [B] on the device.  Returns (o [B,H,d], lse [B,H])."""
+    _req(q, "q", torch.bfloat16, 3)
+    _req(kpages, "kpages", torch.bfloat16, 4)
+    _req(vpages, "vpages", torch.bfloat16, 4)
+    _req(block_table, "block_table", torch.int32, 2)
+    _req(seqlens, "seqlens", torch.int32, 1)
+    B, H, d = q.shape
+    num_pages, Hkv, page_size = kpages.shape[0], kpages.shape[1], kpages.shape[2]
+    if (tuple(kpages.shape) != (num_pages, Hkv, page_size, d) or vpages.shape != kpages.shape
+            or H % Hkv):
+        raise ValueError("page pools must be [num_pages, Hkv, page_size, d] with Hkv dividing H")
+    if block_table.shape[0] != B or seqlens.shape[0] != B:
+        raise ValueError("block_table and seqlens must have B rows")
+    pages_per_seq = block_table.shape[1]
+    scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
+    out = torch.empty_like(q) if out is None else out
+    _req(out, "out", torch.bfloat16, 3)
+    if lse is None and want_lse:
+        lse = torch.empty((B, H), dtype=torch.float32, device=q.device)
+    need = decode_workspace_size(B, H, pages_per_seq * page_size, d)
+    if workspace is None:
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=q.device)
+    st = lib().fa_decode_paged(q.data_ptr(), kpages.data_ptr(), vpages.data_ptr(),
+                               block_table.data_ptr(), seqlens.data_ptr(), out.data_ptr(),
+                               _ptr(lse), B, H, Hkv, page_size, pages_per_seq, num_pages, d,
+                               scale, workspace.data_ptr(),
+                               workspace.numel() * workspace.element_size(), _stream_ptr(stream))
+    _check("fa_decode_paged", st)
     return out, lse
 
 

@@ -7,7 +7,8 @@ explicitly, so both the CUDA path and the fp64 oracle see bit-identical inputs.
 Recipe (the pages' seed 42 is the base; each workload adds its index):
 
 * forward:  q, k, v ~ iid N(0,1) * std, drawn in that order as float32, then
-  rounded to bf16 (round-to-nearest-even);
+  rounded to bf16 (round-to-nearest-even); k and v may have fewer heads
+  (grouped queries) and another length than q;
 * backward: q, k, v, dO drawn in that order the same way;
 * decode:   seqlens ~ U{Lmin .. Lmax} (both ends inclusive) first, then
   q ~ N(0,1) [B, H, d], then for each sequence b in order: K_b, V_b ~ N(0,1)
@@ -39,6 +40,7 @@ class Workload:
     Lmax: int = 0
     seed: int = BASE_SEED
     Hkv: int = 0         # key/value heads (0: same as H; fewer: grouped-query attention)
+    page: int = 0        # decode: rows per cache page (0: contiguous cache)
 
     @property
     def kv_heads(self) -> int:
@@ -71,6 +73,9 @@ WORKLOADS = {
                  causal=True, seed=BASE_SEED + 6, Hkv=8),
         Workload("decode_gqa_B16_H32_Hkv8_d128_L4096-16384", "decode", 16, 32, 128,
                  Lmin=4096, Lmax=16384, seed=BASE_SEED + 7, Hkv=8),
+        # the decode workload over a paged cache (16-row pages, random page order)
+        Workload("decode_paged_B16_H32_d128_L4096-16384_p16", "decode", 16, 32, 128,
+                 Lmin=4096, Lmax=16384, seed=BASE_SEED + 8, page=16),
     )
 }
 
@@ -87,22 +92,25 @@ def _randn_bf16(g: torch.Generator, shape, std: float = 1.0) -> torch.Tensor:
 
 
 def fwd_inputs(B: int, H: int, N: int, d: int, seed: int, std: float = 1.0,
-               Hkv: int | None = None):
-    """q [B, H, N, d] and k, v [B, Hkv, N, d] (Hkv defaults to H) as contiguous
-    bf16 CPU tensors."""
+               Hkv: int | None = None, Nk: int | None = None):
+    """q [B, H, N, d] and k, v [B, Hkv, Nk, d] (Hkv defaults to H, Nk to N) as
+    contiguous bf16 CPU tensors."""
     g = _gen(seed)
     hk = Hkv or H
-    return (_randn_bf16(g, (B, H, N, d), std), _randn_bf16(g, (B, hk, N, d), std),
-            _randn_bf16(g, (B, hk, N, d), std))
+    nk = N if Nk is None else Nk
+    return (_randn_bf16(g, (B, H, N, d), std), _randn_bf16(g, (B, hk, nk, d), std),
+            _randn_bf16(g, (B, hk, nk, d), std))
 
 
 def bwd_inputs(B: int, H: int, N: int, d: int, seed: int, std: float = 1.0,
-               Hkv: int | None = None):
-    """q, k, v, dO as contiguous bf16 CPU tensors (k, v with Hkv heads)."""
+               Hkv: int | None = None, Nk: int | None = None):
+    """q, k, v, dO as contiguous bf16 CPU tensors (k, v with Hkv heads of Nk
+    rows)."""
     g = _gen(seed)
     hk = Hkv or H
-    return (_randn_bf16(g, (B, H, N, d), std), _randn_bf16(g, (B, hk, N, d), std),
-            _randn_bf16(g, (B, hk, N, d), std), _randn_bf16(g, (B, H, N, d), std))
+    nk = N if Nk is None else Nk
+    return (_randn_bf16(g, (B, H, N, d), std), _randn_bf16(g, (B, hk, nk, d), std),
+            _randn_bf16(g, (B, hk, nk, d), std), _randn_bf16(g, (B, H, N, d), std))
 
 
 def decode_inputs(B: int, H: int, d: int, Lmin: int, Lmax: int, seed: int,
@@ -130,6 +138,37 @@ def decode_inputs(B: int, H: int, d: int, Lmin: int, Lmax: int, seed: int,
         kc[b, :, :L] = _randn_bf16(g, (hk, L, d))
         vc[b, :, :L] = _randn_bf16(g, (hk, L, d))
     return q, kc, vc, seqlens.to(torch.int32)
+
+
+def page_cache(kc: torch.Tensor, vc: torch.Tensor, seqlens, page_size: int, seed: int,
+               spare_pages: int = 3):
+    """Scatter contiguous caches [B, Hkv, Lcap, d] into page pools
+    [num_pages, Hkv, page_size, d] in a seeded random page order.
+
+    Returns (kpages, vpages, block_table int32 [B, pages_per_seq]).  Logical
+    page p of sequence b goes to pool page block_table[b, p]; table entries
+    past a sequence's last page are -1, and the ``spare_pages`` pool pages
+    that no sequence uses, like the rows past a sequence's end, hold NaN.
+    Pure data movement: no attention arithmetic."""
+    B, hk, Lcap, d = kc.shape
+    pps = -(-Lcap // page_size)
+    seqlens = torch.as_tensor(seqlens, dtype=torch.int64)
+    used = [int(-(-int(seqlens[b]) // page_size)) for b in range(B)]
+    num_pages = sum(used) + spare_pages
+    perm = torch.randperm(num_pages, generator=_gen(seed))
+    kp = torch.full((num_pages, hk, page_size, d), float("nan"), dtype=kc.dtype)
+    vp = torch.full((num_pages, hk, page_size, d), float("nan"), dtype=vc.dtype)
+    table = torch.full((B, pps), -1, dtype=torch.int32)
+    nxt = 0
+    for b in range(B):
+        for p in range(used[b]):
+            page = int(perm[nxt])
+            nxt += 1
+            table[b, p] = page
+            r0, r1 = p * page_size, min((p + 1) * page_size, Lcap)
+            kp[page, :, :r1 - r0] = kc[b, :, r0:r1]
+            vp[page, :, :r1 - r0] = vc[b, :, r0:r1]
+    return kp, vp, table
 
 
 def workload_inputs(w: Workload):

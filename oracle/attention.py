@@ -183,7 +183,8 @@ def attention_backward(q: np.ndarray, k: np.ndarray, v: np.ndarray,
         dS = P * (dP - D)          (zero where masked, since P is zero there)
         dQ = scale * dS K
         dK = scale * dS^T Q
-    Shapes as in ``attention_forward`` (Nq == Nk when causal).  With grouped
+    Shapes as in ``attention_forward`` (causal with Nq != Nk: bottom-right
+    aligned, rows that see no key get zero gradient).  With grouped
     K/V heads the gradient of a shared head is the sum over its group of
     query heads.  Returns (dq, dk, dv, D) with D = the row term above,
     float64.

@@ -80,6 +80,27 @@ def test_host_validation_rejects_bad_arguments(fa_mod):
     assert lib.fa_decode(P, P, P, P + 2, P, None, 1, 1, 1024, 128, 1.0, P, 1 << 20, None) == INVALID
     assert lib.fa_decode(P, P, P, P, P, None, 1, 1, 1024, 80, 1.0, P, 1 << 20, None) == UNSUPPORTED
     assert lib.fa_decode(P, P, None, P, P, None, 1, 1, 1024, 128, 1.0, P, 1 << 20, None) == INVALID
+    # separate query / key lengths
+    ext = lib.fa_fwd_ext
+    assert ext(P, P, P, P, None, 1, 2, 3, 8, 8, 64, 0, 1.0, None) == INVALID    # 3 does not divide 2
+    assert ext(P, P, P, P, None, 1, 2, 1, -1, 8, 64, 0, 1.0, None) == INVALID   # Nq < 0
+    assert ext(P, P, P, P, None, 1, 2, 1, 8, -1, 64, 0, 1.0, None) == INVALID   # Nk < 0
+    assert ext(P, None, P, P, None, 1, 2, 1, 8, 8, 64, 0, 1.0, None) == INVALID  # k null, Nk > 0
+    assert ext(P, P, P, P, None, 1, 1, 1, (1 << 30) + 1, 1 << 30, 64, 0, 1.0, None) == INVALID
+    bext = lib.fa_bwd_ext
+    assert bext(*args, None, 0, 1, 1, 1, 8, 5, 64, 1, 1.0, None) == WORKSPACE
+    assert bext(P, P, P, P, P, P, P, None, P, P, 1 << 20, 1, 1, 1, 8, 5, 64, 1, 1.0,
+                None) == INVALID                                                # dk null
+    # paged decode: page size must be a power of two, table needed
+    dp = lib.fa_decode_paged
+    assert dp(P, P, P, P, P, P, None, 2, 4, 2, 24, 8, 16, 128, 1.0, P, 1 << 20, None) == INVALID
+    assert dp(P, P, P, P, P, P, None, 2, 4, 2, 0, 8, 16, 128, 1.0, P, 1 << 20, None) == INVALID
+    assert dp(P, P, P, None, P, P, None, 2, 4, 2, 16, 8, 16, 128, 1.0, P, 1 << 20, None) == INVALID
+    assert dp(P, P, P, P, P, P, None, 2, 4, 3, 16, 8, 16, 128, 1.0, P, 1 << 20, None) == INVALID
+    assert dp(P, P, P, P, P, P, None, 2, 4, 2, 16, 8, 16, 96, 1.0, P, 1 << 20, None) == UNSUPPORTED
+    assert dp(P, P, P, P, P, P, None, 2, 4, 2, 16, 8, 16, 128, 1.0, None, 0, None) == WORKSPACE
+    assert dp(P, P, P, P, P, P, None, 2, 4, 2, 1 << 16, 1 << 15, 16, 128, 1.0, P, 1 << 20,
+              None) == INVALID                                                  # Lmax > INT_MAX
 
 
 def test_binding_fails_loudly_without_cuda_tensors(fa_mod):
