@@ -27,8 +27,9 @@
 //              once dP^T is ready.  In the epilogue warpgroup 0 writes dV and
 //              warpgroup 1 writes dK.
 //   warps 8-11 dQ warpgroup: thread t owns query row t of the dQ tile.
-//   warp 12    TMA producer: K_j, V_j once; Q_i, dO_i, LSE_i, D_i through a
-//              two-stage ring.
+//   warp 12    TMA producer: K_j, V_j once; Q_i with LSE_i and dO_i with D_i
+//              through a two-stage ring whose Q and dO halves are filled and
+//              released separately.
 //   warp 13    tensor-memory allocator and MMA issuer, in the order
 //                S^T(i) dP^T(i) | dV(i) | dK(i) dQ(i) | S^T(i+1) ...
 //              where "|" waits for the P^T phase, the dS^T phase, and (before
@@ -39,6 +40,8 @@
 // scores it has already read; dQ_i lands in [128, 128+d) afterwards.
 // dQ_i leaves tensor memory into the Q_i / dO_i stage it was computed from
 // (free once dQ_i is complete), so the dS buffer is never shared with it.
+// The reduction of the half staged over Q_i is committed first: Q_{i+2} is
+// needed by the next S^T before dO_{i+2} is needed by the next dP^T.
 #include <cstdlib>
 #include <cstring>
 
@@ -68,9 +71,9 @@ struct Smem {
   static constexpr int LSE_OFF = DS_OFF + DS_BYTES;    // 2 stages x 128 fp32
   static constexpr int DD_OFF = LSE_OFF + 2 * 512;     // 2 stages x 128 fp32
   static constexpr int BAR_OFF = DD_OFF + 2 * 512;
-  // kv_full, qd_full[2], qd_empty[2], st_full, dpt_full, ds_full, dq_full,
-  // dq_free, dkv_final, mma_final, stg_full, p_full
-  static constexpr int NBAR = 14;
+  // kv_full, q_full[2], q_empty[2], st_full, dpt_full, ds_full, dq_full,
+  // dq_free, dkv_final, mma_final, stg_full, p_full, do_full[2], do_empty[2]
+  static constexpr int NBAR = 18;
   static constexpr int MISC_OFF = BAR_OFF + NBAR * 8;
   static constexpr int BYTES = MISC_OFF + 16;
   static constexpr int ALLOC = BYTES > 118784 ? BYTES : 118784;
@@ -118,8 +121,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   }
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::BAR_OFF);
   uint64_t* kv_full = bars + 0;
-  uint64_t* qd_full = bars + 1;   // [2]
-  uint64_t* qd_empty = bars + 3;  // [2]
+  uint64_t* q_full = bars + 1;    // [2] Q_i and LSE_i loaded
+  uint64_t* q_empty = bars + 3;   // [2] Q_i stage released
+  uint64_t* do_full = bars + 14;  // [2] dO_i and D_i loaded
+  uint64_t* do_empty = bars + 16; // [2] dO_i stage released
   uint64_t* st_full = bars + 5;
   uint64_t* dpt_full = bars + 6;
   uint64_t* ds_full = bars + 7;    // dS^T (TMEM) and dS (shared) written
@@ -181,7 +186,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     if (lane == 0) {
       tma_prefetch_desc(&tm_q);
       tma_prefetch_desc(&tm_do);
-      int last[2] = {-1, -1};
+      int last_q[2] = {-1, -1}, last_do[2] = {-1, -1};
       mbar_arrive_expect_tx(kv_full, 2 * L::TILE);
       for (int pn = 0; pn < L::NPANEL; ++pn) {
         tma_load_3d(smem + L::K_OFF + pn * PANEL_BYTES, &tm_k, kv_full, pn * 64, key0, bkv);
@@ -192,21 +197,26 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         const int r = it >> 1;
         const int q0 = it_q0(it);
         const int bh = it_head(it);
-        if (it >= 2 && !mbar_wait(&qd_empty[st], (r - 1) & 1, abort_flag)) break;
-        mbar_arrive_expect_tx(&qd_full[st], 2 * L::TILE + 1024);
-        for (int pn = 0; pn < L::NPANEL; ++pn) {
-          tma_load_3d(smem + L::Q_OFF + st * L::TILE + pn * PANEL_BYTES, &tm_q, &qd_full[st],
+        if (it >= 2 && !mbar_wait(&q_empty[st], (r - 1) & 1, abort_flag)) break;
+        mbar_arrive_expect_tx(&q_full[st], L::TILE + 512);
+        for (int pn = 0; pn < L::NPANEL; ++pn)
+          tma_load_3d(smem + L::Q_OFF + st * L::TILE + pn * PANEL_BYTES, &tm_q, &q_full[st],
                       pn * 64, q0, bh);
-          tma_load_3d(smem + L::DO_OFF + st * L::TILE + pn * PANEL_BYTES, &tm_do, &qd_full[st],
+        tma_load_2d(smem + L::LSE_OFF + st * 512, &tm_lse, &q_full[st], q0, bh);
+        last_q[st] = r;
+        if (it >= 2 && !mbar_wait(&do_empty[st], (r - 1) & 1, abort_flag)) break;
+        mbar_arrive_expect_tx(&do_full[st], L::TILE + 512);
+        for (int pn = 0; pn < L::NPANEL; ++pn)
+          tma_load_3d(smem + L::DO_OFF + st * L::TILE + pn * PANEL_BYTES, &tm_do, &do_full[st],
                       pn * 64, q0, bh);
-        }
-        tma_load_2d(smem + L::LSE_OFF + st * 512, &tm_lse, &qd_full[st], q0, bh);
-        tma_load_2d(smem + L::DD_OFF + st * 512, &tm_dd, &qd_full[st], q0, bh);
-        last[st] = r;
+        tma_load_2d(smem + L::DD_OFF + st * 512, &tm_dd, &do_full[st], q0, bh);
+        last_do[st] = r;
       }
       mbar_wait_drain(kv_full, 0);
-      for (int s = 0; s < 2; ++s)
-        if (last[s] >= 0) mbar_wait_drain(&qd_full[s], last[s] & 1);
+      for (int s = 0; s < 2; ++s) {
+        if (last_q[s] >= 0) mbar_wait_drain(&q_full[s], last_q[s] & 1);
+        if (last_do[s] >= 0) mbar_wait_drain(&do_full[s], last_do[s] & 1);
+      }
     }
   } else if (warp == 13) {
     // ------------------------------------------------------------ MMA issuer
@@ -235,7 +245,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       for (int it = 0; ok && it < n_it; ++it) {
         const int st = it & 1;
         const uint64_t soff = static_cast<uint64_t>((st * L::TILE) >> 4);
-        if (!mbar_wait(&qd_full[st], (it >> 1) & 1, abort_flag)) { ok = false; break; }
+        if (!mbar_wait(&q_full[st], (it >> 1) & 1, abort_flag)) { ok = false; break; }
         tc_fence_after();
         // S^T = K_j Q_i^T  (M = keys, N = queries, K = d)
 #pragma unroll
@@ -243,6 +253,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           mma_bf16_ss(tSt, kdK + koff(kk), qdK0 + soff + koff(kk), IDESC_SS, kk > 0 ? 1u : 0u);
         mma_commit(st_full);
         // dP^T = V_j dO_i^T, into columns the dQ warps must have emptied.
+        if (!mbar_wait(&do_full[st], (it >> 1) & 1, abort_flag)) { ok = false; break; }
         if (it >= 1 && !mbar_wait(dq_free, (it - 1) & 1, abort_flag)) { ok = false; break; }
         tc_fence_after();
 #pragma unroll
@@ -268,8 +279,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 #pragma unroll
         for (int kk = 0; kk < BLOCK / 16; ++kk)  // dQ_i = dS K_j (M = queries, K = keys)
           mma_bf16_ss(tdPt, dsdM + moff(kk), kdM + moff(kk), IDESC_DQ, kk > 0 ? 1u : 0u);
-        // Q_i / dO_i (stage st) are released by the dQ warps, which stage
-        // dQ_i there once it is complete.
+        // Q_i and dO_i (stage st) are released by the dQ warps, which
+        // stage dQ_i there once it is complete.
         mma_commit(dq_full);
       }
       if (ok) mma_commit(dkv_final);
@@ -414,8 +425,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     // 128-byte swizzle (boxes 0 .. d/64-1 over Q_i's panels, the rest over
     // dO_i's), and one thread adds them to the fp32 accumulator with bulk
     // tensor reductions (performed in L2).  dq_free is signalled as soon as
-    // the tensor-memory reads are done; the stage goes back to the producer
-    // (qd_empty) once the reductions have read it.
+    // the tensor-memory reads are done; each half of the stage goes back to
+    // the producer (q_empty, do_empty) once its reduction has read it.
     const int t = threadIdx.x - 2 * BLOCK;  // query row of the dQ tile, TMEM lane
     const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
     const uint32_t sw = static_cast<uint32_t>(t & 7);
@@ -455,12 +466,19 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       mbar_arrive(stg_full);
       if (t == 0) {
         if (!mbar_wait(stg_full, it & 1, abort_flag)) break;
+        // the half over Q_i first, as its own group: Q_{i+2} is needed first
 #pragma unroll
-        for (int b = 0; b < NBOX; ++b) tma_reduce_add_3d(&tm_dq, box_addr(st, b), 32 * b, q0, bh);
+        for (int b = 0; b < L::NPANEL; ++b)
+          tma_reduce_add_3d(&tm_dq, box_addr(st, b), 32 * b, q0, bh);
         bulk_commit_group();
+#pragma unroll
+        for (int b = L::NPANEL; b < NBOX; ++b)
+          tma_reduce_add_3d(&tm_dq, box_addr(st, b), 32 * b, q0, bh);
+        bulk_commit_group();
+        bulk_wait_group_read1();
+        mbar_arrive(&q_empty[st]);   // Q_i's stage may be reloaded
         bulk_wait_group_read0();
-        // Q_i / dO_i (stage st) may be reloaded
-        mbar_arrive(&qd_empty[st]);
+        mbar_arrive(&do_empty[st]);  // dO_i's stage may be reloaded
       }
     }
     if (t == 0) bulk_wait_group0();
