@@ -158,6 +158,12 @@ def fwd_flops(w):
     return f * 0.5 if w.causal else f
 
 
+def varlen_flops(w, lens):
+    """Forward FLOPs of a ragged batch: the fwd convention per sequence."""
+    f = sum(4.0 * w.H * L * L * w.d for L in lens)
+    return f * 0.5 if w.causal else f
+
+
 def decode_bytes(w, seqlens):
     """Algorithmic KV bytes: every cached key and value row read once."""
     return float(sum(int(L) for L in seqlens)) * w.kv_heads * w.d * 2 * 2
@@ -179,6 +185,17 @@ class Runner:
             self.unit, self.kind_bound = "TFLOP/s", "tensor"
             self.launches_per_step = 1
             self.kernel_key = f"fa_fwd_kernel<{w.d},{str(w.causal).lower()}>"
+            self.out_host = torch.empty(self.o.shape, dtype=torch.bfloat16).pin_memory()
+        elif w.kind == "fwd_varlen":
+            q, k, v, cu_q, cu_k = self.dbuf
+            lens = (self.host[3][1:] - self.host[3][:-1]).tolist()
+            self.max_len = max(lens)
+            self.o = torch.empty_like(q)
+            self.lse = torch.empty((q.shape[1], q.shape[0]), dtype=torch.float32, device=dev)
+            self.work = varlen_flops(w, lens)
+            self.unit, self.kind_bound = "TFLOP/s", "tensor"
+            self.launches_per_step = 1
+            self.kernel_key = f"fa_fwd_kernel<{w.d},{str(w.causal).lower()},varlen>"
             self.out_host = torch.empty(self.o.shape, dtype=torch.bfloat16).pin_memory()
         elif w.kind == "bwd":
             q, k, v, do = self.dbuf
@@ -224,6 +241,10 @@ class Runner:
         b = bufs if bufs is not None else self.dbuf
         if w.kind == "fwd":
             fa.fwd(b[0], b[1], b[2], causal=w.causal, scale=w.scale, out=self.o, lse=self.lse)
+            return self.o
+        if w.kind == "fwd_varlen":
+            fa.fwd_varlen(b[0], b[1], b[2], b[3], b[4], self.max_len, causal=w.causal,
+                          scale=w.scale, out=self.o, lse=self.lse)
             return self.o
         if w.kind == "bwd":
             fa.bwd(b[0], b[1], b[2], self.o, b[3], self.lse, causal=w.causal, scale=w.scale,
@@ -323,7 +344,35 @@ def run_reference(args, w, total_budget=150.0, emit=True):
     f64 = inputs.to_f64
     budget = total_budget / max(1, args.steps + args.warmup)  # seconds per step
     rng = np.random.default_rng(w.seed)
-    if w.kind in ("fwd", "bwd"):
+    if w.kind == "fwd_varlen":
+        q, k, v, cu_q, cu_k = host
+        lens = (cu_q[1:] - cu_q[:-1]).tolist()
+        group = w.H // w.kv_heads
+        seq_heads = [(b, h) for b in range(w.B) for h in range(w.H)]
+        L0, c0 = lens[0], int(cu_q[0])
+        t0 = time.perf_counter()
+        oracle.attention_forward_rows(f64(q[c0:c0 + L0, 0]), f64(k[c0:c0 + L0, 0]),
+                                      f64(v[c0:c0 + L0, 0]), w.causal, w.scale,
+                                      np.arange(min(64, L0)))
+        per_row = (time.perf_counter() - t0) / min(64, L0)
+        rows_per_step = int(max(1, budget / max(per_row, 1e-9)))
+        sample = (f"up to {rows_per_step} query rows of one (sequence, head) per step, "
+                  "rows drawn uniformly")
+
+        def step(i):
+            b, h = seq_heads[i % len(seq_heads)]
+            L, q0, k0 = lens[b], int(cu_q[b]), int(cu_k[b])
+            rows = np.sort(rng.integers(0, L, min(rows_per_step, L)))
+            qh = f64(q[q0:q0 + L, h])
+            kh, vh = f64(k[k0:k0 + L, h // group]), f64(v[k0:k0 + L, h // group])
+            t = time.perf_counter()
+            oracle.attention_forward_rows(qh, kh, vh, w.causal, w.scale, rows)
+            dt = time.perf_counter() - t
+            keys = (rows + 1).sum() if w.causal else rows.size * L
+            return dt, 4.0 * keys * w.d, 1.0
+        unit = "TFLOP/s"
+        scale_out = 1e12
+    elif w.kind in ("fwd", "bwd"):
         q, k, v = (t for t in host[:3])
         heads = [(b, h) for b in range(w.B) for h in range(w.H)]
         # rows per step sized from a probe so that a step stays within budget
@@ -410,7 +459,7 @@ def main():
     if args.B is not None:
         import dataclasses
         w = dataclasses.replace(w, B=args.B, name=f"{w.name}[B={args.B}]")
-    default_steps = {"fwd": 4000, "bwd": 300, "decode": 800}[w.kind]
+    default_steps = {"fwd": 4000, "bwd": 300, "decode": 800, "fwd_varlen": 1000}[w.kind]
     if w.name == "fwd_causal_B1_H32_N32768_d128":
         default_steps = 200
     if args.steps is None:

@@ -99,6 +99,31 @@ fa_status fa_fwd_ext(const void* q, const void* k, const void* v, void* o, float
                      fa_stream_t stream);
 
 /*
+ * Forward over a ragged batch: B sequences of different lengths packed
+ * without padding (each sequence is the attention problem of its own rows;
+ * "DL101 chapter 9", section 3.3 for Lq x Lk).
+ *   q            : bf16 [total_q, H, d], token-major: the rows of sequence b
+ *                  are cu_seqlens_q[b] .. cu_seqlens_q[b+1]-1; read only.
+ *   k, v         : bf16 [total_k, Hkv, d], likewise with cu_seqlens_k.
+ *   o            : bf16 [total_q, H, d], written.
+ *   lse          : float32 [H, total_q], written; may be NULL.
+ *   cu_seqlens_q,
+ *   cu_seqlens_k : int32 [B + 1] in DEVICE memory: 0, then the running sums
+ *                  of the lengths, ending at total_q / total_k.  A sequence
+ *                  whose range leaves the packed array is treated as empty.
+ *   max_seqlen_q : host upper bound of the query lengths (sizes the launch).
+ *                  A longer sequence records FA_ERR_INVALID_ARG in the device
+ *                  error word and its rows past max_seqlen_q are not written.
+ * Causal masking is bottom-right aligned per sequence (query i of a sequence
+ * keeps key j iff j <= i + Lk_b - Lq_b).  A sequence with no keys gets O = 0,
+ * LSE = -inf.  Pointers to empty arrays may be NULL.  Returns as fa_fwd.
+ */
+fa_status fa_fwd_varlen(const void* q, const void* k, const void* v, void* o, float* lse,
+                        const int* cu_seqlens_q, const int* cu_seqlens_k,
+                        int B, int H, int Hkv, int total_q, int total_k, int max_seqlen_q,
+                        int d, int causal, float scale, fa_stream_t stream);
+
+/*
  * Bytes of device workspace fa_bwd needs: D = rowsum(dO * O) and
  * log2(e) * LSE as float32 [B, H, Np] with Np = N rounded up to a multiple
  * of 128, followed by the float32 dQ accumulator [B, H, N, d], each region
@@ -155,6 +180,38 @@ fa_status fa_bwd_ext(const void* q, const void* k, const void* v, const void* o,
                      void* workspace, size_t ws_bytes,
                      int B, int H, int Hkv, int Nq, int Nk, int d, int causal, float scale,
                      fa_stream_t stream);
+
+/*
+ * Bytes of device workspace fa_bwd_varlen needs: D and log2(e) * LSE as
+ * float32 [H, P] (every sequence's rows in their own padded segment, P about
+ * total_q + 132 B), then the float32 dQ accumulator [total_q, H, d], each
+ * region 256-byte aligned.  Returns 0 for invalid sizes.
+ */
+size_t fa_bwd_varlen_workspace_size(int B, int H, int total_q, int d);
+
+/*
+ * Backward over a ragged batch (the inverse of fa_fwd_varlen; recomputation
+ * as fa_bwd):
+ *   q, o, dout   : bf16 [total_q, H, d] token-major, read only.
+ *   lse          : float32 [H, total_q] from fa_fwd_varlen, read only.
+ *   k, v         : bf16 [total_k, Hkv, d], read only.
+ *   dq           : bf16 [total_q, H, d], written.
+ *   dk, dv       : bf16 [total_k, Hkv, d], written (zero for keys that no
+ *                  query sees and for rows outside every sequence).
+ *   cu_seqlens_q,
+ *   cu_seqlens_k : int32 [B + 1] in device memory, as fa_fwd_varlen.
+ *   max_seqlen_k : host upper bound of the key lengths (sizes the launch).
+ *   workspace    : fa_bwd_varlen_workspace_size(B, H, total_q, d) bytes,
+ *                  256-byte aligned, owned by the caller.
+ * Returns FA_OK, FA_ERR_INVALID_ARG, FA_ERR_UNSUPPORTED, FA_ERR_WORKSPACE or
+ * FA_ERR_CUDA.
+ */
+fa_status fa_bwd_varlen(const void* q, const void* k, const void* v, const void* o,
+                        const void* dout, const float* lse, void* dq, void* dk, void* dv,
+                        const int* cu_seqlens_q, const int* cu_seqlens_k,
+                        void* workspace, size_t ws_bytes,
+                        int B, int H, int Hkv, int total_q, int total_k, int max_seqlen_k,
+                        int d, int causal, float scale, fa_stream_t stream);
 
 /*
  * Bytes of device workspace fa_decode needs for the split-KV partials

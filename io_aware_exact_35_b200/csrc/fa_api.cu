@@ -78,6 +78,34 @@ fa_status make_tmap_bf16_3d(CUtensorMap* map, const void* base, uint64_t d, uint
   return r == CUDA_SUCCESS ? FA_OK : FA_ERR_CUDA;
 }
 
+fa_status make_tmap_bf16_rows_heads(CUtensorMap* map, const void* base, uint64_t d,
+                                    uint64_t heads, uint64_t rows, uint32_t box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (fn == nullptr) return FA_ERR_CUDA;
+  const cuuint64_t dims[3] = {d, heads, rows};
+  const cuuint64_t strides[2] = {d * 2, heads * d * 2};  // bytes, dims 1 and 2
+  const cuuint32_t box[3] = {64u, 1u, box_rows};
+  const cuuint32_t estr[3] = {1u, 1u, 1u};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims,
+                  strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? FA_OK : FA_ERR_CUDA;
+}
+
+fa_status make_tmap_f32_rows_heads_sw128(CUtensorMap* map, const void* base, uint64_t d,
+                                         uint64_t heads, uint64_t rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (fn == nullptr) return FA_ERR_CUDA;
+  const cuuint64_t dims[3] = {d, heads, rows};
+  const cuuint64_t strides[2] = {d * 4, heads * d * 4};
+  const cuuint32_t box[3] = {32u, 1u, 128u};
+  const cuuint32_t estr[3] = {1u, 1u, 1u};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, const_cast<void*>(base), dims, strides,
+                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? FA_OK : FA_ERR_CUDA;
+}
+
 fa_status make_tmap_f32_2d(CUtensorMap* map, const void* base, uint64_t n, uint64_t outer) {
   EncodeTiledFn fn = encode_fn();
   if (fn == nullptr) return FA_ERR_CUDA;
@@ -155,6 +183,31 @@ fa_status fa_fwd_ext(const void* q, const void* k, const void* v, void* o, float
                     reinterpret_cast<cudaStream_t>(stream));
 }
 
+fa_status fa_fwd_varlen(const void* q, const void* k, const void* v, void* o, float* lse,
+                        const int* cu_seqlens_q, const int* cu_seqlens_k, int B, int H, int Hkv,
+                        int total_q, int total_k, int max_seqlen_q, int d, int causal,
+                        float scale, fa_stream_t stream) {
+  if (B < 1 || H < 1 || Hkv < 1 || H % Hkv != 0) return FA_ERR_INVALID_ARG;
+  if (total_q < 0 || total_k < 0 || max_seqlen_q < 0) return FA_ERR_INVALID_ARG;
+  if (static_cast<long long>(B) * H > INT_MAX) return FA_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
+  if (!cu_seqlens_q || !cu_seqlens_k) return FA_ERR_INVALID_ARG;
+  if (total_q > 0 && (!q || !o)) return FA_ERR_INVALID_ARG;
+  if (total_k > 0 && (!k || !v)) return FA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) ||
+      (reinterpret_cast<uintptr_t>(cu_seqlens_q) & 3u) ||
+      (reinterpret_cast<uintptr_t>(cu_seqlens_k) & 3u) ||
+      (lse != nullptr && (reinterpret_cast<uintptr_t>(lse) & 3u)))
+    return FA_ERR_INVALID_ARG;
+  if (causal != 0 && causal != 1) return FA_ERR_INVALID_ARG;
+  if (!(scale == scale)) return FA_ERR_INVALID_ARG;
+  fa_status st = check_device();
+  if (st != FA_OK) return st;
+  return launch_fwd_varlen(q, k, v, o, lse, cu_seqlens_q, cu_seqlens_k, B, H, Hkv, total_q,
+                           total_k, max_seqlen_q, d, causal, scale,
+                           reinterpret_cast<cudaStream_t>(stream));
+}
+
 size_t fa_bwd_workspace_size(int B, int H, int N, int d) {
   if (check_shape(B, H, N, d) != FA_OK) return 0;
   const size_t bh = static_cast<size_t>(B) * H;
@@ -205,6 +258,45 @@ fa_status fa_bwd_ext(const void* q, const void* k, const void* v, const void* o,
   if (Nq == 0 && Nk == 0) return FA_OK;
   return launch_bwd(q, k, v, o, dout, lse, dq, dk, dv, workspace, B, H, Hkv, Nq, Nk, d, causal,
                     scale, reinterpret_cast<cudaStream_t>(stream));
+}
+
+size_t fa_bwd_varlen_workspace_size(int B, int H, int total_q, int d) {
+  if (B < 1 || H < 1 || total_q < 0 || (d != 64 && d != 128)) return 0;
+  if (static_cast<long long>(B) * H > INT_MAX) return 0;
+  const size_t P = bwd_varlen_table_rows(B, total_q);
+  return 2 * align_up(static_cast<size_t>(H) * P * sizeof(float), 256) +
+         align_up(static_cast<size_t>(total_q) * H * d * sizeof(float), 256);
+}
+
+fa_status fa_bwd_varlen(const void* q, const void* k, const void* v, const void* o,
+                        const void* dout, const float* lse, void* dq, void* dk, void* dv,
+                        const int* cu_seqlens_q, const int* cu_seqlens_k, void* workspace,
+                        size_t ws_bytes, int B, int H, int Hkv, int total_q, int total_k,
+                        int max_seqlen_k, int d, int causal, float scale, fa_stream_t stream) {
+  if (B < 1 || H < 1 || Hkv < 1 || H % Hkv != 0) return FA_ERR_INVALID_ARG;
+  if (total_q < 0 || total_k < 0 || max_seqlen_k < 0) return FA_ERR_INVALID_ARG;
+  if (static_cast<long long>(B) * H > INT_MAX) return FA_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
+  if (!cu_seqlens_q || !cu_seqlens_k) return FA_ERR_INVALID_ARG;
+  if (total_q > 0 && (!q || !o || !dout || !lse || !dq)) return FA_ERR_INVALID_ARG;
+  if (total_k > 0 && (!k || !v || !dk || !dv)) return FA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(dout) ||
+      !aligned16(dq) || !aligned16(dk) || !aligned16(dv) ||
+      (reinterpret_cast<uintptr_t>(lse) & 3u) ||
+      (reinterpret_cast<uintptr_t>(cu_seqlens_q) & 3u) ||
+      (reinterpret_cast<uintptr_t>(cu_seqlens_k) & 3u))
+    return FA_ERR_INVALID_ARG;
+  if (causal != 0 && causal != 1) return FA_ERR_INVALID_ARG;
+  if (!(scale == scale)) return FA_ERR_INVALID_ARG;
+  const size_t need = fa_bwd_varlen_workspace_size(B, H, total_q, d);
+  if (total_q > 0 && total_k > 0 &&
+      (workspace == nullptr || ws_bytes < need || !aligned256(workspace)))
+    return FA_ERR_WORKSPACE;
+  fa_status st = check_device();
+  if (st != FA_OK) return st;
+  return launch_bwd_varlen(q, k, v, o, dout, lse, dq, dk, dv, cu_seqlens_q, cu_seqlens_k,
+                           workspace, B, H, Hkv, total_q, total_k, max_seqlen_k, d, causal, scale,
+                           reinterpret_cast<cudaStream_t>(stream));
 }
 
 size_t fa_decode_workspace_size(int B, int H, int Lmax, int d) {

@@ -83,17 +83,102 @@ struct Params {
   __nv_bfloat16* dk;
   __nv_bfloat16* dv;
   float* dqacc;
-  int Nq;            // query rows per head
-  int Nk;            // key / value rows per head
+  int Nq;            // query rows per head (padded layout)
+  int Nk;            // key / value rows per head (padded layout)
   int causal_off;    // Nk - Nq: query i sits at key position i + causal_off
-  int n_qt;          // query tiles per head, ceil(Nq / 128)
-  int n_kt;          // key tiles per head, ceil(Nk / 128)
+  int n_qt;          // query tiles per head, ceil(Nq / 128) (padded layout)
+  int n_kt;          // key tiles per head, ceil(Nk / 128), or of the longest
+                     // sequence (ragged batch)
   int group;         // query heads per key/value head (1 without grouping)
   int BHkv;          // batch x key/value heads
   int lpt_order;     // 1: key tile 0 of every head first; 0: head-major
   float scale_log2;  // scale * log2(e)
   float scale;
+  // ragged batch (token-major packing): sequence b owns rows cu_q[b] ..
+  // cu_q[b+1]-1 of q / o / dO / dQ and cu_k[b] .. of k / v / dK / dV; its
+  // rows of the LSE / D tables start at table_row0(cu_q[b], b)
+  const int* cu_q;
+  const int* cu_k;
+  int Hkv;           // key/value heads
+  int total_q, total_k;
+  // element strides of dK / dV: [head][row] at head * kv_head + row * kv_row
+  size_t kv_head, kv_row;
 };
+
+// First row of sequence b in the ragged LSE / D tables: a multiple of 4 (a
+// bulk tensor copy must start 16-byte aligned) followed by at least 127
+// padding rows before the next sequence, so a 128-row tile read from the
+// sequence's last tile stays inside its padding (+inf / 0).
+__host__ __device__ __forceinline__ long long table_row0(int cu_q_b, int b) {
+  return 4LL * ((static_cast<long long>(cu_q_b) + 3) / 4) + 132LL * b;
+}
+
+// Where a CTA's key tile lives.  Rows are counted within the sequence; q0 /
+// k0 are the sequence's first rows in the tensor maps and t0 its first row
+// of the LSE / D tables (all 0 for the padded layout).
+struct CtaGeo {
+  int kv_tile;
+  int kv_head;      // head coordinate of K / V / dK / dV
+  int q_head0;      // head coordinate of the group's first query head
+  int q0, k0, t0;
+  int Nq, Nk, off;  // lengths of the sequence and Nk - Nq
+  int n_qt;         // query tiles of the sequence
+};
+
+template <bool VARLEN>
+__device__ __forceinline__ CtaGeo cta_geo(const Params& p, int bx) {
+  CtaGeo g;
+  int bkv;
+  if (p.lpt_order) {
+    g.kv_tile = bx / p.BHkv;
+    bkv = bx - g.kv_tile * p.BHkv;
+  } else {
+    g.kv_tile = bx % p.n_kt;
+    bkv = bx / p.n_kt;
+  }
+  if constexpr (!VARLEN) {
+    g.kv_head = bkv;
+    g.q_head0 = bkv * p.group;
+    g.q0 = g.k0 = g.t0 = 0;
+    g.Nq = p.Nq;
+    g.Nk = p.Nk;
+  } else {
+    const int b = bkv / p.Hkv;
+    g.kv_head = bkv - b * p.Hkv;
+    g.q_head0 = g.kv_head * p.group;
+    g.q0 = p.cu_q[b];
+    g.k0 = p.cu_k[b];
+    g.Nq = p.cu_q[b + 1] - g.q0;
+    g.Nk = p.cu_k[b + 1] - g.k0;
+    // offsets outside the packed arrays are never used: the sequence is empty
+    if (g.q0 < 0 || g.Nq < 0 || g.q0 + g.Nq > p.total_q) g.Nq = 0;
+    if (g.k0 < 0 || g.Nk < 0 || g.k0 + g.Nk > p.total_k) g.Nk = 0;
+    g.t0 = static_cast<int>(table_row0(g.q0, b));
+  }
+  g.off = g.Nk - g.Nq;
+  g.n_qt = (g.Nq + BLOCK - 1) / BLOCK;
+  return g;
+}
+
+// Bulk tensor loads / reductions of 128 rows starting at `row` of head
+// `head`: the padded maps are [heads, rows, columns], the ragged ones
+// [rows, heads, columns].
+template <bool VARLEN>
+__device__ __forceinline__ void load_rows(void* dst, const CUtensorMap* map, uint64_t* bar, int x,
+                                          int row, int head) {
+  if constexpr (VARLEN)
+    tma_load_3d(dst, map, bar, x, head, row);
+  else
+    tma_load_3d(dst, map, bar, x, row, head);
+}
+template <bool VARLEN>
+__device__ __forceinline__ void reduce_rows(const CUtensorMap* map, const void* src, int x, int row,
+                                            int head) {
+  if constexpr (VARLEN)
+    tma_reduce_add_3d(map, src, x, head, row);
+  else
+    tma_reduce_add_3d(map, src, x, row, head);
+}
 
 __device__ __forceinline__ void tma_load_2d(void* smem_dst, const void* desc, uint64_t* bar,
                                             int c0, int c1) {
@@ -104,7 +189,7 @@ __device__ __forceinline__ void tma_load_2d(void* smem_dst, const void* desc, ui
       : "memory");
 }
 
-template <int D, bool CAUSAL>
+template <int D, bool CAUSAL, bool VARLEN>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     fa_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                   const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
@@ -147,16 +232,16 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   // Head-major order keeps one head's Q / dO tiles shared in L2 by its
   // resident CTAs; longest-first order (key tile 0, which sees every query
   // tile, of all heads first) balances few long CTAs.
-  const int bx = static_cast<int>(blockIdx.x);
-  const int kv_tile = p.lpt_order ? bx / p.BHkv : bx % p.n_kt;
-  const int bkv = p.lpt_order ? bx - kv_tile * p.BHkv : bx / p.n_kt;
-  const int key0 = kv_tile * BLOCK;
-  // causal: the first query that sees key key0 is row key0 - causal_off
-  const int i_begin = CAUSAL ? max(0, key0 - p.causal_off) / BLOCK : 0;
-  const int n_per = max(0, p.n_qt - i_begin);  // query tiles per query head
-  const int n_it = n_per * p.group;            // 0: dK = dV = 0
-  // iteration it -> (query head, first row of its query tile)
-  auto it_head = [&](int it) { return bkv * p.group + it / n_per; };
+  const CtaGeo geo = cta_geo<VARLEN>(p, static_cast<int>(blockIdx.x));
+  // ragged batch: key tiles past the end of their sequence have no work
+  if (VARLEN && geo.kv_tile * BLOCK >= geo.Nk) return;
+  const int key0 = geo.kv_tile * BLOCK;
+  // causal: the first query that sees key key0 is row key0 - off
+  const int i_begin = CAUSAL ? max(0, key0 - geo.off) / BLOCK : 0;
+  const int n_per = max(0, geo.n_qt - i_begin);  // query tiles per query head
+  const int n_it = n_per * p.group;              // 0: dK = dV = 0
+  // iteration it -> (query head, first row of its query tile in the sequence)
+  auto it_head = [&](int it) { return geo.q_head0 + it / n_per; };
   auto it_q0 = [&](int it) { return (i_begin + it % n_per) * BLOCK; };
 
   if (threadIdx.x == 0) {
@@ -189,8 +274,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       int last_q[2] = {-1, -1}, last_do[2] = {-1, -1};
       mbar_arrive_expect_tx(kv_full, 2 * L::TILE);
       for (int pn = 0; pn < L::NPANEL; ++pn) {
-        tma_load_3d(smem + L::K_OFF + pn * PANEL_BYTES, &tm_k, kv_full, pn * 64, key0, bkv);
-        tma_load_3d(smem + L::V_OFF + pn * PANEL_BYTES, &tm_v, kv_full, pn * 64, key0, bkv);
+        load_rows<VARLEN>(smem + L::K_OFF + pn * PANEL_BYTES, &tm_k, kv_full, pn * 64,
+                          geo.k0 + key0, geo.kv_head);
+        load_rows<VARLEN>(smem + L::V_OFF + pn * PANEL_BYTES, &tm_v, kv_full, pn * 64,
+                          geo.k0 + key0, geo.kv_head);
       }
       for (int it = 0; it < n_it; ++it) {
         const int st = it & 1;
@@ -200,16 +287,16 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         if (it >= 2 && !mbar_wait(&q_empty[st], (r - 1) & 1, abort_flag)) break;
         mbar_arrive_expect_tx(&q_full[st], L::TILE + 512);
         for (int pn = 0; pn < L::NPANEL; ++pn)
-          tma_load_3d(smem + L::Q_OFF + st * L::TILE + pn * PANEL_BYTES, &tm_q, &q_full[st],
-                      pn * 64, q0, bh);
-        tma_load_2d(smem + L::LSE_OFF + st * 512, &tm_lse, &q_full[st], q0, bh);
+          load_rows<VARLEN>(smem + L::Q_OFF + st * L::TILE + pn * PANEL_BYTES, &tm_q,
+                            &q_full[st], pn * 64, geo.q0 + q0, bh);
+        tma_load_2d(smem + L::LSE_OFF + st * 512, &tm_lse, &q_full[st], geo.t0 + q0, bh);
         last_q[st] = r;
         if (it >= 2 && !mbar_wait(&do_empty[st], (r - 1) & 1, abort_flag)) break;
         mbar_arrive_expect_tx(&do_full[st], L::TILE + 512);
         for (int pn = 0; pn < L::NPANEL; ++pn)
-          tma_load_3d(smem + L::DO_OFF + st * L::TILE + pn * PANEL_BYTES, &tm_do, &do_full[st],
-                      pn * 64, q0, bh);
-        tma_load_2d(smem + L::DD_OFF + st * 512, &tm_dd, &do_full[st], q0, bh);
+          load_rows<VARLEN>(smem + L::DO_OFF + st * L::TILE + pn * PANEL_BYTES, &tm_do,
+                            &do_full[st], pn * 64, geo.q0 + q0, bh);
+        tma_load_2d(smem + L::DD_OFF + st * 512, &tm_dd, &do_full[st], geo.t0 + q0, bh);
         last_do[st] = r;
       }
       mbar_wait_drain(kv_full, 0);
@@ -293,7 +380,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     const int g = warp >> 2;
     const int t = threadIdx.x - g * BLOCK;  // key row, TMEM lane
     const int key_g = key0 + t;
-    const bool key_ok = key_g < p.Nk;
+    const bool key_ok = key_g < geo.Nk;
     const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
     const float sl2 = p.scale_log2;
     uint8_t* ds_row = smem + L::DS_OFF + g * PANEL_BYTES + t * 128;  // row t of panel g
@@ -309,7 +396,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       // Causal: key row t is kept for query q of the tile iff
       // key0 + t <= q0 + q + causal_off, i.e. q >= t + delta; tiles with
       // delta <= -(BLOCK - 1) keep everything.
-      const int delta = key0 - q0 - p.causal_off;
+      const int delta = key0 - q0 - geo.off;
       const bool diag = CAUSAL && (delta > -(BLOCK - 1));
       // Phase 1: P^T = exp2(scale log2(e) S^T - log2(e) LSE) as bf16 pairs,
       // over the score columns already read; kept in registers for phase 2.
@@ -387,7 +474,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     // accumulators: it stores zeros.
     if (ok && mbar_wait_warp(dkv_final, 0, abort_flag)) {
       tc_fence_after();
-      const size_t rowoff = (static_cast<size_t>(bkv) * p.Nk + key_g) * D;
+      const size_t rowoff = static_cast<size_t>(geo.kv_head) * p.kv_head +
+                            static_cast<size_t>(geo.k0 + key_g) * p.kv_row;
       {
         const int which = g;
         const uint32_t tacc = which == 0 ? tdV : tdK;
@@ -469,11 +557,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         // the half over Q_i first, as its own group: Q_{i+2} is needed first
 #pragma unroll
         for (int b = 0; b < L::NPANEL; ++b)
-          tma_reduce_add_3d(&tm_dq, box_addr(st, b), 32 * b, q0, bh);
+          reduce_rows<VARLEN>(&tm_dq, box_addr(st, b), 32 * b, geo.q0 + q0, bh);
         bulk_commit_group();
 #pragma unroll
         for (int b = L::NPANEL; b < NBOX; ++b)
-          tma_reduce_add_3d(&tm_dq, box_addr(st, b), 32 * b, q0, bh);
+          reduce_rows<VARLEN>(&tm_dq, box_addr(st, b), 32 * b, geo.q0 + q0, bh);
         bulk_commit_group();
         bulk_wait_group_read1();
         mbar_arrive(&q_empty[st]);   // Q_i's stage may be reloaded
@@ -538,6 +626,58 @@ __global__ void __launch_bounds__(256)
   }
 }
 
+// Ragged batch: the same tables over [H, P] with the rows of sequence b
+// starting at table_row0(cu_q[b], b); rows outside every sequence hold D = 0
+// and lse2 = +inf.  (dQacc is zeroed separately.)
+template <int D>
+__global__ void __launch_bounds__(256)
+    fa_bwd_preprocess_varlen_kernel(const __nv_bfloat16* __restrict__ o,
+                                    const __nv_bfloat16* __restrict__ dout,
+                                    const float* __restrict__ lse, float* __restrict__ dd,
+                                    float* __restrict__ lse2, const int* __restrict__ cu_q, int B,
+                                    int H, int total_q, long long P) {
+  constexpr int LPR = D / 8;     // lanes per row, 16 bytes each
+  constexpr int RPW = 32 / LPR;  // rows per warp
+  const int lane = threadIdx.x & 31;
+  const long long warp_g = (static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  const long long prow_g = warp_g * RPW + lane / LPR;  // over H * P
+  const int sub = lane % LPR;
+  const bool in = prow_g < static_cast<long long>(H) * P;
+  const int h = in ? static_cast<int>(prow_g / P) : 0;
+  const long long prow = in ? prow_g - static_cast<long long>(h) * P : 0;
+  // the sequence whose segment holds prow: the last b with table_row0(b) <= prow
+  int lo = 0, hi = B - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (table_row0(cu_q[mid], mid) <= prow) lo = mid;
+    else hi = mid - 1;
+  }
+  const int b = lo;
+  const long long n = prow - table_row0(cu_q[b], b);
+  const int q0 = cu_q[b], q1 = cu_q[b + 1];
+  const bool real = in && q0 >= 0 && q1 >= q0 && q1 <= total_q && n >= 0 && n < q1 - q0;
+  const long long tok = q0 + n;
+  float acc = 0.f;
+  if (real) {
+    const size_t off = (static_cast<size_t>(tok) * H + h) * D + sub * 8;
+    const uint4 a = *reinterpret_cast<const uint4*>(o + off);
+    const uint4 c = *reinterpret_cast<const uint4*>(dout + off);
+    const uint32_t wa[4] = {a.x, a.y, a.z, a.w}, wc[4] = {c.x, c.y, c.z, c.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      acc = fmaf(__uint_as_float(wa[i] << 16), __uint_as_float(wc[i] << 16), acc);
+      acc = fmaf(__uint_as_float(wa[i] & 0xFFFF0000u), __uint_as_float(wc[i] & 0xFFFF0000u), acc);
+    }
+  }
+#pragma unroll
+  for (int off = LPR / 2; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+  if (in && sub == 0) {
+    const float l = real ? lse[static_cast<size_t>(h) * total_q + tok] : INFINITY;
+    dd[prow_g] = real ? acc : 0.f;
+    lse2[prow_g] = (l == -INFINITY) ? INFINITY : l * LOG2E;
+  }
+}
+
 // dQ = scale * dQacc in bf16, 8 elements per thread.
 __global__ void __launch_bounds__(256)
     fa_bwd_dq_convert_kernel(const float* __restrict__ dqacc, __nv_bfloat16* __restrict__ dq,
@@ -551,9 +691,9 @@ __global__ void __launch_bounds__(256)
                  pack_bf16x2(b.x * scale, b.y * scale), pack_bf16x2(b.z * scale, b.w * scale));
 }
 
-template <int D, bool CAUSAL>
+template <int D, bool CAUSAL, bool VARLEN>
 fa_status launch_main(const CUtensorMap* maps, const Params& prm, int BH, cudaStream_t stream) {
-  auto kern = fa_bwd_kernel<D, CAUSAL>;
+  auto kern = fa_bwd_kernel<D, CAUSAL, VARLEN>;
   static bool configured = false;
   if (!configured) {
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Smem<D>::ALLOC) !=
@@ -648,16 +788,120 @@ fa_status launch_bwd(const void* q, const void* k, const void* v, const void* o,
   }
   prm.scale_log2 = scale * bwd::LOG2E;
   prm.scale = scale;
+  prm.cu_q = nullptr;
+  prm.cu_k = nullptr;
+  prm.Hkv = Hkv;
+  prm.total_q = 0;
+  prm.total_k = 0;
+  prm.kv_head = static_cast<size_t>(Nk) * d;
+  prm.kv_row = static_cast<size_t>(d);
   if (d == 128)
-    st = causal ? bwd::launch_main<128, true>(maps, prm, BHkv, stream)
-                : bwd::launch_main<128, false>(maps, prm, BHkv, stream);
+    st = causal ? bwd::launch_main<128, true, false>(maps, prm, BHkv, stream)
+                : bwd::launch_main<128, false, false>(maps, prm, BHkv, stream);
   else
-    st = causal ? bwd::launch_main<64, true>(maps, prm, BHkv, stream)
-                : bwd::launch_main<64, false>(maps, prm, BHkv, stream);
+    st = causal ? bwd::launch_main<64, true, false>(maps, prm, BHkv, stream)
+                : bwd::launch_main<64, false, false>(maps, prm, BHkv, stream);
   if (st != FA_OK) return st;
   // 3. dQ = scale * accumulator
   {
     const long long n8 = rows * d / 8;
+    const long long blocks = (n8 + 255) / 256;
+    bwd::fa_bwd_dq_convert_kernel<<<static_cast<unsigned>(blocks), 256, 0, stream>>>(
+        dqacc, static_cast<__nv_bfloat16*>(dq), n8, scale);
+    if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
+  }
+  return FA_OK;
+}
+
+size_t bwd_varlen_table_rows(int B, int total_q) {
+  return static_cast<size_t>(bwd::table_row0(total_q, B));  // a multiple of 4
+}
+
+fa_status launch_bwd_varlen(const void* q, const void* k, const void* v, const void* o,
+                            const void* dout, const float* lse, void* dq, void* dk, void* dv,
+                            const int* cu_q, const int* cu_k, void* workspace, int B, int H,
+                            int Hkv, int total_q, int total_k, int max_seqlen_k, int d,
+                            int causal, float scale, cudaStream_t stream) {
+  // No queries anywhere: no gradient reaches K or V.  No keys: dQ = 0.
+  if (total_q == 0 || total_k == 0 || max_seqlen_k == 0) {
+    if (total_k > 0) {
+      const size_t kv = static_cast<size_t>(total_k) * Hkv * d * 2;
+      if (cudaMemsetAsync(dk, 0, kv, stream) != cudaSuccess ||
+          cudaMemsetAsync(dv, 0, kv, stream) != cudaSuccess)
+        return FA_ERR_CUDA;
+    }
+    if (total_q > 0 &&
+        cudaMemsetAsync(dq, 0, static_cast<size_t>(total_q) * H * d * 2, stream) != cudaSuccess)
+      return FA_ERR_CUDA;
+    return FA_OK;
+  }
+  const long long P = static_cast<long long>(bwd_varlen_table_rows(B, total_q));
+  const size_t table = align_up(static_cast<size_t>(H) * P * 4, 256);
+  float* dd = static_cast<float*>(workspace);
+  float* lse2 = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + table);
+  float* dqacc = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + 2 * table);
+  const size_t dq_elems = static_cast<size_t>(total_q) * H * d;
+  // Key rows of a sequence that no query sees get dK = dV = 0 from the main
+  // kernel; key rows outside every sequence are never written: clear all.
+  if (cudaMemsetAsync(dqacc, 0, dq_elems * 4, stream) != cudaSuccess ||
+      cudaMemsetAsync(dk, 0, static_cast<size_t>(total_k) * Hkv * d * 2, stream) != cudaSuccess ||
+      cudaMemsetAsync(dv, 0, static_cast<size_t>(total_k) * Hkv * d * 2, stream) != cudaSuccess)
+    return FA_ERR_CUDA;
+  // 1. D and log2(e) * LSE in per-sequence padded segments
+  {
+    const int rows_per_block = (256 / 32) * (32 / (d / 8));
+    const long long prows = static_cast<long long>(H) * P;
+    const long long blocks = (prows + rows_per_block - 1) / rows_per_block;
+    if (d == 128)
+      bwd::fa_bwd_preprocess_varlen_kernel<128><<<static_cast<unsigned>(blocks), 256, 0, stream>>>(
+          static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(dout), lse, dd,
+          lse2, cu_q, B, H, total_q, P);
+    else
+      bwd::fa_bwd_preprocess_varlen_kernel<64><<<static_cast<unsigned>(blocks), 256, 0, stream>>>(
+          static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(dout), lse, dd,
+          lse2, cu_q, B, H, total_q, P);
+    if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
+  }
+  // 2. dK, dV and the dQ accumulation, token-major maps
+  CUtensorMap maps[7];
+  fa_status st;
+  if ((st = make_tmap_bf16_rows_heads(&maps[0], q, d, H, total_q, bwd::BLOCK)) != FA_OK) return st;
+  if ((st = make_tmap_bf16_rows_heads(&maps[1], k, d, Hkv, total_k, bwd::BLOCK)) != FA_OK) return st;
+  if ((st = make_tmap_bf16_rows_heads(&maps[2], v, d, Hkv, total_k, bwd::BLOCK)) != FA_OK) return st;
+  if ((st = make_tmap_bf16_rows_heads(&maps[3], dout, d, H, total_q, bwd::BLOCK)) != FA_OK)
+    return st;
+  if ((st = make_tmap_f32_2d(&maps[4], lse2, P, H)) != FA_OK) return st;
+  if ((st = make_tmap_f32_2d(&maps[5], dd, P, H)) != FA_OK) return st;
+  if ((st = make_tmap_f32_rows_heads_sw128(&maps[6], dqacc, d, H, total_q)) != FA_OK) return st;
+  bwd::Params prm;
+  prm.dk = static_cast<__nv_bfloat16*>(dk);
+  prm.dv = static_cast<__nv_bfloat16*>(dv);
+  prm.dqacc = dqacc;
+  prm.Nq = prm.Nk = prm.causal_off = prm.n_qt = 0;
+  prm.n_kt = (max_seqlen_k + bwd::BLOCK - 1) / bwd::BLOCK;
+  prm.group = H / Hkv;
+  prm.BHkv = B * Hkv;
+  prm.lpt_order = 0;  // head-major: a sequence's key tiles adjacent
+  prm.scale_log2 = scale * bwd::LOG2E;
+  prm.scale = scale;
+  prm.cu_q = cu_q;
+  prm.cu_k = cu_k;
+  prm.Hkv = Hkv;
+  prm.total_q = total_q;
+  prm.total_k = total_k;
+  prm.kv_head = static_cast<size_t>(d);
+  prm.kv_row = static_cast<size_t>(Hkv) * d;
+  if (static_cast<long long>(prm.n_kt) * prm.BHkv > 0x7fffffffLL) return FA_ERR_INVALID_ARG;
+  if (d == 128)
+    st = causal ? bwd::launch_main<128, true, true>(maps, prm, prm.BHkv, stream)
+                : bwd::launch_main<128, false, true>(maps, prm, prm.BHkv, stream);
+  else
+    st = causal ? bwd::launch_main<64, true, true>(maps, prm, prm.BHkv, stream)
+                : bwd::launch_main<64, false, true>(maps, prm, prm.BHkv, stream);
+  if (st != FA_OK) return st;
+  // 3. dQ = scale * accumulator (same element order as dq)
+  {
+    const long long n8 = static_cast<long long>(dq_elems / 8);
     const long long blocks = (n8 + 255) / 256;
     bwd::fa_bwd_dq_convert_kernel<<<static_cast<unsigned>(blocks), 256, 0, stream>>>(
         dqacc, static_cast<__nv_bfloat16*>(dq), n8, scale);

@@ -82,15 +82,26 @@ struct Smem {
 struct Params {
   __nv_bfloat16* o;
   float* lse;
-  int Nq;            // query rows per head
-  int Nk;            // key / value rows per head
+  int Nq;            // query rows per head (padded layout)
+  int Nk;            // key / value rows per head (padded layout)
   int causal_off;    // Nk - Nq: query i sits at key position i + causal_off
-  int BH;
+  int BH;            // batch x query heads
   int group;         // query heads per key/value head (1 without grouping)
-  int n_cta_tiles;   // ceil(Nq / 256)
+  int n_cta_tiles;   // 256-row tiles per (batch, head): ceil(Nq / 256), or of
+                     // the longest sequence (ragged batch)
   int total_items;   // BH * n_cta_tiles
   int lpt_order;     // 1: all heads' longest tiles first; 0: head-major
   float scale_log2;  // scale * log2(e)
+  // ragged batch (token-major packing): sequence b owns rows cu_q[b] ..
+  // cu_q[b+1]-1 of q / o and cu_k[b] .. cu_k[b+1]-1 of k / v
+  const int* cu_q;
+  const int* cu_k;
+  int H;             // query heads
+  int total_q;       // packed query rows
+  int total_k;       // packed key rows
+  // element strides of O and LSE: O[head][row] at head * o_head + row * o_row,
+  // LSE at head * lse_head + row, with head = b*H + h (padded) or h (ragged)
+  size_t o_head, o_row, lse_head;
 };
 
 // Work item -> (batch*head, 256-row tile).  In LPT order the longest tiles of
@@ -108,13 +119,65 @@ __device__ __forceinline__ void item_coords(const Params& p, int item, int& bh, 
   }
 }
 
+// Where a work item lives.  Rows are counted within the sequence; q0 / k0 are
+// the sequence's first rows in the tensor maps (0 for the padded layout).
+struct ItemGeo {
+  int tile;        // 256-row query tile of the sequence
+  int head;        // head coordinate of Q / O / LSE
+  int kv_head;     // head coordinate of K / V
+  int q0, k0;
+  int Nq, Nk, off; // lengths of the sequence and Nk - Nq
+  int n_kv_total;  // key tiles of the sequence, at least 1
+};
+
+template <bool VARLEN>
+__device__ __forceinline__ ItemGeo item_geo(const Params& p, int item) {
+  ItemGeo g;
+  int bh;
+  item_coords(p, item, bh, g.tile);
+  if constexpr (!VARLEN) {
+    g.head = bh;
+    g.kv_head = bh / p.group;
+    g.q0 = 0;
+    g.k0 = 0;
+    g.Nq = p.Nq;
+    g.Nk = p.Nk;
+  } else {
+    const int b = bh / p.H;
+    const int h = bh - b * p.H;
+    g.head = h;
+    g.kv_head = h / p.group;
+    g.q0 = p.cu_q[b];
+    g.k0 = p.cu_k[b];
+    g.Nq = p.cu_q[b + 1] - g.q0;
+    g.Nk = p.cu_k[b + 1] - g.k0;
+    // offsets outside the packed arrays are never used: the sequence is empty
+    if (g.q0 < 0 || g.Nq < 0 || g.q0 + g.Nq > p.total_q) g.Nq = 0;
+    if (g.k0 < 0 || g.Nk < 0 || g.k0 + g.Nk > p.total_k) g.Nk = 0;
+  }
+  g.off = g.Nk - g.Nq;
+  g.n_kv_total = max(1, (g.Nk + BLOCK_N - 1) / BLOCK_N);
+  return g;
+}
+
+// TMA load of 128 rows x 64 columns starting at `row` of head `head`: the
+// padded maps are [heads, rows, d], the ragged ones [rows, heads, d].
+template <bool VARLEN>
+__device__ __forceinline__ void load_rows(void* dst, const CUtensorMap* map, uint64_t* bar, int x,
+                                          int row, int head) {
+  if constexpr (VARLEN)
+    tma_load_3d(dst, map, bar, x, head, row);
+  else
+    tma_load_3d(dst, map, bar, x, row, head);
+}
+
 // The k-th work item of CTA c out of G: rounds alternate direction so that a
 // CTA that drew a long item in one round draws a short one in the next.
 __device__ __forceinline__ int cta_item(int c, int k, int G) {
   return k * G + ((k & 1) ? (G - 1 - c) : c);
 }
 
-template <int D, bool CAUSAL>
+template <int D, bool CAUSAL, bool VARLEN>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q,
                   const __grid_constant__ CUtensorMap tm_k,
@@ -147,16 +210,23 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   const int lane = threadIdx.x & 31;
   const int G = static_cast<int>(gridDim.x);
   const int cta = static_cast<int>(blockIdx.x);
-  const int n_kv_total = (p.Nk + BLOCK_N - 1) / BLOCK_N;  // >= 1
-  // Key tiles seen by query tile w of 256-row tile `tile`; causal: up to the
+  // Key tiles seen by query tile w (128 rows) of an item; causal: up to the
   // tile holding the last admissible key of its last row.  At least one, so
-  // that a tile whose rows see no key at all (only when Nq > Nk) still runs
-  // the pipeline once and comes out fully masked: O = 0, LSE = -inf.
-  auto n_kv_of = [&](int tile, int w) {
-    if (!CAUSAL) return n_kv_total;
-    const int last_key = tile * BLOCK_M + w * TILE_M + TILE_M - 1 + p.causal_off;
-    return last_key < 0 ? 1 : min(last_key / BLOCK_N + 1, n_kv_total);
+  // that rows that see no key at all (Nq > Nk, or no keys) still run the
+  // pipeline once and come out fully masked: O = 0, LSE = -inf.
+  auto n_kv_of = [&](const ItemGeo& g, int w) {
+    if (!CAUSAL) return g.n_kv_total;
+    const int last_key = g.tile * BLOCK_M + w * TILE_M + TILE_M - 1 + g.off;
+    return last_key < 0 ? 1 : min(last_key / BLOCK_N + 1, g.n_kv_total);
   };
+  if constexpr (VARLEN) {
+    // one item per CTA; tiles past the end of their sequence have no work
+    const ItemGeo g = item_geo<true>(p, cta);
+    if (g.tile == 0 && g.Nq > p.n_cta_tiles * BLOCK_M) {
+      if (threadIdx.x == 0) record_error(1 /* FA_ERR_INVALID_ARG: max_seqlen_q too small */);
+    }
+    if (g.tile * BLOCK_M >= g.Nq) return;
+  }
 
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
@@ -200,16 +270,15 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       for (int k = 0; ok; ++k) {
         const int item = cta_item(cta, k, G);
         if (item >= p.total_items) break;
-        int bh, tile;
-        item_coords(p, item, bh, tile);
-        const int n_kv1 = n_kv_of(tile, 1);
+        const ItemGeo g = item_geo<VARLEN>(p, item);
+        const int n_kv1 = n_kv_of(g, 1);
         // the Q pair of the previous item must have been consumed by its S MMAs
         if (k > 0 && !mbar_wait(q_empty, (k - 1) & 1, abort_flag)) break;
         mbar_arrive_expect_tx(q_full, NQ * L::TILE);
         for (int w = 0; w < NQ; ++w)
           for (int pn = 0; pn < L::NPANEL; ++pn)
-            tma_load_3d(smem + L::Q_OFF + w * L::TILE + pn * PANEL_BYTES, &tm_q, q_full,
-                        pn * 64, tile * BLOCK_M + w * TILE_M, bh);
+            load_rows<VARLEN>(smem + L::Q_OFF + w * L::TILE + pn * PANEL_BYTES, &tm_q, q_full,
+                              pn * 64, g.q0 + g.tile * BLOCK_M + w * TILE_M, g.head);
         ++n_items;
         for (int j = 0; j < n_kv1 && ok; ++j, ++kv) {
           // K_kv is ring tile 2 kv, V_kv is ring tile 2 kv + 1
@@ -222,9 +291,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             }
             mbar_arrive_expect_tx(&full[slot], L::TILE);
             for (int pn = 0; pn < L::NPANEL; ++pn)
-              tma_load_3d(smem + L::RING_OFF + slot * L::TILE + pn * PANEL_BYTES,
-                          half ? &tm_v : &tm_k, &full[slot], pn * 64, j * BLOCK_N,
-                          bh / p.group);
+              load_rows<VARLEN>(smem + L::RING_OFF + slot * L::TILE + pn * PANEL_BYTES,
+                                half ? &tm_v : &tm_k, &full[slot], pn * 64,
+                                g.k0 + j * BLOCK_N, g.kv_head);
             ++loaded;
           }
         }
@@ -292,10 +361,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       for (int k = 0; ok; ++k) {
         const int item = cta_item(cta, k, G);
         if (item >= p.total_items) break;
-        int bh, tile;
-        item_coords(p, item, bh, tile);
-        const int n0 = n_kv_of(tile, 0);
-        const int n1 = n_kv_of(tile, 1);
+        const ItemGeo g = item_geo<VARLEN>(p, item);
+        const int n0 = n_kv_of(g, 0);
+        const int n1 = n_kv_of(g, 1);
         if (!mbar_wait(q_full, k & 1, abort_flag) || !kwait(kv)) { ok = false; break; }
         tc_fence_after();
         issue_s(0, kslot(kv));
@@ -346,11 +414,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     for (int k = 0; ok; ++k) {
       const int item = cta_item(cta, k, G);
       if (item >= p.total_items) break;
-      int bh, tile;
-      item_coords(p, item, bh, tile);
-      const int q_row0 = tile * BLOCK_M + w * TILE_M;
+      const ItemGeo g = item_geo<VARLEN>(p, item);
+      const int q_row0 = g.tile * BLOCK_M + w * TILE_M;  // within the sequence
       const int row_g = q_row0 + row;
-      const int n_kv = n_kv_of(tile, w);
+      const int n_kv = n_kv_of(g, w);
       float m = -INFINITY;  // running max of scale * log2(e) * s
       float l = 0.f;
       for (int j = 0; j < n_kv; ++j) {
@@ -367,13 +434,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         tmem_ld32(tS + 96, *reinterpret_cast<uint32_t(*)[32]>(&sr[96]));
         tmem_ld_wait();
         const int key0 = j * BLOCK_N;
-        const bool need_mask = (key0 + BLOCK_N > p.Nk) ||
-                               (CAUSAL && key0 + BLOCK_N - 1 > q_row0 + p.causal_off);
+        const bool need_mask = (key0 + BLOCK_N > g.Nk) ||
+                               (CAUSAL && key0 + BLOCK_N - 1 > q_row0 + g.off);
         // four independent max chains (latency, not throughput, bounds this loop)
         float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
         if (need_mask) {
           // last admissible key (below 0: none, the row stays at -inf)
-          const int lim = CAUSAL ? min(p.Nk - 1, row_g + p.causal_off) : p.Nk - 1;
+          const int lim = CAUSAL ? min(g.Nk - 1, row_g + g.off) : g.Nk - 1;
 #pragma unroll
           for (int c = 0; c < 128; ++c) {
             const float s = (key0 + c <= lim) ? __uint_as_float(sr[c]) : -INFINITY;
@@ -448,8 +515,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       }
       tc_fence_after();
       const float inv_l = (l > 0.f) ? 1.f / l : 0.f;
-      const bool valid = row_g < p.Nq;
-      __nv_bfloat16* orow_g = p.o + (static_cast<size_t>(bh) * p.Nq + row_g) * D;
+      const bool valid = row_g < g.Nq;
+      __nv_bfloat16* orow_g = p.o + static_cast<size_t>(g.head) * p.o_head +
+                              static_cast<size_t>(g.q0 + row_g) * p.o_row;
 #pragma unroll
       for (int c = 0; c < D; c += 32) {
         uint32_t orow[32];
@@ -473,7 +541,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       if (valid && p.lse != nullptr) {
         // LSE = ln(sum exp(scale * s)) = (m + log2 l) * ln 2, m in log2 units.
         const float lse = (l > 0.f) ? (m + lg2_approx(l)) * 0.6931471805599453f : -INFINITY;
-        p.lse[static_cast<size_t>(bh) * p.Nq + row_g] = lse;
+        p.lse[static_cast<size_t>(g.head) * p.lse_head + g.q0 + row_g] = lse;
       }
       pv_base += n_kv;
     }
@@ -490,10 +558,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   }
 }
 
-template <int D, bool CAUSAL>
+template <int D, bool CAUSAL, bool VARLEN>
 fa_status launch(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                  const Params& prm, int grid_size, cudaStream_t stream) {
-  auto kern = fa_fwd_kernel<D, CAUSAL>;
+  auto kern = fa_fwd_kernel<D, CAUSAL, VARLEN>;
   static bool configured = false;  // per process; the attribute is per function
   if (!configured) {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -583,11 +651,70 @@ fa_status launch_fwd(const void* q, const void* k, const void* v, void* o, float
   prm.total_items = static_cast<int>(items);
   prm.lpt_order = persistent ? 1 : 0;
   prm.scale_log2 = scale * 1.4426950408889634f;
+  prm.cu_q = nullptr;
+  prm.cu_k = nullptr;
+  prm.H = H;
+  prm.total_q = 0;
+  prm.total_k = 0;
+  prm.o_head = static_cast<size_t>(Nq) * d;
+  prm.o_row = static_cast<size_t>(d);
+  prm.lse_head = static_cast<size_t>(Nq);
   if (d == 128)
-    return causal ? fwd::launch<128, true>(tq, tk, tv, prm, grid, stream)
-                  : fwd::launch<128, false>(tq, tk, tv, prm, grid, stream);
-  return causal ? fwd::launch<64, true>(tq, tk, tv, prm, grid, stream)
-                : fwd::launch<64, false>(tq, tk, tv, prm, grid, stream);
+    return causal ? fwd::launch<128, true, false>(tq, tk, tv, prm, grid, stream)
+                  : fwd::launch<128, false, false>(tq, tk, tv, prm, grid, stream);
+  return causal ? fwd::launch<64, true, false>(tq, tk, tv, prm, grid, stream)
+                : fwd::launch<64, false, false>(tq, tk, tv, prm, grid, stream);
+}
+
+fa_status launch_fwd_varlen(const void* q, const void* k, const void* v, void* o, float* lse,
+                            const int* cu_q, const int* cu_k, int B, int H, int Hkv,
+                            int total_q, int total_k, int max_seqlen_q, int d, int causal,
+                            float scale, cudaStream_t stream) {
+  if (total_q == 0 || max_seqlen_q == 0) return FA_OK;
+  const long long n_cta_tiles = (static_cast<long long>(max_seqlen_q) + fwd::BLOCK_M - 1) /
+                                fwd::BLOCK_M;
+  const long long items = static_cast<long long>(B) * H * n_cta_tiles;
+  if (items > 0x7fffffffLL) return FA_ERR_INVALID_ARG;
+  // token-major maps: [rows, heads, d]; a key map over zero rows still needs
+  // one row of extent, and its loads are all masked
+  CUtensorMap tq, tk, tv;
+  fa_status st;
+  if ((st = make_tmap_bf16_rows_heads(&tq, q, d, H, total_q, fwd::TILE_M)) != FA_OK) return st;
+  const uint64_t krows = total_k > 0 ? static_cast<uint64_t>(total_k) : 1;
+  const void* kb = total_k > 0 ? k : q;  // any valid address; never read unmasked
+  const void* vb = total_k > 0 ? v : q;
+  if ((st = make_tmap_bf16_rows_heads(&tk, kb, d, total_k > 0 ? Hkv : H, krows, fwd::BLOCK_N)) !=
+      FA_OK)
+    return st;
+  if ((st = make_tmap_bf16_rows_heads(&tv, vb, d, total_k > 0 ? Hkv : H, krows, fwd::BLOCK_N)) !=
+      FA_OK)
+    return st;
+  fwd::Params prm;
+  prm.o = static_cast<__nv_bfloat16*>(o);
+  prm.lse = lse;
+  prm.Nq = 0;
+  prm.Nk = 0;
+  prm.causal_off = 0;
+  prm.BH = B * H;
+  prm.group = H / Hkv;
+  prm.n_cta_tiles = static_cast<int>(n_cta_tiles);
+  prm.total_items = static_cast<int>(items);
+  prm.lpt_order = 0;  // one CTA per tile, a head's tiles adjacent, longest first
+  prm.scale_log2 = scale * 1.4426950408889634f;
+  prm.cu_q = cu_q;
+  prm.cu_k = cu_k;
+  prm.H = H;
+  prm.total_q = total_q;
+  prm.total_k = total_k;
+  prm.o_head = static_cast<size_t>(d);
+  prm.o_row = static_cast<size_t>(H) * d;
+  prm.lse_head = static_cast<size_t>(total_q);
+  const int grid = static_cast<int>(items);
+  if (d == 128)
+    return causal ? fwd::launch<128, true, true>(tq, tk, tv, prm, grid, stream)
+                  : fwd::launch<128, false, true>(tq, tk, tv, prm, grid, stream);
+  return causal ? fwd::launch<64, true, true>(tq, tk, tv, prm, grid, stream)
+                : fwd::launch<64, false, true>(tq, tk, tv, prm, grid, stream);
 }
 
 }  // namespace fa

@@ -18,6 +18,12 @@ namespace fa {
 fa_status make_tmap_bf16_3d(CUtensorMap* map, const void* base, uint64_t d, uint64_t rows,
                             uint64_t outer, uint32_t box_rows);
 
+// 3-D bf16 tensor map over a token-major [rows, heads, d] array (d
+// innermost) with a box of 64 x 1 x box_rows and 128-byte swizzle; the
+// coordinates are (column, head, row).  Rows beyond `rows` read as zero.
+fa_status make_tmap_bf16_rows_heads(CUtensorMap* map, const void* base, uint64_t d,
+                                    uint64_t heads, uint64_t rows, uint32_t box_rows);
+
 // 2-D float32 tensor map over a [outer, n] array with a 128 x 1 box and no
 // swizzle; n * 4 must be a multiple of 16 bytes.
 fa_status make_tmap_f32_2d(CUtensorMap* map, const void* base, uint64_t n, uint64_t outer);
@@ -26,6 +32,12 @@ fa_status make_tmap_f32_2d(CUtensorMap* map, const void* base, uint64_t n, uint6
 // (128 bytes wide) and 128-byte swizzle, for bulk reductions of 128-row tiles.
 fa_status make_tmap_f32_3d_sw128(CUtensorMap* map, const void* base, uint64_t d, uint64_t rows,
                                  uint64_t outer);
+
+// 3-D float32 tensor map over a token-major [rows, heads, d] array with a
+// 32 x 1 x 128 box (128 bytes wide) and 128-byte swizzle, for bulk
+// reductions of 128-row tiles; coordinates (column, head, row).
+fa_status make_tmap_f32_rows_heads_sw128(CUtensorMap* map, const void* base, uint64_t d,
+                                         uint64_t heads, uint64_t rows);
 
 // Row stride (elements) of the per-row float32 tables of the backward
 // workspace: N rounded up to whole 128-row tiles.
@@ -36,6 +48,24 @@ inline size_t bwd_row_pad(int N) { return (static_cast<size_t>(N) + 127) / 128 *
 fa_status launch_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B,
                      int H, int Hkv, int Nq, int Nk, int d, int causal, float scale,
                      cudaStream_t stream);
+
+// Ragged batch, token-major packing: q / o [total_q, H, d], k / v
+// [total_k, Hkv, d], lse [H, total_q]; cu_q / cu_k int32 [B + 1] on the device.
+fa_status launch_fwd_varlen(const void* q, const void* k, const void* v, void* o, float* lse,
+                            const int* cu_q, const int* cu_k, int B, int H, int Hkv,
+                            int total_q, int total_k, int max_seqlen_q, int d, int causal,
+                            float scale, cudaStream_t stream);
+
+// Ragged batch backward (layouts as launch_fwd_varlen; dq like q, dk / dv like
+// k).  The workspace holds D and log2(e) * LSE as float32 [H, P] with
+// P = bwd_varlen_table_rows(B, total_q), then the float32 dQ accumulator
+// [total_q, H, d], each region 256-byte aligned.
+size_t bwd_varlen_table_rows(int B, int total_q);
+fa_status launch_bwd_varlen(const void* q, const void* k, const void* v, const void* o,
+                            const void* dout, const float* lse, void* dq, void* dk, void* dv,
+                            const int* cu_q, const int* cu_k, void* workspace, int B, int H,
+                            int Hkv, int total_q, int total_k, int max_seqlen_k, int d,
+                            int causal, float scale, cudaStream_t stream);
 
 fa_status launch_bwd(const void* q, const void* k, const void* v, const void* o,
                      const void* dout, const float* lse, void* dq, void* dk, void* dv,

@@ -31,7 +31,12 @@ SIGNATURES = {
     "fa_fwd": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _P]),
     "fa_fwd_gqa": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _P]),
     "fa_fwd_ext": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _F, _P]),
+    "fa_fwd_varlen": (_I, [_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _F,
+                           _P]),
     "fa_bwd_workspace_size": (_S, [_I, _I, _I, _I]),
+    "fa_bwd_varlen_workspace_size": (_S, [_I, _I, _I, _I]),
+    "fa_bwd_varlen": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _S, _I, _I, _I, _I, _I,
+                           _I, _I, _I, _F, _P]),
     "fa_bwd": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _S, _I, _I, _I, _I, _I, _F, _P]),
     "fa_bwd_gqa": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _S, _I, _I, _I, _I, _I, _I, _F,
                         _P]),
@@ -137,6 +142,45 @@ def fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, causal: bool = False,
     return out, lse
 
 
+def fwd_varlen(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, cu_seqlens_q: torch.Tensor,
+               cu_seqlens_k: torch.Tensor, max_seqlen_q: int, causal: bool = False,
+               scale: Optional[float] = None, out: Optional[torch.Tensor] = None,
+               lse: Optional[torch.Tensor] = None, want_lse: bool = True, stream=None):
+    """Forward over a ragged batch packed token-major: q [total_q, H, d],
+    k, v [total_k, Hkv, d] bf16; cu_seqlens_q / cu_seqlens_k int32 [B + 1] on
+    the device; max_seqlen_q bounds the query lengths.  Returns
+    (o [total_q, H, d], lse [H, total_q])."""
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _req(t, n, torch.bfloat16, 3)
+    _req(cu_seqlens_q, "cu_seqlens_q", torch.int32, 1)
+    _req(cu_seqlens_k, "cu_seqlens_k", torch.int32, 1)
+    total_q, H, d = q.shape
+    total_k, Hkv = k.shape[0], k.shape[1]
+    if tuple(k.shape) != (total_k, Hkv, d) or v.shape != k.shape or Hkv < 1 or H % Hkv:
+        raise ValueError("k and v must be [total_k, Hkv, d] with Hkv dividing q's H")
+    B = cu_seqlens_q.shape[0] - 1
+    if B < 1 or cu_seqlens_k.shape[0] != B + 1:
+        raise ValueError("cu_seqlens_q and cu_seqlens_k must both have B + 1 entries")
+    scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
+    if out is None:
+        out = torch.empty_like(q)
+    _req(out, "out", torch.bfloat16, 3)
+    if out.shape != q.shape:
+        raise ValueError("out must match q")
+    if lse is None and want_lse:
+        lse = torch.empty((H, total_q), dtype=torch.float32, device=q.device)
+    if lse is not None:
+        _req(lse, "lse", torch.float32, 2)
+        if tuple(lse.shape) != (H, total_q):
+            raise ValueError("lse must be [H, total_q]")
+    st = lib().fa_fwd_varlen(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), _ptr(lse),
+                             cu_seqlens_q.data_ptr(), cu_seqlens_k.data_ptr(), B, H, Hkv, total_q,
+                             total_k, int(max_seqlen_q), d, int(bool(causal)), scale,
+                             _stream_ptr(stream))
+    _check("fa_fwd_varlen", st)
+    return out, lse
+
+
 def bwd_workspace_size(B: int, H: int, N: int, d: int) -> int:
     return int(lib().fa_bwd_workspace_size(B, H, N, d))
 
@@ -172,6 +216,48 @@ def bwd(q, k, v, o, do, lse, causal: bool = False, scale: Optional[float] = None
                           workspace.data_ptr(), workspace.numel() * workspace.element_size(),
                           B, H, Hkv, N, Nk, d, int(bool(causal)), scale, _stream_ptr(stream))
     _check("fa_bwd_ext", st)
+    return dq, dk, dv
+
+
+def bwd_varlen(q, k, v, o, do, lse, cu_seqlens_q, cu_seqlens_k, max_seqlen_k: int,
+               causal: bool = False, scale: Optional[float] = None, dq=None, dk=None, dv=None,
+               workspace: Optional[torch.Tensor] = None, stream=None):
+    """Backward over a ragged batch packed token-major (layouts of
+    fwd_varlen; lse [H, total_q]).  Returns (dq, dk, dv)."""
+    for t, n in ((q, "q"), (k, "k"), (v, "v"), (o, "o"), (do, "do")):
+        _req(t, n, torch.bfloat16, 3)
+    _req(lse, "lse", torch.float32, 2)
+    _req(cu_seqlens_q, "cu_seqlens_q", torch.int32, 1)
+    _req(cu_seqlens_k, "cu_seqlens_k", torch.int32, 1)
+    total_q, H, d = q.shape
+    total_k, Hkv = k.shape[0], k.shape[1]
+    if o.shape != q.shape or do.shape != q.shape:
+        raise ValueError("o and do must match q's shape")
+    if tuple(k.shape) != (total_k, Hkv, d) or v.shape != k.shape or H % Hkv:
+        raise ValueError("k and v must be [total_k, Hkv, d] with Hkv dividing q's H")
+    if tuple(lse.shape) != (H, total_q):
+        raise ValueError("lse must be [H, total_q]")
+    B = cu_seqlens_q.shape[0] - 1
+    if B < 1 or cu_seqlens_k.shape[0] != B + 1:
+        raise ValueError("cu_seqlens_q and cu_seqlens_k must both have B + 1 entries")
+    scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    for t, n in ((dq, "dq"), (dk, "dk"), (dv, "dv")):
+        _req(t, n, torch.bfloat16, 3)
+    if dq.shape != q.shape or dk.shape != k.shape or dv.shape != v.shape:
+        raise ValueError("gradient buffers must match q, k, v")
+    need = int(lib().fa_bwd_varlen_workspace_size(B, H, total_q, d))
+    if workspace is None:
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=q.device)
+    st = lib().fa_bwd_varlen(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(),
+                             do.data_ptr(), lse.data_ptr(), dq.data_ptr(), dk.data_ptr(),
+                             dv.data_ptr(), cu_seqlens_q.data_ptr(), cu_seqlens_k.data_ptr(),
+                             workspace.data_ptr(), workspace.numel() * workspace.element_size(),
+                             B, H, Hkv, total_q, total_k, int(max_seqlen_k), d,
+                             int(bool(causal)), scale, _stream_ptr(stream))
+    _check("fa_bwd_varlen", st)
     return dq, dk, dv
 
 

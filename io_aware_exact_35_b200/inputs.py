@@ -29,14 +29,14 @@ BASE_SEED = 42
 @dataclass(frozen=True)
 class Workload:
     name: str
-    kind: str            # "fwd" | "bwd" | "decode"
+    kind: str            # "fwd" | "bwd" | "decode" | "fwd_varlen"
     B: int
     H: int
     d: int
     N: int = 0           # sequence length (fwd / bwd)
     causal: bool = False
     std: float = 1.0
-    Lmin: int = 0        # decode: cache length range, inclusive
+    Lmin: int = 0        # decode / ragged batch: length range, inclusive
     Lmax: int = 0
     seed: int = BASE_SEED
     Hkv: int = 0         # key/value heads (0: same as H; fewer: grouped-query attention)
@@ -73,6 +73,9 @@ WORKLOADS = {
                  causal=True, seed=BASE_SEED + 6, Hkv=8),
         Workload("decode_gqa_B16_H32_Hkv8_d128_L4096-16384", "decode", 16, 32, 128,
                  Lmin=4096, Lmax=16384, seed=BASE_SEED + 7, Hkv=8),
+        # a ragged prefill batch: 16 sequences of U{512..4096} tokens, packed
+        Workload("fwd_varlen_causal_B16_H16_d128_L512-4096", "fwd_varlen", 16, 16, 128,
+                 causal=True, Lmin=512, Lmax=4096, seed=BASE_SEED + 9),
         # the decode workload over a paged cache (16-row pages, random page order)
         Workload("decode_paged_B16_H32_d128_L4096-16384_p16", "decode", 16, 32, 128,
                  Lmin=4096, Lmax=16384, seed=BASE_SEED + 8, page=16),
@@ -140,6 +143,26 @@ def decode_inputs(B: int, H: int, d: int, Lmin: int, Lmax: int, seed: int,
     return q, kc, vc, seqlens.to(torch.int32)
 
 
+def varlen_inputs(seqlens_q, seqlens_k, H: int, Hkv: int, d: int, seed: int,
+                  std: float = 1.0, with_do: bool = False):
+    """A ragged batch packed without padding, token-major: q [total_q, H, d],
+    k, v [total_k, Hkv, d] (and dO like q when ``with_do``) as bf16 CPU
+    tensors, plus cu_seqlens_q / cu_seqlens_k int32 [B + 1] (prefix sums of
+    the lengths, starting at 0).  Draw order: q, k, v, dO, each over the
+    packed rows."""
+    g = _gen(seed)
+    lq = [int(x) for x in seqlens_q]
+    lk = [int(x) for x in seqlens_k]
+    cu_q = torch.tensor([0] + list(np.cumsum(lq)), dtype=torch.int32)
+    cu_k = torch.tensor([0] + list(np.cumsum(lk)), dtype=torch.int32)
+    tq, tk = int(cu_q[-1]), int(cu_k[-1])
+    out = [_randn_bf16(g, (tq, H, d), std), _randn_bf16(g, (tk, Hkv, d), std),
+           _randn_bf16(g, (tk, Hkv, d), std)]
+    if with_do:
+        out.append(_randn_bf16(g, (tq, H, d), std))
+    return (*out, cu_q, cu_k)
+
+
 def page_cache(kc: torch.Tensor, vc: torch.Tensor, seqlens, page_size: int, seed: int,
                spare_pages: int = 3):
     """Scatter contiguous caches [B, Hkv, Lcap, d] into page pools
@@ -171,7 +194,16 @@ def page_cache(kc: torch.Tensor, vc: torch.Tensor, seqlens, page_size: int, seed
     return kp, vp, table
 
 
+def varlen_lengths(w: Workload) -> list:
+    """Sequence lengths of a ragged-batch workload, drawn first from its seed."""
+    g = _gen(w.seed)
+    return torch.randint(w.Lmin, w.Lmax + 1, (w.B,), generator=g).tolist()
+
+
 def workload_inputs(w: Workload):
+    if w.kind == "fwd_varlen":
+        lens = varlen_lengths(w)
+        return varlen_inputs(lens, lens, w.H, w.kv_heads, w.d, w.seed + 1, w.std)
     if w.kind == "fwd":
         return fwd_inputs(w.B, w.H, w.N, w.d, w.seed, w.std, Hkv=w.kv_heads)
     if w.kind == "bwd":

@@ -91,6 +91,22 @@ def test_host_validation_rejects_bad_arguments(fa_mod):
     assert bext(*args, None, 0, 1, 1, 1, 8, 5, 64, 1, 1.0, None) == WORKSPACE
     assert bext(P, P, P, P, P, P, P, None, P, P, 1 << 20, 1, 1, 1, 8, 5, 64, 1, 1.0,
                 None) == INVALID                                                # dk null
+    # ragged batch
+    vl = lib.fa_fwd_varlen
+    assert vl(P, P, P, P, None, None, P, 2, 4, 2, 100, 100, 64, 128, 1, 1.0, None) == INVALID  # cu_q null
+    assert vl(P, P, P, P, None, P, P, 2, 4, 3, 100, 100, 64, 128, 1, 1.0, None) == INVALID    # Hkv
+    assert vl(P, P, P, P, None, P, P, 0, 4, 2, 100, 100, 64, 128, 1, 1.0, None) == INVALID    # B < 1
+    assert vl(P, P, P, P, None, P, P, 2, 4, 2, -1, 100, 64, 128, 1, 1.0, None) == INVALID     # total_q
+    assert vl(P, P, P, P, None, P + 2, P, 2, 4, 2, 100, 100, 64, 128, 1, 1.0, None) == INVALID
+    assert vl(P, P, P, P, None, P, P, 2, 4, 2, 100, 100, 64, 80, 1, 1.0, None) == UNSUPPORTED
+    assert vl(P, None, P, P, None, P, P, 2, 4, 2, 100, 100, 64, 128, 1, 1.0, None) == INVALID  # k null
+    bvl = lib.fa_bwd_varlen
+    ten = [P] * 9 + [P, P]  # q k v o dout lse dq dk dv cu_q cu_k
+    assert bvl(*ten, None, 0, 2, 4, 2, 100, 100, 64, 128, 1, 1.0, None) == WORKSPACE
+    assert bvl(*ten[:9], None, P, P, 1 << 30, 2, 4, 2, 100, 100, 64, 128, 1, 1.0, None) == INVALID
+    assert bvl(*ten, P, 1 << 30, 2, 4, 2, 100, 100, 64, 96, 1, 1.0, None) == UNSUPPORTED
+    assert lib.fa_bwd_varlen_workspace_size(2, 4, 100, 128) > 0
+    assert lib.fa_bwd_varlen_workspace_size(0, 4, 100, 128) == 0
     # paged decode: page size must be a power of two, table needed
     dp = lib.fa_decode_paged
     assert dp(P, P, P, P, P, P, None, 2, 4, 2, 24, 8, 16, 128, 1.0, P, 1 << 20, None) == INVALID

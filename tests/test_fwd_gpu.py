@@ -111,9 +111,13 @@ sys.path.insert(0, {root!r})
 import oracle
 from io_aware_exact_35_b200 import fa, inputs
 from tests._parity import check_o, check_lse
-for (B, H, N, d, causal) in [(2, 3, 1000, 128, True), (1, 5, 777, 64, True), (3, 2, 513, 128, False),
-                             (2, 4, 2048, 128, True)]:
-    q, k, v = inputs.fwd_inputs(B, H, N, d, seed=N + d)
+# (B, H, Hkv, Nq, Nk, d, causal); with Nq > Nk many work items have halves
+# that see the same number of key tiles, with Nq < Nk none do
+for (B, H, Hkv, N, Nk, d, causal) in [(2, 3, 3, 1000, 1000, 128, True), (1, 5, 5, 777, 777, 64, True),
+                                      (3, 2, 2, 513, 513, 128, False), (2, 4, 4, 2048, 2048, 128, True),
+                                      (1, 4, 2, 3000, 1000, 128, True), (2, 2, 1, 1500, 4000, 64, True),
+                                      (1, 3, 3, 2900, 2900, 128, True)]:
+    q, k, v = inputs.fwd_inputs(B, H, N, d, seed=N + d, Hkv=Hkv, Nk=Nk)
     o, lse = fa.fwd(q.cuda(), k.cuda(), v.cuda(), causal=causal)
     torch.cuda.synchronize()
     assert fa.get_device_error() == 0
@@ -127,8 +131,9 @@ print("ok")
 @pytest.mark.parametrize("schedule", ["persistent", "grid"])
 def test_fwd_both_work_schedules(fa_mod, cuda_device, schedule):
     """The forward runs either one CTA per 256-row tile or persistently (each
-    CTA loops over several tiles, barrier phases carried across them); both
-    must give the oracle's result."""
+    CTA loops over several tiles, barrier phases carried across them, the
+    two query-tile streams running into the next tile independently); both
+    must give the oracle's result, also for unequal query / key lengths."""
     import os
     import subprocess
     import sys
