@@ -54,6 +54,8 @@ def load_peaks():
 
 KERNEL_SOURCES = {
     "fwd": ("fa_fwd.cu", "sm100.cuh"),
+    "fwd_varlen": ("fa_fwd.cu", "sm100.cuh"),
+    "fwd_fp8": ("fa_fwd.cu", "sm100.cuh"),
     "bwd": ("fa_bwd.cu", "sm100.cuh"),
     "decode": ("fa_decode.cu", "sm100.cuh"),
 }
@@ -176,6 +178,8 @@ class Runner:
         from io_aware_exact_35_b200 import fa
         self.fa, self.w, self.dev = fa, w, dev
         self.host = inputs.workload_inputs(w)
+        if w.kind == "fwd_fp8":  # e4m3 q, k, vt and their descale factors
+            self.host, self.fp8_scales = list(self.host[:3]), self.host[3]
         self.dbuf = [t.to(dev) for t in self.host]
         if w.kind == "fwd":
             q, k, v = self.dbuf
@@ -185,6 +189,15 @@ class Runner:
             self.unit, self.kind_bound = "TFLOP/s", "tensor"
             self.launches_per_step = 1
             self.kernel_key = f"fa_fwd_kernel<{w.d},{str(w.causal).lower()}>"
+            self.out_host = torch.empty(self.o.shape, dtype=torch.bfloat16).pin_memory()
+        elif w.kind == "fwd_fp8":
+            q8 = self.host[0]
+            self.o = torch.empty(q8.shape, dtype=torch.bfloat16, device=dev)
+            self.lse = torch.empty(q8.shape[:3], dtype=torch.float32, device=dev)
+            self.work = fwd_flops(w)
+            self.unit, self.kind_bound = "TFLOP/s", "tensor_fp8"
+            self.launches_per_step = 1
+            self.kernel_key = f"fa_fwd_kernel<{w.d},{str(w.causal).lower()},e4m3>"
             self.out_host = torch.empty(self.o.shape, dtype=torch.bfloat16).pin_memory()
         elif w.kind == "fwd_varlen":
             q, k, v, cu_q, cu_k = self.dbuf
@@ -241,6 +254,11 @@ class Runner:
         b = bufs if bufs is not None else self.dbuf
         if w.kind == "fwd":
             fa.fwd(b[0], b[1], b[2], causal=w.causal, scale=w.scale, out=self.o, lse=self.lse)
+            return self.o
+        if w.kind == "fwd_fp8":
+            qs, ks, vs = self.fp8_scales
+            fa.fwd_fp8(b[0], b[1], b[2], qs, ks, vs, causal=w.causal, scale=w.scale, out=self.o,
+                       lse=self.lse)
             return self.o
         if w.kind == "fwd_varlen":
             fa.fwd_varlen(b[0], b[1], b[2], b[3], b[4], self.max_len, causal=w.causal,
@@ -372,8 +390,14 @@ def run_reference(args, w, total_budget=150.0, emit=True):
             return dt, 4.0 * keys * w.d, 1.0
         unit = "TFLOP/s"
         scale_out = 1e12
-    elif w.kind in ("fwd", "bwd"):
-        q, k, v = (t for t in host[:3])
+    elif w.kind in ("fwd", "bwd", "fwd_fp8"):
+        if w.kind == "fwd_fp8":  # the oracle takes the real (descaled) values
+            q8, k8, vt8, (qs, ks, vs) = host
+            q = torch.from_numpy(inputs.fp8_to_f64(q8, qs))
+            k = torch.from_numpy(inputs.fp8_to_f64(k8, ks))
+            v = torch.from_numpy(inputs.fp8_to_f64(vt8.transpose(-1, -2).contiguous(), vs))
+        else:
+            q, k, v = (t for t in host[:3])
         heads = [(b, h) for b in range(w.B) for h in range(w.H)]
         # rows per step sized from a probe so that a step stays within budget
         b0, h0 = heads[0]
@@ -459,7 +483,8 @@ def main():
     if args.B is not None:
         import dataclasses
         w = dataclasses.replace(w, B=args.B, name=f"{w.name}[B={args.B}]")
-    default_steps = {"fwd": 4000, "bwd": 300, "decode": 800, "fwd_varlen": 1000}[w.kind]
+    default_steps = {"fwd": 4000, "bwd": 300, "decode": 800, "fwd_varlen": 1000,
+                     "fwd_fp8": 4000}[w.kind]
     if w.name == "fwd_causal_B1_H32_N32768_d128":
         default_steps = 200
     if args.steps is None:
@@ -499,6 +524,15 @@ def main():
         roof = {"bound": "tensor", "achieved": ach, "peak": peak, "unit": "TFLOP/s",
                 "frac": ach / peak, "traffic": traffic,
                 "peak_source": f"{peak_src} bf16_tflops (burst)"}
+    elif r.kind_bound == "tensor_fp8":
+        # the 8-bit contraction's peak: the measured bf16 peak x the nominal
+        # fp8 / bf16 ratio (4.5 / 2.25 PFLOP/s dense)
+        peak = 2.0 * float(peaks["bf16_tflops"])
+        ach = r.work / mean_s / 1e12
+        traffic = profiled_traffic(r.kernel_key, r.w.kind)
+        roof = {"bound": "tensor", "achieved": ach, "peak": peak, "unit": "TFLOP/s",
+                "frac": ach / peak, "traffic": traffic,
+                "peak_source": f"{peak_src} bf16_tflops (burst) x 2 (nominal e4m3 / bf16)"}
     else:
         peak = float(peaks["hbm_gbs"])
         ach = r.work / mean_s / 1e9
@@ -510,7 +544,7 @@ def main():
         "metric": METRIC, "value": value, "unit": r.unit, "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": mean_s * 1e3,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-        "dtype": "bf16", "data": "synthetic",
+        "dtype": "e4m3" if w.kind == "fwd_fp8" else "bf16", "data": "synthetic",
         "config": dict(workload_config(w, f"replicas{world}" if world > 1 else "single"),
                        l2="flushed (256 MB write) before every step" if r.flush is not None
                        else "inputs larger than L2"),

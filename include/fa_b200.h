@@ -13,9 +13,15 @@
  *    "bf16" arguments are void pointers to IEEE bfloat16 bit patterns.
  *  - Q, K, V, O, dO, dQ, dK, dV are [B, H, N, d] (batch, head, sequence, head
  *    dimension; the multi-head layout of "DL101 chapter 9", section 3).
- *    LSE and D are [B, H, N] float32.
- *  - Supported head dimensions: d = 64 and d = 128.  Any N >= 0 (ragged tails
- *    are masked inside the kernels).
+ *    LSE and D are [B, H, N] float32.  The ragged-batch entry points
+ *    (_varlen) take sequences packed token-major, [total, heads, d], and the
+ *    paged decode takes page pools; each states its layout.
+ *  - Supported head dimensions: d = 64 and d = 128 (fa_fwd_fp8: 128).  Any
+ *    N >= 0 (ragged tails are masked inside the kernels).
+ *  - Key / value tensors may have fewer heads than queries (Hkv dividing H;
+ *    the _gqa, _ext, _varlen, _paged and _fp8 entry points): query head h
+ *    attends key / value head h / (H / Hkv) ("DL101 chapter 9", sections 3.1
+ *    MQA and 3.2 GQA).
  *  - scale multiplies Q K^T before the softmax; callers normally pass
  *    1/sqrt(d) ("DL101 chapter 9", section 1.1).
  *  - Causal masking keeps key j for query i iff j <= i + Nk - Nq (diagonal
@@ -122,6 +128,30 @@ fa_status fa_fwd_varlen(const void* q, const void* k, const void* v, void* o, fl
                         const int* cu_seqlens_q, const int* cu_seqlens_k,
                         int B, int H, int Hkv, int total_q, int total_k, int max_seqlen_q,
                         int d, int causal, float scale, fa_stream_t stream);
+
+/*
+ * Forward with 8-bit float inputs (e4m3, OCP FP8): the FP8 path the pages
+ * mention for FlashAttention-3 ("Flash Attention La Gi?", FlashAttention-3).
+ * The pages give no scaling convention; here each input tensor carries one
+ * descale factor (real value = stored e4m3 value x factor), the products run
+ * on the tensor core's 8-bit path with f32 accumulation, and the softmax
+ * probabilities are rounded to e4m3 before the P V product (relative error
+ * up to 2^-4 per probability, so O carries a few percent relative error).
+ *   q       : e4m3 [B, H, Nq, 128] (bytes), read only.
+ *   k       : e4m3 [B, Hkv, Nk, 128], read only.
+ *   vt      : e4m3 [B, Hkv, 128, Nk]: V transposed (row r holds component r
+ *             of every value), read only.  Nk must be a multiple of 16.
+ *   q_scale, k_scale, v_scale : the descale factors.
+ *   o       : bf16 [B, H, Nq, 128], written (real, descaled values).
+ *   lse     : float32 [B, H, Nq], written; may be NULL.
+ *   d       : must be 128.
+ * Masking, grouping, scale and errors as fa_fwd_ext; FA_ERR_UNSUPPORTED for
+ * d != 128 or Nk not a multiple of 16.
+ */
+fa_status fa_fwd_fp8(const void* q, const void* k, const void* vt, void* o, float* lse,
+                     float q_scale, float k_scale, float v_scale,
+                     int B, int H, int Hkv, int Nq, int Nk, int d, int causal, float scale,
+                     fa_stream_t stream);
 
 /*
  * Bytes of device workspace fa_bwd needs: D = rowsum(dO * O) and

@@ -106,6 +106,20 @@ fa_status make_tmap_f32_rows_heads_sw128(CUtensorMap* map, const void* base, uin
   return r == CUDA_SUCCESS ? FA_OK : FA_ERR_CUDA;
 }
 
+fa_status make_tmap_u8_3d(CUtensorMap* map, const void* base, uint64_t inner, uint64_t rows,
+                          uint64_t outer, uint32_t box_inner, uint32_t box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (fn == nullptr) return FA_ERR_CUDA;
+  const cuuint64_t dims[3] = {inner, rows, outer};
+  const cuuint64_t strides[2] = {inner, rows * inner};  // bytes, dims 1 and 2
+  const cuuint32_t box[3] = {box_inner, box_rows, 1u};
+  const cuuint32_t estr[3] = {1u, 1u, 1u};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(base), dims, strides,
+                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? FA_OK : FA_ERR_CUDA;
+}
+
 fa_status make_tmap_f32_2d(CUtensorMap* map, const void* base, uint64_t n, uint64_t outer) {
   EncodeTiledFn fn = encode_fn();
   if (fn == nullptr) return FA_ERR_CUDA;
@@ -206,6 +220,29 @@ fa_status fa_fwd_varlen(const void* q, const void* k, const void* v, void* o, fl
   return launch_fwd_varlen(q, k, v, o, lse, cu_seqlens_q, cu_seqlens_k, B, H, Hkv, total_q,
                            total_k, max_seqlen_q, d, causal, scale,
                            reinterpret_cast<cudaStream_t>(stream));
+}
+
+fa_status fa_fwd_fp8(const void* q, const void* k, const void* vt, void* o, float* lse,
+                     float q_scale, float k_scale, float v_scale, int B, int H, int Hkv, int Nq,
+                     int Nk, int d, int causal, float scale, fa_stream_t stream) {
+  fa_status st = check_shape(B, H, Nq, d);
+  if (st != FA_OK) return st;
+  if ((st = check_shape(B, Hkv, Nk, d)) != FA_OK) return st;
+  if (d != 128) return FA_ERR_UNSUPPORTED;
+  if (Nk % 16 != 0) return FA_ERR_UNSUPPORTED;  // rows of vt must be 16-byte multiples
+  if (static_cast<long long>(Nq) + Nk > INT_MAX) return FA_ERR_INVALID_ARG;
+  if (Hkv < 1 || H % Hkv != 0) return FA_ERR_INVALID_ARG;
+  if (Nq > 0 && (!q || !o || (Nk > 0 && (!k || !vt)))) return FA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(vt) || !aligned16(o)) return FA_ERR_INVALID_ARG;
+  if (lse != nullptr && (reinterpret_cast<uintptr_t>(lse) & 3u)) return FA_ERR_INVALID_ARG;
+  if (causal != 0 && causal != 1) return FA_ERR_INVALID_ARG;
+  if (!(scale == scale) || !(q_scale == q_scale) || !(k_scale == k_scale) ||
+      !(v_scale == v_scale))
+    return FA_ERR_INVALID_ARG;
+  if ((st = check_device()) != FA_OK) return st;
+  if (Nq == 0) return FA_OK;
+  return launch_fwd_fp8(q, k, vt, o, lse, q_scale, k_scale, v_scale, B, H, Hkv, Nq, Nk, causal,
+                        scale, reinterpret_cast<cudaStream_t>(stream));
 }
 
 size_t fa_bwd_workspace_size(int B, int H, int N, int d) {

@@ -46,6 +46,40 @@
 
 namespace fa {
 
+// ---- 8-bit float (e4m3) helpers of the FP8 forward
+// D (f32, tensor memory) (+)= A B^T with 8-bit float operands, both from
+// shared memory (kind::f8f6f4: K = 32 per instruction, 32 bytes per row).
+__device__ __forceinline__ void mma_f8_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                          uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// Instruction descriptor for kind::f8f6f4: f32 accumulator, A and B e4m3
+// (format code 0), both K-major, M x N.
+__host__ __device__ constexpr uint32_t idesc_e4m3_f32(int M, int N) {
+  return (1u << 4)                                   // D: f32
+         | (static_cast<uint32_t>(N >> 3) << 17)      // N / 8
+         | (static_cast<uint32_t>(M >> 4) << 24);     // M / 16
+}
+
+// Four float32 values rounded to e4m3 (round to nearest even, saturating to
+// +-448), packed little-endian: x0 in the lowest byte.
+__device__ __forceinline__ uint32_t pack_e4m3x4(float x0, float x1, float x2, float x3) {
+  uint32_t r;
+  asm("{\n\t.reg .b16 lo, hi;\n\t"
+      "cvt.rn.satfinite.e4m3x2.f32 lo, %2, %1;\n\t"
+      "cvt.rn.satfinite.e4m3x2.f32 hi, %4, %3;\n\t"
+      "mov.b32 %0, {lo, hi};\n\t}"
+      : "=r"(r)
+      : "f"(x0), "f"(x1), "f"(x2), "f"(x3));
+  return r;
+}
+
 namespace fwd {
 
 constexpr int TILE_M = 128;   // rows per softmax warpgroup
@@ -61,14 +95,19 @@ constexpr float RESCALE_THRESHOLD = 8.0f;  // log2 units
 #endif
 constexpr int EMU_PAIRS = FA_FWD_EMU_PAIRS;  // of every 4 exp pairs, on the FMA pipe
 
-template <int D>
+// Shared-memory plan.  A panel is 128 rows x 128 bytes (64 bf16 or 128 e4m3
+// values per row).  With 8-bit inputs (F8) the ring carries K_j and V_j^T
+// tiles, and P_w goes through shared memory (the 8-bit product reads both
+// operands from there).
+template <int D, bool F8 = false>
 struct Smem {
-  static constexpr int NPANEL = D / 64;
-  static constexpr int TILE = NPANEL * PANEL_BYTES;  // 128 rows x D bf16
+  static constexpr int NPANEL = F8 ? D / 128 : D / 64;
+  static constexpr int TILE = NPANEL * PANEL_BYTES;  // 128 rows x D elements
   static constexpr int NSLOT = 5;                    // K/V ring slots
   static constexpr int Q_OFF = 0;                    // NQ tiles
   static constexpr int RING_OFF = NQ * TILE;
-  static constexpr int BAR_OFF = RING_OFF + NSLOT * TILE;
+  static constexpr int P_OFF = RING_OFF + NSLOT * TILE;  // F8: NQ tiles of 128 x 128 e4m3
+  static constexpr int BAR_OFF = P_OFF + (F8 ? NQ * PANEL_BYTES : 0);
   // barriers: q_full, q_empty, full[NSLOT], empty[NSLOT],
   //           s_full[NQ], p_full[NQ], o_done[NQ], o_final[NQ], o_free[NQ], mma_final
   static constexpr int NBAR = 2 + 2 * NSLOT + 5 * NQ + 1;
@@ -91,7 +130,8 @@ struct Params {
                      // the longest sequence (ragged batch)
   int total_items;   // BH * n_cta_tiles
   int lpt_order;     // 1: all heads' longest tiles first; 0: head-major
-  float scale_log2;  // scale * log2(e)
+  float scale_log2;  // scale * log2(e) (times the q and k descales for e4m3)
+  float o_scale;     // multiplies O / l: 1, or the v descale for e4m3
   // ragged batch (token-major packing): sequence b owns rows cu_q[b] ..
   // cu_q[b+1]-1 of q / o and cu_k[b] .. cu_k[b+1]-1 of k / v
   const int* cu_q;
@@ -177,12 +217,18 @@ __device__ __forceinline__ int cta_item(int c, int k, int G) {
   return k * G + ((k & 1) ? (G - 1 - c) : c);
 }
 
-template <int D, bool CAUSAL, bool VARLEN>
+// F8: q, k are e4m3 [heads, rows, d], v is given transposed, e4m3
+// [heads, d, rows], so that both products read K-major tiles; P_w is rounded
+// to e4m3 (P <= 2^8 < 448 under the stale-maximum rule) and the accumulators
+// stay f32.
+template <int D, bool CAUSAL, bool VARLEN, bool F8 = false>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q,
                   const __grid_constant__ CUtensorMap tm_k,
                   const __grid_constant__ CUtensorMap tm_v, const Params p) {
-  using L = Smem<D>;
+  static_assert(!F8 || (D == 128 && !VARLEN), "e4m3 inputs: d = 128, padded layout");
+  using L = Smem<D, F8>;
+  constexpr int XSTEP = F8 ? 128 : 64;  // columns per panel
   constexpr int NSLOT = L::NSLOT;
   extern __shared__ __align__(1024) uint8_t smem[];
   // The swizzled operand tiles need 1024-byte alignment; the kernel declares
@@ -278,7 +324,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         for (int w = 0; w < NQ; ++w)
           for (int pn = 0; pn < L::NPANEL; ++pn)
             load_rows<VARLEN>(smem + L::Q_OFF + w * L::TILE + pn * PANEL_BYTES, &tm_q, q_full,
-                              pn * 64, g.q0 + g.tile * BLOCK_M + w * TILE_M, g.head);
+                              pn * XSTEP, g.q0 + g.tile * BLOCK_M + w * TILE_M, g.head);
         ++n_items;
         for (int j = 0; j < n_kv1 && ok; ++j, ++kv) {
           // K_kv is ring tile 2 kv, V_kv is ring tile 2 kv + 1
@@ -290,10 +336,16 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
               break;
             }
             mbar_arrive_expect_tx(&full[slot], L::TILE);
-            for (int pn = 0; pn < L::NPANEL; ++pn)
-              load_rows<VARLEN>(smem + L::RING_OFF + slot * L::TILE + pn * PANEL_BYTES,
-                                half ? &tm_v : &tm_k, &full[slot], pn * 64,
-                                g.k0 + j * BLOCK_N, g.kv_head);
+            if (F8 && half) {
+              // V_j^T: rows d, columns keys j*128 ..
+              tma_load_3d(smem + L::RING_OFF + slot * L::TILE, &tm_v, &full[slot], j * BLOCK_N, 0,
+                          g.kv_head);
+            } else {
+              for (int pn = 0; pn < L::NPANEL; ++pn)
+                load_rows<VARLEN>(smem + L::RING_OFF + slot * L::TILE + pn * PANEL_BYTES,
+                                  half ? &tm_v : &tm_k, &full[slot], pn * XSTEP,
+                                  g.k0 + j * BLOCK_N, g.kv_head);
+            }
             ++loaded;
           }
         }
@@ -307,8 +359,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   } else if (warp == 9) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      constexpr uint32_t IDESC_S = idesc_bf16_f32(TILE_M, BLOCK_N, false, false);
-      constexpr uint32_t IDESC_O = idesc_bf16_f32(TILE_M, D, false, true);
+      constexpr uint32_t IDESC_S =
+          F8 ? idesc_e4m3_f32(TILE_M, BLOCK_N) : idesc_bf16_f32(TILE_M, BLOCK_N, false, false);
+      constexpr uint32_t IDESC_O =
+          F8 ? idesc_e4m3_f32(TILE_M, D) : idesc_bf16_f32(TILE_M, D, false, true);
+      const uint64_t p_desc0 = sdesc_kmajor_sw128(smem_u32(smem + L::P_OFF));  // F8 only
       const uint32_t q_addr = smem_u32(smem + L::Q_OFF);
       const uint32_t ring_addr = smem_u32(smem + L::RING_OFF);
       int pcount[NQ] = {0, 0};  // P tiles consumed per warpgroup (all items)
@@ -326,10 +381,18 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         const uint64_t qd = q_desc0 + static_cast<uint64_t>((w * L::TILE) >> 4);
         const uint64_t kd = ring_kdesc0 + static_cast<uint64_t>((slot * L::TILE) >> 4);
         const uint32_t dS = tmem_base + w * 128;
+        if constexpr (F8) {
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint64_t off = static_cast<uint64_t>(((kk >> 2) * PANEL_BYTES + (kk & 3) * 32) >> 4);
-          mma_bf16_ss(dS, qd + off, kd + off, IDESC_S, kk > 0 ? 1u : 0u);
+          for (int kk = 0; kk < D / 32; ++kk) {  // 32 e4m3 = 32 bytes per step
+            const uint64_t off = static_cast<uint64_t>(((kk >> 2) * PANEL_BYTES + (kk & 3) * 32) >> 4);
+            mma_f8_ss(dS, qd + off, kd + off, IDESC_S, kk > 0 ? 1u : 0u);
+          }
+        } else {
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint64_t off = static_cast<uint64_t>(((kk >> 2) * PANEL_BYTES + (kk & 3) * 32) >> 4);
+            mma_bf16_ss(dS, qd + off, kd + off, IDESC_S, kk > 0 ? 1u : 0u);
+          }
         }
         mma_commit(&s_full[w]);
       };
@@ -338,14 +401,25 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         if (!mbar_wait(&p_full[w], pcount[w] & 1, abort_flag)) return false;
         ++pcount[w];
         tc_fence_after();
-        const uint64_t vd = ring_vdesc0 + static_cast<uint64_t>((slot * L::TILE) >> 4);
-        const uint32_t tP = tmem_base + w * 128;
         const uint32_t tO = tmem_base + 256 + w * 128;
+        if constexpr (F8) {
+          // A = P_w (queries x keys) and B = V_j^T (d x keys), both K-major
+          const uint64_t pd = p_desc0 + static_cast<uint64_t>((w * PANEL_BYTES) >> 4);
+          const uint64_t vd = ring_kdesc0 + static_cast<uint64_t>((slot * L::TILE) >> 4);
 #pragma unroll
-        for (int kk = 0; kk < BLOCK_N / 16; ++kk) {
-          // keys 16kk .. 16kk+15: P columns 8kk.., V rows 16kk.. (2048 bytes per step)
-          mma_bf16_ts(tO, tP + kk * 8, vd + static_cast<uint64_t>((kk * 2048) >> 4), IDESC_O,
-                      (!first || kk > 0) ? 1u : 0u);
+          for (int kk = 0; kk < BLOCK_N / 32; ++kk) {
+            const uint64_t off = static_cast<uint64_t>((kk * 32) >> 4);
+            mma_f8_ss(tO, pd + off, vd + off, IDESC_O, (!first || kk > 0) ? 1u : 0u);
+          }
+        } else {
+          const uint64_t vd = ring_vdesc0 + static_cast<uint64_t>((slot * L::TILE) >> 4);
+          const uint32_t tP = tmem_base + w * 128;
+#pragma unroll
+          for (int kk = 0; kk < BLOCK_N / 16; ++kk) {
+            // keys 16kk .. 16kk+15: P columns 8kk.., V rows 16kk.. (2048 bytes per step)
+            mma_bf16_ts(tO, tP + kk * 8, vd + static_cast<uint64_t>((kk * 2048) >> 4), IDESC_O,
+                        (!first || kk > 0) ? 1u : 0u);
+          }
         }
         mma_commit(&o_done[w]);
         if (last) mma_commit(&o_final[w]);
@@ -466,6 +540,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 #pragma unroll
         for (int c = 0; c < 128; c += 32) {
           uint32_t pk[16];
+          float pf[32];
 #pragma unroll
           for (int e = 0; e < 32; e += 2) {
             const float x0 = fmaf(__uint_as_float(sr[c + e]), sl2, -m_ref);
@@ -479,10 +554,32 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
               p1 = ex2_approx(x1);
             }
             rs[(e >> 1) & 3] += p0 + p1;
-            pk[e >> 1] = pack_bf16x2(p0, p1);
+            if constexpr (F8) {
+              pf[e] = p0;
+              pf[e + 1] = p1;
+            } else {
+              pk[e >> 1] = pack_bf16x2(p0, p1);
+            }
           }
-          tmem_st16(tS + (c >> 1), pk);
+          if constexpr (F8) {
+            // keys c .. c+31 of row `row`: two 16-byte chunks of the 128-byte
+            // row, 128-byte swizzle (chunk index xor row % 8)
+            uint8_t* prow = smem + L::P_OFF + w * PANEL_BYTES + row * 128;
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+              const uint32_t ch = static_cast<uint32_t>((c >> 4) + h) ^ static_cast<uint32_t>(row & 7);
+              const float* f = pf + 16 * h;
+              *reinterpret_cast<uint4*>(prow + ch * 16) =
+                  make_uint4(pack_e4m3x4(f[0], f[1], f[2], f[3]), pack_e4m3x4(f[4], f[5], f[6], f[7]),
+                             pack_e4m3x4(f[8], f[9], f[10], f[11]),
+                             pack_e4m3x4(f[12], f[13], f[14], f[15]));
+            }
+          } else {
+            tmem_st16(tS + (c >> 1), pk);
+          }
         }
+        // e4m3 P is read by the async proxy (tensor core) from shared memory
+        if constexpr (F8) fence_proxy_async_smem();
         l = l * alpha + ((rs[0] + rs[1]) + (rs[2] + rs[3]));
         if (warp_grow && j > 0) {
           // O holds P_0 V_0 + ... + P_{j-1} V_{j-1} relative to the old max.
@@ -514,7 +611,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         break;
       }
       tc_fence_after();
-      const float inv_l = (l > 0.f) ? 1.f / l : 0.f;
+      const float inv_l = (l > 0.f) ? p.o_scale / l : 0.f;
       const bool valid = row_g < g.Nq;
       __nv_bfloat16* orow_g = p.o + static_cast<size_t>(g.head) * p.o_head +
                               static_cast<size_t>(g.q0 + row_g) * p.o_row;
@@ -558,18 +655,18 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   }
 }
 
-template <int D, bool CAUSAL, bool VARLEN>
+template <int D, bool CAUSAL, bool VARLEN, bool F8 = false>
 fa_status launch(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                  const Params& prm, int grid_size, cudaStream_t stream) {
-  auto kern = fa_fwd_kernel<D, CAUSAL, VARLEN>;
+  auto kern = fa_fwd_kernel<D, CAUSAL, VARLEN, F8>;
+  constexpr int SMEM = Smem<D, F8>::ALLOC;
   static bool configured = false;  // per process; the attribute is per function
   if (!configured) {
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         Smem<D>::ALLOC);
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM);
     if (e != cudaSuccess) return FA_ERR_CUDA;
     configured = true;
   }
-  kern<<<grid_size, NUM_THREADS, Smem<D>::ALLOC, stream>>>(tq, tk, tv, prm);
+  kern<<<grid_size, NUM_THREADS, SMEM, stream>>>(tq, tk, tv, prm);
   return cuda_status(cudaGetLastError());
 }
 
@@ -651,6 +748,7 @@ fa_status launch_fwd(const void* q, const void* k, const void* v, void* o, float
   prm.total_items = static_cast<int>(items);
   prm.lpt_order = persistent ? 1 : 0;
   prm.scale_log2 = scale * 1.4426950408889634f;
+  prm.o_scale = 1.f;
   prm.cu_q = nullptr;
   prm.cu_k = nullptr;
   prm.H = H;
@@ -701,6 +799,7 @@ fa_status launch_fwd_varlen(const void* q, const void* k, const void* v, void* o
   prm.total_items = static_cast<int>(items);
   prm.lpt_order = 0;  // one CTA per tile, a head's tiles adjacent, longest first
   prm.scale_log2 = scale * 1.4426950408889634f;
+  prm.o_scale = 1.f;
   prm.cu_q = cu_q;
   prm.cu_k = cu_k;
   prm.H = H;
@@ -715,6 +814,72 @@ fa_status launch_fwd_varlen(const void* q, const void* k, const void* v, void* o
                   : fwd::launch<128, false, true>(tq, tk, tv, prm, grid, stream);
   return causal ? fwd::launch<64, true, true>(tq, tk, tv, prm, grid, stream)
                 : fwd::launch<64, false, true>(tq, tk, tv, prm, grid, stream);
+}
+
+}  // namespace fa
+
+namespace fa {
+
+fa_status launch_fwd_fp8(const void* q, const void* k, const void* vt, void* o, float* lse,
+                         float q_scale, float k_scale, float v_scale, int B, int H, int Hkv,
+                         int Nq, int Nk, int causal, float scale, cudaStream_t stream) {
+  constexpr int d = 128;
+  const int BH = B * H;
+  if (Nq == 0) return FA_OK;
+  int dev = 0, sms = 148;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+    return FA_ERR_CUDA;
+  if (Nk == 0) {
+    fwd::fa_fwd_no_keys_kernel<<<4 * sms, 256, 0, stream>>>(
+        static_cast<__nv_bfloat16*>(o), lse, static_cast<size_t>(BH) * Nq, d);
+    return cuda_status(cudaGetLastError());
+  }
+  const long long n_cta_tiles = (Nq + fwd::BLOCK_M - 1) / fwd::BLOCK_M;
+  const long long items = static_cast<long long>(BH) * n_cta_tiles;
+  if (items > 0x7fffffffLL) return FA_ERR_INVALID_ARG;
+  CUtensorMap tq, tk, tv;
+  fa_status st;
+  const uint64_t BHkv = static_cast<uint64_t>(B) * Hkv;
+  // q, k: [heads, rows, 128 bytes]; vt: [heads, 128 rows (d), Nk bytes]
+  if ((st = make_tmap_u8_3d(&tq, q, d, Nq, BH, 128, fwd::TILE_M)) != FA_OK) return st;
+  if ((st = make_tmap_u8_3d(&tk, k, d, Nk, BHkv, 128, fwd::BLOCK_N)) != FA_OK) return st;
+  if ((st = make_tmap_u8_3d(&tv, vt, Nk, d, BHkv, 128, d)) != FA_OK) return st;
+  const double kv_bytes = 2.0 * B * Hkv * static_cast<double>(Nk) * d;
+  const int mode = fwd::schedule_mode();
+  bool persistent = causal && items > sms && kv_bytes <= 96.0 * 1024 * 1024;
+  int grid = persistent ? sms : static_cast<int>(items);
+  if (mode == 1) {
+    persistent = false;
+    grid = static_cast<int>(items);
+  } else if (mode == 2) {
+    persistent = true;
+    grid = static_cast<int>(std::min<long long>(sms, std::max<long long>(1, items / 3)));
+  }
+  fwd::Params prm;
+  prm.o = static_cast<__nv_bfloat16*>(o);
+  prm.lse = lse;
+  prm.Nq = Nq;
+  prm.Nk = Nk;
+  prm.causal_off = Nk - Nq;
+  prm.BH = BH;
+  prm.group = H / Hkv;
+  prm.n_cta_tiles = static_cast<int>(n_cta_tiles);
+  prm.total_items = static_cast<int>(items);
+  prm.lpt_order = persistent ? 1 : 0;
+  // scores of the real (descaled) values: q_scale * k_scale * (Q8 K8^T)
+  prm.scale_log2 = scale * q_scale * k_scale * 1.4426950408889634f;
+  prm.o_scale = v_scale;
+  prm.cu_q = nullptr;
+  prm.cu_k = nullptr;
+  prm.H = H;
+  prm.total_q = 0;
+  prm.total_k = 0;
+  prm.o_head = static_cast<size_t>(Nq) * d;
+  prm.o_row = static_cast<size_t>(d);
+  prm.lse_head = static_cast<size_t>(Nq);
+  return causal ? fwd::launch<128, true, false, true>(tq, tk, tv, prm, grid, stream)
+                : fwd::launch<128, false, false, true>(tq, tk, tv, prm, grid, stream);
 }
 
 }  // namespace fa

@@ -24,6 +24,12 @@ fa_status make_tmap_bf16_3d(CUtensorMap* map, const void* base, uint64_t d, uint
 fa_status make_tmap_bf16_rows_heads(CUtensorMap* map, const void* base, uint64_t d,
                                     uint64_t heads, uint64_t rows, uint32_t box_rows);
 
+// 3-D byte tensor map over an [outer, rows, inner] array (inner contiguous,
+// inner a multiple of 16) with a box_inner x box_rows x 1 box, box_inner = 128
+// (one 128-byte swizzle row); coordinates (column, row, outer).
+fa_status make_tmap_u8_3d(CUtensorMap* map, const void* base, uint64_t inner, uint64_t rows,
+                          uint64_t outer, uint32_t box_inner, uint32_t box_rows);
+
 // 2-D float32 tensor map over a [outer, n] array with a 128 x 1 box and no
 // swizzle; n * 4 must be a multiple of 16 bytes.
 fa_status make_tmap_f32_2d(CUtensorMap* map, const void* base, uint64_t n, uint64_t outer);
@@ -66,6 +72,12 @@ fa_status launch_bwd_varlen(const void* q, const void* k, const void* v, const v
                             const int* cu_q, const int* cu_k, void* workspace, int B, int H,
                             int Hkv, int total_q, int total_k, int max_seqlen_k, int d,
                             int causal, float scale, cudaStream_t stream);
+
+// e4m3 forward: q [B*H, Nq, 128], k [B*Hkv, Nk, 128], vt [B*Hkv, 128, Nk]
+// (V transposed), real values = stored values x the per-tensor descales.
+fa_status launch_fwd_fp8(const void* q, const void* k, const void* vt, void* o, float* lse,
+                         float q_scale, float k_scale, float v_scale, int B, int H, int Hkv,
+                         int Nq, int Nk, int causal, float scale, cudaStream_t stream);
 
 fa_status launch_bwd(const void* q, const void* k, const void* v, const void* o,
                      const void* dout, const float* lse, void* dq, void* dk, void* dv,

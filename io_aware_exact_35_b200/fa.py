@@ -33,6 +33,7 @@ SIGNATURES = {
     "fa_fwd_ext": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _F, _P]),
     "fa_fwd_varlen": (_I, [_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _F,
                            _P]),
+    "fa_fwd_fp8": (_I, [_P, _P, _P, _P, _P, _F, _F, _F, _I, _I, _I, _I, _I, _I, _I, _F, _P]),
     "fa_bwd_workspace_size": (_S, [_I, _I, _I, _I]),
     "fa_bwd_varlen_workspace_size": (_S, [_I, _I, _I, _I]),
     "fa_bwd_varlen": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _S, _I, _I, _I, _I, _I,
@@ -178,6 +179,32 @@ def fwd_varlen(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, cu_seqlens_q: 
                              total_k, int(max_seqlen_q), d, int(bool(causal)), scale,
                              _stream_ptr(stream))
     _check("fa_fwd_varlen", st)
+    return out, lse
+
+
+def fwd_fp8(q: torch.Tensor, k: torch.Tensor, vt: torch.Tensor, q_scale: float,
+            k_scale: float, v_scale: float, causal: bool = False, scale: Optional[float] = None,
+            out: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None,
+            want_lse: bool = True, stream=None):
+    """Forward with e4m3 inputs: q [B, H, Nq, 128], k [B, Hkv, Nk, 128] and V
+    transposed, vt [B, Hkv, 128, Nk] (torch.float8_e4m3fn), one descale factor
+    per tensor.  Returns (o [B, H, Nq, 128] bf16, lse [B, H, Nq])."""
+    for t, n in ((q, "q"), (k, "k"), (vt, "vt")):
+        _req(t, n, torch.float8_e4m3fn, 4)
+    B, H, N, d = q.shape
+    Hkv, Nk = k.shape[1], k.shape[2]
+    if tuple(k.shape) != (B, Hkv, Nk, d) or tuple(vt.shape) != (B, Hkv, d, Nk) or H % Hkv:
+        raise ValueError("k must be [B, Hkv, Nk, d] and vt [B, Hkv, d, Nk], Hkv dividing H")
+    scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
+    if out is None:
+        out = torch.empty((B, H, N, d), dtype=torch.bfloat16, device=q.device)
+    _req(out, "out", torch.bfloat16, 4)
+    if lse is None and want_lse:
+        lse = torch.empty((B, H, N), dtype=torch.float32, device=q.device)
+    st = lib().fa_fwd_fp8(q.data_ptr(), k.data_ptr(), vt.data_ptr(), out.data_ptr(), _ptr(lse),
+                          float(q_scale), float(k_scale), float(v_scale), B, H, Hkv, N, Nk, d,
+                          int(bool(causal)), scale, _stream_ptr(stream))
+    _check("fa_fwd_fp8", st)
     return out, lse
 
 

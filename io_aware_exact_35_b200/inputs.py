@@ -29,7 +29,7 @@ BASE_SEED = 42
 @dataclass(frozen=True)
 class Workload:
     name: str
-    kind: str            # "fwd" | "bwd" | "decode" | "fwd_varlen"
+    kind: str            # "fwd" | "bwd" | "decode" | "fwd_varlen" | "fwd_fp8"
     B: int
     H: int
     d: int
@@ -76,6 +76,9 @@ WORKLOADS = {
         # a ragged prefill batch: 16 sequences of U{512..4096} tokens, packed
         Workload("fwd_varlen_causal_B16_H16_d128_L512-4096", "fwd_varlen", 16, 16, 128,
                  causal=True, Lmin=512, Lmax=4096, seed=BASE_SEED + 9),
+        # the 2K-context prefill with e4m3 inputs (V supplied transposed)
+        Workload("fwd_fp8_causal_B4_H16_N2048_d128", "fwd_fp8", 4, 16, 128, N=2048,
+                 causal=True, seed=BASE_SEED + 10),
         # the decode workload over a paged cache (16-row pages, random page order)
         Workload("decode_paged_B16_H32_d128_L4096-16384_p16", "decode", 16, 32, 128,
                  Lmin=4096, Lmax=16384, seed=BASE_SEED + 8, page=16),
@@ -163,6 +166,38 @@ def varlen_inputs(seqlens_q, seqlens_k, H: int, Hkv: int, d: int, seed: int,
     return (*out, cu_q, cu_k)
 
 
+E4M3_MAX = 448.0
+
+
+def fp8_inputs(B: int, H: int, Nq: int, d: int, seed: int, Hkv: int | None = None,
+               Nk: int | None = None, std: float = 1.0):
+    """e4m3 inputs for the FP8 forward: q [B, H, Nq, d], k [B, Hkv, Nk, d] and
+    V transposed, vt [B, Hkv, d, Nk], as torch.float8_e4m3fn CPU tensors, with
+    one descale factor per tensor (real value = stored value x factor).
+
+    q, k, v ~ N(0,1) * std are drawn as float32 in that order; each tensor is
+    divided by its factor amax / 448 and rounded to e4m3 (round to nearest
+    even) -- data preparation, no attention arithmetic.  Returns
+    (q8, k8, vt8, (q_scale, k_scale, v_scale))."""
+    g = _gen(seed)
+    hk = Hkv or H
+    nk = Nq if Nk is None else Nk
+    out, scales = [], []
+    for shape in ((B, H, Nq, d), (B, hk, nk, d), (B, hk, nk, d)):
+        x = torch.randn(shape, generator=g, dtype=torch.float32) * std
+        amax = float(x.abs().max()) if x.numel() else 1.0
+        sc = max(amax, 1e-30) / E4M3_MAX
+        out.append((x / sc).to(torch.float8_e4m3fn))
+        scales.append(sc)
+    q8, k8, v8 = out
+    return q8, k8, v8.transpose(-1, -2).contiguous(), tuple(scales)
+
+
+def fp8_to_f64(t: torch.Tensor, scale: float) -> np.ndarray:
+    """Exact real values of an e4m3 tensor: stored value x descale factor."""
+    return t.to(torch.float64).numpy() * scale
+
+
 def page_cache(kc: torch.Tensor, vc: torch.Tensor, seqlens, page_size: int, seed: int,
                spare_pages: int = 3):
     """Scatter contiguous caches [B, Hkv, Lcap, d] into page pools
@@ -201,6 +236,8 @@ def varlen_lengths(w: Workload) -> list:
 
 
 def workload_inputs(w: Workload):
+    if w.kind == "fwd_fp8":
+        return fp8_inputs(w.B, w.H, w.N, w.d, w.seed, Hkv=w.kv_heads, std=w.std)
     if w.kind == "fwd_varlen":
         lens = varlen_lengths(w)
         return varlen_inputs(lens, lens, w.H, w.kv_heads, w.d, w.seed + 1, w.std)

@@ -107,6 +107,12 @@ def test_host_validation_rejects_bad_arguments(fa_mod):
     assert bvl(*ten, P, 1 << 30, 2, 4, 2, 100, 100, 64, 96, 1, 1.0, None) == UNSUPPORTED
     assert lib.fa_bwd_varlen_workspace_size(2, 4, 100, 128) > 0
     assert lib.fa_bwd_varlen_workspace_size(0, 4, 100, 128) == 0
+    f8 = lib.fa_fwd_fp8
+    assert f8(P, P, P, P, None, 1.0, 1.0, 1.0, 1, 2, 2, 64, 64, 64, 0, 1.0, None) == UNSUPPORTED   # d
+    assert f8(P, P, P, P, None, 1.0, 1.0, 1.0, 1, 2, 2, 64, 40, 128, 0, 1.0, None) == UNSUPPORTED  # Nk % 16
+    assert f8(P, P, P, P, None, float("nan"), 1.0, 1.0, 1, 2, 2, 64, 64, 128, 0, 1.0, None) == INVALID
+    assert f8(P, P, None, P, None, 1.0, 1.0, 1.0, 1, 2, 2, 64, 64, 128, 0, 1.0, None) == INVALID
+    assert f8(P, P, P, P, None, 1.0, 1.0, 1.0, 1, 2, 3, 64, 64, 128, 0, 1.0, None) == INVALID
     # paged decode: page size must be a power of two, table needed
     dp = lib.fa_decode_paged
     assert dp(P, P, P, P, P, P, None, 2, 4, 2, 24, 8, 16, 128, 1.0, P, 1 << 20, None) == INVALID
