@@ -293,6 +293,9 @@ __global__ void __launch_bounds__(THREADS)
 #pragma unroll
     for (int e = 0; e < 8; ++e) qf[g][e] *= scale_log2;
   }
+  const size_t bkv = static_cast<size_t>(b) * Hkv + hk;
+  const __nv_bfloat16* kbase = kc + bkv * static_cast<size_t>(Lmax) * D + sub * 8;
+  const __nv_bfloat16* vbase = vc + bkv * static_cast<size_t>(Lmax) * D + sub * 8;
   __shared__ int spages[PAGED ? CHUNK : 1];
   const auto rows = kv_rows<D, PAGED>(kc, vc, pg, spages, b, hk, Hkv, Lmax, c0, c1, sub);
   float m[G], l[G], acc[G][8];
@@ -306,24 +309,29 @@ __global__ void __launch_bounds__(THREADS)
   constexpr int KEYS_PER_ROUND = WARPS * UN * KPW;
   for (int r0 = c0; r0 < c1; r0 += KEYS_PER_ROUND) {
     uint4 ku[UN], vu[UN];
-    bool live[UN];
+    int key[UN];
+    bool live[UN];  // paged: the key exists and its page entry is valid
 #pragma unroll
     for (int u = 0; u < UN; ++u) {
-      const int key = r0 + (warp * UN + u) * KPW + kin;
-      long long off;
+      key[u] = r0 + (warp * UN + u) * KPW + kin;
       if constexpr (PAGED) {
-        off = key < c1 ? rows.off(key) : 0;
-        live[u] = key < c1 && off >= 0;
+        const long long off = key[u] < c1 ? rows.off(key[u]) : 0;
+        live[u] = key[u] < c1 && off >= 0;
+        if (live[u]) {
+          ku[u] = ld_stream(rows.k + off);
+          vu[u] = ld_stream(rows.v + off);
+        } else {
+          ku[u] = make_uint4(0, 0, 0, 0);
+          vu[u] = make_uint4(0, 0, 0, 0);
+        }
       } else {
-        off = static_cast<long long>(static_cast<size_t>(key) * D);
-        live[u] = key < c1;
-      }
-      if (live[u]) {
-        ku[u] = ld_stream(rows.k + off);
-        vu[u] = ld_stream(rows.v + off);
-      } else {
-        ku[u] = make_uint4(0, 0, 0, 0);
-        vu[u] = make_uint4(0, 0, 0, 0);
+        if (key[u] < c1) {
+          ku[u] = ld_stream(kbase + static_cast<size_t>(key[u]) * D);
+          vu[u] = ld_stream(vbase + static_cast<size_t>(key[u]) * D);
+        } else {
+          ku[u] = make_uint4(0, 0, 0, 0);
+          vu[u] = make_uint4(0, 0, 0, 0);
+        }
       }
     }
     float s[UN][G];
@@ -338,7 +346,10 @@ __global__ void __launch_bounds__(THREADS)
         for (int e = 0; e < 8; ++e) t = fmaf(qf[g][e], kf[e], t);
 #pragma unroll
         for (int off = LPK / 2; off > 0; off >>= 1) t += __shfl_xor_sync(0xffffffffu, t, off);
-        s[u][g] = live[u] ? t : -INFINITY;
+        bool keep;
+        if constexpr (PAGED) keep = live[u];
+        else keep = key[u] < c1;
+        s[u][g] = keep ? t : -INFINITY;
       }
     }
 #pragma unroll
