@@ -46,15 +46,19 @@ def test_gqa_backward(fa_mod, cuda_device, shape, causal):
     check_grad(dv.cpu(), rv, "dV")
 
 
-@pytest.mark.parametrize("Hkv", [1, 4, 8])
-def test_gqa_decode(fa_mod, cuda_device, Hkv):
-    q, kc, vc, sl = inputs.decode_inputs(3, 8, 128, 1, 2100, seed=500 + Hkv, Hkv=Hkv,
-                                         seqlens=[0, 700, 2100], Lcap=2100)
+@pytest.mark.parametrize("d", [128, 64])
+@pytest.mark.parametrize("Hkv", [1, 2, 4, 8])
+def test_gqa_decode(fa_mod, cuda_device, Hkv, d):
+    """Groups of 8, 4, 2 and 1 query heads per cached head; lengths around the
+    shared-memory stage (32 / 64 rows) and split (512 rows) boundaries, and 0."""
+    sl = [0, 1, 31, 32, 33, 64, 511, 512, 513, 700, 2100]
+    q, kc, vc, sl = inputs.decode_inputs(len(sl), 8, d, 0, 2100, seed=500 + Hkv + d, Hkv=Hkv,
+                                         seqlens=sl, Lcap=2100)
     o, lse = fa_mod.decode(q.cuda(), kc.cuda(), vc.cuda(), sl.cuda())
     torch.cuda.synchronize()
     assert fa_mod.get_device_error() == 0
     ref_o, ref_l = oracle.decode_forward(inputs.to_f64(q), inputs.to_f64(kc), inputs.to_f64(vc),
-                                         sl.tolist(), 1 / np.sqrt(128))
+                                         sl.tolist(), 1 / np.sqrt(d))
     check_o(o.cpu(), ref_o)
     check_lse(lse.cpu(), ref_l)
 
