@@ -351,6 +351,20 @@ fa_status fa_decode_static(const void* q, const void* kcache, const void* vcache
  */
 fa_status fa_get_device_error(fa_stream_t stream);
 
+/*
+ * Self-check of the failure detection behind FA_ERR_TIMEOUT ("FlashAttention:
+ * Fast and Memory-Efficient Exact Attention with IO-Awareness" fixes no
+ * failure model; this is the library's own).  Launches one CTA that waits,
+ * with the same bounded waits as the attention kernels (a single-thread wait
+ * and a warp-collective one), on an mbarrier that nothing arrives on.  After
+ * the wait limit (2 s) both give up: the device error word becomes
+ * FA_ERR_TIMEOUT and 2 is added to *gave_up (a device int, 4-byte aligned,
+ * owned by the caller), and the kernel returns; the context stays usable.
+ * Returns FA_ERR_INVALID_ARG for a null or misaligned pointer,
+ * FA_ERR_UNSUPPORTED off sm_100, FA_ERR_CUDA if the launch fails.
+ */
+fa_status fa_check_bounded_wait(int* gave_up, fa_stream_t stream);
+
 /* Static, NUL-terminated description of a status code. */
 const char* fa_status_string(fa_status status);
 

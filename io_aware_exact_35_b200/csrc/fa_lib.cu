@@ -6,3 +6,4 @@
 #include "fa_bwd.cu"
 #include "fa_decode.cu"
 #include "fa_decode_static.cu"
+#include "fa_selftest.cu"

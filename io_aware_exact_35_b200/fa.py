@@ -50,6 +50,7 @@ SIGNATURES = {
     "fa_decode_paged": (_I, [_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _F, _P, _S,
                              _P]),
     "fa_get_device_error": (_I, [_P]),
+    "fa_check_bounded_wait": (_I, [_P, _P]),
     "fa_status_string": (ctypes.c_char_p, [_I]),
     "fa_version": (_I, []),
 }
@@ -395,3 +396,12 @@ def decode_static(q, kcache, vcache, seqlens, scale: Optional[float] = None, out
 def get_device_error(stream=None) -> int:
     """Synchronise the stream and return (and clear) the device error word."""
     return int(lib().fa_get_device_error(_stream_ptr(stream)))
+
+
+def check_bounded_wait(gave_up: torch.Tensor, stream=None) -> None:
+    """Launch the bounded-wait self-check: one CTA waits on a barrier that
+    never completes, gives up after the wait limit and records FA_ERR_TIMEOUT
+    in the device error word; 2 is added to ``gave_up`` (an int32 CUDA tensor)."""
+    _req(gave_up, "gave_up", torch.int32, 1)
+    _check("fa_check_bounded_wait", lib().fa_check_bounded_wait(gave_up.data_ptr(),
+                                                                _stream_ptr(stream)))

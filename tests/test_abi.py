@@ -130,3 +130,10 @@ def test_binding_fails_loudly_without_cuda_tensors(fa_mod):
     x = torch.zeros(1, 1, 8, 64, dtype=torch.bfloat16)
     with pytest.raises(ValueError):
         fa_mod.fwd(x, x, x)
+
+
+def test_bounded_wait_check_validates_pointer(fa_mod):
+    lib = fa_mod.lib()
+    INVALID = 1
+    assert lib.fa_check_bounded_wait(None, None) == INVALID
+    assert lib.fa_check_bounded_wait((1 << 20) + 2, None) == INVALID
