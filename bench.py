@@ -241,8 +241,10 @@ class Runner:
             self.launches_per_step = 2
             group = w.H // w.kv_heads
             paged = ",paged" if w.page else ""
-            self.kernel_key = (f"fa_decode_group_split_kernel<{w.d},{group}{paged}>"
-                               if group in (2, 4, 8) else f"fa_decode_split_kernel<{w.d}{paged}>")
+            # heads per CTA of the grouped (tensor-core) decode kernel
+            qh = group if group <= 16 else (16 if group % 16 == 0 else (8 if group % 8 == 0 else 0))
+            self.kernel_key = (f"fa_decode_group_mma_kernel<{w.d},{qh}{paged}>"
+                               if group > 1 and qh > 0 else f"fa_decode_split_kernel<{w.d}{paged}>")
             self.out_host = torch.empty(self.o.shape, dtype=torch.bfloat16).pin_memory()
         self.working_set = sum(t.numel() * t.element_size() for t in self.dbuf)
         self.flush = None

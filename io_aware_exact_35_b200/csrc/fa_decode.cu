@@ -12,9 +12,11 @@
 //   M = max_s m_s,  w_s = 2^(m_s - M),  o = sum w_s acc_s / sum w_s l_s,
 //   lse = (M + log2 sum w_s l_s) * ln 2      (m in log2 units).
 //
-// Layout inside a CTA (4 warps): D/8 lanes share one key (8 bf16 = 16 bytes
-// each), so a warp covers 32/(D/8) consecutive keys per step and issues
-// UNROLL steps of K and V loads before using any of them.
+// Layout inside a CTA (4 warps), one query head per CTA: D/8 lanes share one
+// key (8 bf16 = 16 bytes each), so a warp covers 32/(D/8) consecutive keys
+// per step and issues UNROLL steps of K and V loads before using any of them.
+// Grouped query heads (several heads per key/value head) are served together
+// by a tensor-core kernel that reads each cached row once for the group.
 //
 // The cache is either contiguous, [B, Hkv, Lmax, d], or paged: pools of
 // [num_pages, Hkv, page, d] with page a power of two and a per-sequence page
@@ -119,6 +121,22 @@ __device__ __forceinline__ void bf16x8_to_f32(const uint4& u, float (&f)[8]) {
     f[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
   }
 }
+
+// D += A B for one m16n8k16 tile: A 16 x 16 bf16 (row-major fragment a0..a3),
+// B 16 x 8 bf16 (column-major fragment b0, b1), D 16 x 8 f32 (PTX ISA,
+// "Matrix fragments for mma.m16n8k16").
+__device__ __forceinline__ void mma_bf16_16816(float (&d)[4], uint32_t a0, uint32_t a1,
+                                               uint32_t a2, uint32_t a3, uint32_t b0,
+                                               uint32_t b1) {
+  asm("mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, "
+      "{%4, %5, %6, %7}, {%8, %9}, {%0, %1, %2, %3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// A row's maximum is only moved (and O, l rescaled) once it has grown by
+// more than 2^8 (log2 units).
+constexpr float STALE_MAX = 8.0f;
 
 template <int D, bool PAGED>
 __global__ void __launch_bounds__(THREADS)
@@ -257,154 +275,269 @@ __global__ void __launch_bounds__(THREADS)
   }
 }
 
-// Grouped-query decode: one CTA streams one chunk of one key/value head and
-// serves all G query heads that share it, so every cached row is read once.
-// Each lane keeps the G query slices, and per head a running (m, l, acc).
-template <int D, int G, bool PAGED>
+// Grouped-query decode on the tensor cores.  The G query heads that share a
+// key/value head form a small dense contraction, S = Q_g K^T and
+// O_g += P V with Q_g of G rows, so one warp runs it with mma.sync
+// m16n8k16 (bf16 operands, f32 accumulation) straight from registers, 16
+// keys per step: S with the heads as the 16 rows (padded when G < 16), then
+// O^T += V^T P^T with the heads as the 8 columns of each n-tile, which takes
+// the S accumulator re-packed to bf16 as its B operand unchanged.  The
+// per-key work drops from ~60 warp instructions of FMAs and shuffles to
+// ~7, and the kernel is left bound by the cache reads.  (tcgen05 needs at
+// least 64 rows and shared-memory operands; with 2-16 heads the
+// register-only mma.sync form avoids staging.)
+//
+// Operand placement.  The dot product over d and the sum over keys do not
+// depend on the order of their terms, so every lane loads whole 16-byte
+// vectors and the fragment slots are assigned to match them; lane
+// (g, c) = (lane / 4, lane % 4):
+//   S, k-step s (16 of the d values): B = K[key g][dk .. dk+3] and
+//     A = Q[head g (and g + 8)][the same d], dk = 32 (s/2) + 8c + 4 (s%2):
+//     four lanes' 16-byte loads cover 64 consecutive bytes of a key row.
+//   O^T, m-tile t: A = V^T, rows g and g + 8 being d values e = t and
+//     e = t + D/16 of the lane's own list d(e) = 64 (e/8) + 8g + e%8, columns
+//     keys 2c, 2c+1, 2c+8, 2c+9: each lane loads those four rows at d 8g ..
+//     8g+7 (and 64 + 8g ..), eight lanes covering 128 consecutive bytes of a
+//     row per load, and pairs two keys' bf16 with one byte permute.  B = P^T:
+//     column g, keys 2c, 2c+1 (and 2c+8, 2c+9), exactly the S accumulator
+//     entries of lane (g, c).
+// The online softmax is the one of the other decode kernels (log2 units,
+// running max m and sum l per head), with the maximum kept stale until it
+// grows by more than 2^8, as in the forward kernel.
+template <int D, bool HI, bool PAGED>
 __global__ void __launch_bounds__(THREADS)
-    fa_decode_group_split_kernel(const __nv_bfloat16* __restrict__ q,
-                                 const __nv_bfloat16* __restrict__ kc,
-                                 const __nv_bfloat16* __restrict__ vc,
-                                 const int* __restrict__ seqlens, float* __restrict__ part, int H,
-                                 int Hkv, int Lmax, int S, float scale_log2, const Pages pg) {
-  constexpr int LPK = D / 8;
-  constexpr int KPW = 32 / LPK;
-  constexpr int HW = WARPS * KPW;
-  constexpr int UN = G <= 2 ? 8 : (G == 4 ? 4 : 2);  // keys in flight per lane (registers)
+    fa_decode_group_mma_kernel(const __nv_bfloat16* __restrict__ q,
+                               const __nv_bfloat16* __restrict__ kc,
+                               const __nv_bfloat16* __restrict__ vc,
+                               const int* __restrict__ seqlens, float* __restrict__ part, int H,
+                               int Hkv, int group, int qh, int Lmax, int S, float scale_log2,
+                               const Pages pg) {
+  constexpr int ROWS = HI ? 16 : 8;  // head rows that can be real
+  constexpr int NH = HI ? 2 : 1;     // 8-head column tiles of O^T
+  constexpr int KS = D / 16;         // k-steps of S = Q K^T
+  constexpr int MT = D / 16;         // m-tiles of O^T
+  constexpr int NKL = D / 32;        // 16-byte loads per K row per lane
+  constexpr int NVL = D / 64;        // 16-byte loads per V row per lane
   const int split = blockIdx.x;
-  const int hk = blockIdx.y;
+  const int h0 = blockIdx.y * qh;    // first query head of this CTA
   const int b = blockIdx.z;
+  const int hk = h0 / group;
   const int L = min(max(seqlens[b], 0), Lmax);
   const int c0 = split * CHUNK;
   if (c0 >= L) return;
   const int c1 = min(c0 + CHUNK, L);
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int sub = lane % LPK;
-  const int kin = lane / LPK;
-  const int grp = warp * KPW + kin;
-  const size_t bh0 = static_cast<size_t>(b) * H + static_cast<size_t>(hk) * G;  // first query head
+  const int g = lane >> 2;
+  const int c = lane & 3;
 
-  float qf[G][8];
+  // Q as the A operand of S: rows g and g + 8, 4 d values per k-step
+  uint32_t qa[KS][2], qb[KS][2];
+  {
+    const uint32_t* q0 = reinterpret_cast<const uint32_t*>(
+        q + (static_cast<size_t>(b) * H + h0 + g) * D);
+    const uint32_t* q1 = reinterpret_cast<const uint32_t*>(
+        q + (static_cast<size_t>(b) * H + h0 + g + 8) * D);
 #pragma unroll
-  for (int g = 0; g < G; ++g) {
-    const uint4 qu = *reinterpret_cast<const uint4*>(q + (bh0 + g) * D + sub * 8);
-    bf16x8_to_f32(qu, qf[g]);
-#pragma unroll
-    for (int e = 0; e < 8; ++e) qf[g][e] *= scale_log2;
+    for (int s = 0; s < KS; ++s) {
+      const int d0 = 32 * (s >> 1) + 8 * c + 4 * (s & 1);
+      qa[s][0] = g < qh ? q0[d0 >> 1] : 0u;
+      qa[s][1] = g < qh ? q0[(d0 >> 1) + 1] : 0u;
+      qb[s][0] = (HI && g + 8 < qh) ? q1[d0 >> 1] : 0u;
+      qb[s][1] = (HI && g + 8 < qh) ? q1[(d0 >> 1) + 1] : 0u;
+    }
   }
   const size_t bkv = static_cast<size_t>(b) * Hkv + hk;
-  const __nv_bfloat16* kbase = kc + bkv * static_cast<size_t>(Lmax) * D + sub * 8;
-  const __nv_bfloat16* vbase = vc + bkv * static_cast<size_t>(Lmax) * D + sub * 8;
+  const __nv_bfloat16* kbase = kc + bkv * static_cast<size_t>(Lmax) * D;
+  const __nv_bfloat16* vbase = vc + bkv * static_cast<size_t>(Lmax) * D;
   __shared__ int spages[PAGED ? CHUNK : 1];
-  const auto rows = kv_rows<D, PAGED>(kc, vc, pg, spages, b, hk, Hkv, Lmax, c0, c1, sub);
-  float m[G], l[G], acc[G][8];
+  const auto rows = kv_rows<D, PAGED>(kc, vc, pg, spages, b, hk, Hkv, Lmax, c0, c1, 0);
+  // element offset of a key's row; -1 when the key is masked (past the
+  // prefix, or an invalid page entry)
+  auto row_off = [&](int key) -> long long {
+    if (key >= c1) return -1;
+    if constexpr (PAGED) return rows.off(key);
+    else return static_cast<long long>(key) * D;
+  };
+
+  uint4 kr[2][NKL];  // K rows kb + g and kb + 8 + g
+  uint4 vr[4][NVL];  // V rows kb + 2c, kb + 2c + 1, kb + 8 + 2c, kb + 9 + 2c
+  bool klive[2];
+  auto load_k = [&](int kb) {
 #pragma unroll
-  for (int g = 0; g < G; ++g) {
-    m[g] = -INFINITY;
-    l[g] = 0.f;
+    for (int t = 0; t < 2; ++t) {
+      const long long off = row_off(kb + 8 * t + g);
+      klive[t] = off >= 0;
 #pragma unroll
-    for (int e = 0; e < 8; ++e) acc[g][e] = 0.f;
+      for (int i = 0; i < NKL; ++i)
+        kr[t][i] = off >= 0 ? ld_stream((PAGED ? rows.k : kbase) + off + 32 * i + 8 * c)
+                            : make_uint4(0, 0, 0, 0);
+    }
+  };
+  auto load_v = [&](int kb) {
+#pragma unroll
+    for (int r = 0; r < 4; ++r) {
+      const long long off = row_off(kb + 8 * (r >> 1) + 2 * c + (r & 1));
+#pragma unroll
+      for (int i = 0; i < NVL; ++i)
+        vr[r][i] = off >= 0 ? ld_stream((PAGED ? rows.v : vbase) + off + 64 * i + 8 * g)
+                            : make_uint4(0, 0, 0, 0);
+    }
+  };
+  // bf16 pair (key a, key b) at entry e of the lane's V list
+  auto vpair = [&](int ra, int rb, int e) -> uint32_t {
+    const uint4& ua = vr[ra][e >> 3];
+    const uint4& ub = vr[rb][e >> 3];
+    const int w = (e & 7) >> 1;
+    const uint32_t wa = w == 0 ? ua.x : w == 1 ? ua.y : w == 2 ? ua.z : ua.w;
+    const uint32_t wb = w == 0 ? ub.x : w == 1 ? ub.y : w == 2 ? ub.z : ub.w;
+    return __byte_perm(wa, wb, (e & 1) ? 0x7632u : 0x5410u);
+  };
+
+  float o[NH][MT][4];  // O^T: [head tile][d tile]
+#pragma unroll
+  for (int n = 0; n < NH; ++n)
+#pragma unroll
+    for (int t = 0; t < MT; ++t) o[n][t][0] = o[n][t][1] = o[n][t][2] = o[n][t][3] = 0.f;
+  float m[2] = {-INFINITY, -INFINITY};  // heads g, g + 8 (log2 units, stale)
+  float l[2] = {0.f, 0.f};              // this lane's share of their sums
+
+  int kb = c0 + 16 * warp;
+  if (kb < c1) {
+    load_k(kb);
+    load_v(kb);
   }
-  constexpr int KEYS_PER_ROUND = WARPS * UN * KPW;
-  for (int r0 = c0; r0 < c1; r0 += KEYS_PER_ROUND) {
-    uint4 ku[UN], vu[UN];
-    int key[UN];
-    bool live[UN];  // paged: the key exists and its page entry is valid
+  for (; kb < c1; kb += 16 * WARPS) {
+    const int nb = kb + 16 * WARPS;
+    // S = Q K^T for keys kb .. kb+7 (half 0) and kb+8 .. kb+15 (half 1)
+    float sc[2][4];
 #pragma unroll
-    for (int u = 0; u < UN; ++u) {
-      key[u] = r0 + (warp * UN + u) * KPW + kin;
-      if constexpr (PAGED) {
-        const long long off = key[u] < c1 ? rows.off(key[u]) : 0;
-        live[u] = key[u] < c1 && off >= 0;
-        if (live[u]) {
-          ku[u] = ld_stream(rows.k + off);
-          vu[u] = ld_stream(rows.v + off);
-        } else {
-          ku[u] = make_uint4(0, 0, 0, 0);
-          vu[u] = make_uint4(0, 0, 0, 0);
+    for (int t = 0; t < 2; ++t) {
+      sc[t][0] = sc[t][1] = sc[t][2] = sc[t][3] = 0.f;
+#pragma unroll
+      for (int s = 0; s < KS; ++s) {
+        const uint4& u = kr[t][s >> 1];
+        mma_bf16_16816(sc[t], qa[s][0], qb[s][0], qa[s][1], qb[s][1], (s & 1) ? u.z : u.x,
+                       (s & 1) ? u.w : u.y);
+      }
+    }
+    // column 2c + j of half t is key kb + 8t + 2c + j, loaded (or found
+    // masked) by lanes 4 (2c + j) .. 4 (2c + j) + 3
+    bool live[2][2];
+#pragma unroll
+    for (int t = 0; t < 2; ++t)
+#pragma unroll
+      for (int j = 0; j < 2; ++j)
+        live[t][j] = __shfl_sync(0xffffffffu, static_cast<int>(klive[t]), 4 * (2 * c + j)) != 0;
+    if (nb < c1) load_k(nb);
+
+    uint32_t pb[2][2] = {{0u, 0u}, {0u, 0u}};  // P^T as the B operand: [head half][key half]
+    float alpha[2] = {1.f, 1.f};
+    bool grew = false;
+#pragma unroll
+    for (int r = 0; r < NH; ++r) {
+      float x[2][2];
+      float mx = -INFINITY;
+#pragma unroll
+      for (int t = 0; t < 2; ++t)
+#pragma unroll
+        for (int j = 0; j < 2; ++j) {
+          x[t][j] = live[t][j] ? sc[t][2 * r + j] * scale_log2 : -INFINITY;
+          mx = fmaxf(mx, x[t][j]);
         }
-      } else {
-        if (key[u] < c1) {
-          ku[u] = ld_stream(kbase + static_cast<size_t>(key[u]) * D);
-          vu[u] = ld_stream(vbase + static_cast<size_t>(key[u]) * D);
-        } else {
-          ku[u] = make_uint4(0, 0, 0, 0);
-          vu[u] = make_uint4(0, 0, 0, 0);
+      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+      const float m_new = fmaxf(m[r], mx);
+      if (m_new - m[r] > STALE_MAX) {  // also when m = -inf < m_new
+        alpha[r] = ex2_approx(m[r] - m_new);
+        l[r] *= alpha[r];
+        m[r] = m_new;
+        grew = true;
+      }
+      const float mref = (m[r] == -INFINITY) ? 0.f : m[r];
+#pragma unroll
+      for (int t = 0; t < 2; ++t) {
+        const float p0 = ex2_approx(x[t][0] - mref);
+        const float p1 = ex2_approx(x[t][1] - mref);
+        l[r] += p0 + p1;
+        pb[r][t] = pack_bf16x2(p0, p1);
+      }
+    }
+    if (__any_sync(0xffffffffu, grew)) {
+      // column j of head tile n is head 8n + 2c + j, whose factor lane
+      // 4 (2c + j) computed
+#pragma unroll
+      for (int n = 0; n < NH; ++n) {
+        const float a0 = __shfl_sync(0xffffffffu, alpha[n], 8 * c);
+        const float a1 = __shfl_sync(0xffffffffu, alpha[n], 8 * c + 4);
+#pragma unroll
+        for (int t = 0; t < MT; ++t) {
+          o[n][t][0] *= a0;
+          o[n][t][1] *= a1;
+          o[n][t][2] *= a0;
+          o[n][t][3] *= a1;
         }
       }
     }
-    float s[UN][G];
+
+    // O^T += V^T P^T
 #pragma unroll
-    for (int u = 0; u < UN; ++u) {
-      float kf[8];
-      bf16x8_to_f32(ku[u], kf);
+    for (int t = 0; t < MT; ++t) {
+      const uint32_t a0 = vpair(0, 1, t);
+      const uint32_t a1 = vpair(0, 1, t + MT);
+      const uint32_t a2 = vpair(2, 3, t);
+      const uint32_t a3 = vpair(2, 3, t + MT);
 #pragma unroll
-      for (int g = 0; g < G; ++g) {
-        float t = 0.f;
-#pragma unroll
-        for (int e = 0; e < 8; ++e) t = fmaf(qf[g][e], kf[e], t);
-#pragma unroll
-        for (int off = LPK / 2; off > 0; off >>= 1) t += __shfl_xor_sync(0xffffffffu, t, off);
-        bool keep;
-        if constexpr (PAGED) keep = live[u];
-        else keep = key[u] < c1;
-        s[u][g] = keep ? t : -INFINITY;
-      }
+      for (int n = 0; n < NH; ++n) mma_bf16_16816(o[n][t], a0, a1, a2, a3, pb[n][0], pb[n][1]);
     }
-#pragma unroll
-    for (int g = 0; g < G; ++g) {
-      float mg = m[g];
-#pragma unroll
-      for (int u = 0; u < UN; ++u) mg = fmaxf(mg, s[u][g]);
-      const float mref = (mg == -INFINITY) ? 0.f : mg;
-      const float alpha = ex2_approx(m[g] - mref);
-      l[g] *= alpha;
-#pragma unroll
-      for (int e = 0; e < 8; ++e) acc[g][e] *= alpha;
-#pragma unroll
-      for (int u = 0; u < UN; ++u) {
-        const float pu = ex2_approx(s[u][g] - mref);
-        l[g] += pu;
-        float vf[8];
-        bf16x8_to_f32(vu[u], vf);
-#pragma unroll
-        for (int e = 0; e < 8; ++e) acc[g][e] = fmaf(pu, vf[e], acc[g][e]);
-      }
-      m[g] = mg;
-    }
+    if (nb < c1) load_v(nb);
   }
-  __shared__ float red_m[G][HW], red_l[G][HW];
-  __shared__ float red_o[G][HW][D];
+
+  // Merge the four warps of the CTA: per head, M = max m_w, then
+  // sum_w 2^(m_w - M) (O_w, l_w).
 #pragma unroll
-  for (int g = 0; g < G; ++g) {
+  for (int r = 0; r < 2; ++r) {
+    l[r] += __shfl_xor_sync(0xffffffffu, l[r], 1);
+    l[r] += __shfl_xor_sync(0xffffffffu, l[r], 2);
+  }
+  __shared__ float red_m[ROWS][WARPS], red_l[ROWS][WARPS];
+  __shared__ float red_o[ROWS][WARPS][D];
 #pragma unroll
-    for (int e = 0; e < 8; ++e) red_o[g][grp][sub * 8 + e] = acc[g][e];
-    if (sub == 0) {
-      red_m[g][grp] = m[g];
-      red_l[g][grp] = l[g];
+  for (int n = 0; n < NH; ++n) {
+#pragma unroll
+    for (int t = 0; t < MT; ++t) {
+      const int dlo = 64 * (t >> 3) + 8 * g + (t & 7);                  // entry t
+      const int dhi = 64 * ((t + MT) >> 3) + 8 * g + ((t + MT) & 7);    // entry t + D/16
+#pragma unroll
+      for (int j = 0; j < 2; ++j) {
+        red_o[8 * n + 2 * c + j][warp][dlo] = o[n][t][j];
+        red_o[8 * n + 2 * c + j][warp][dhi] = o[n][t][2 + j];
+      }
+    }
+    if (c == 0) {
+      red_m[8 * n + g][warp] = m[n];
+      red_l[8 * n + g][warp] = l[n];
     }
   }
   __syncthreads();
-  for (int t = threadIdx.x; t < D; t += THREADS) {
-#pragma unroll 1
-    for (int g = 0; g < G; ++g) {
-      float M = -INFINITY;
+  for (int idx = threadIdx.x; idx < qh * D; idx += THREADS) {
+    const int row = idx / D;
+    const int t = idx - row * D;
+    float M = -INFINITY;
 #pragma unroll
-      for (int k2 = 0; k2 < HW; ++k2) M = fmaxf(M, red_m[g][k2]);
-      float o = 0.f, lt = 0.f;
+    for (int w = 0; w < WARPS; ++w) M = fmaxf(M, red_m[row][w]);
+    float acc = 0.f, lt = 0.f;
 #pragma unroll
-      for (int k2 = 0; k2 < HW; ++k2) {
-        const float w = (red_m[g][k2] == -INFINITY) ? 0.f : ex2_approx(red_m[g][k2] - M);
-        o = fmaf(w, red_o[g][k2][t], o);
-        lt = fmaf(w, red_l[g][k2], lt);
-      }
-      float* out = part + ((bh0 + g) * S + split) * (D + 2);
-      out[t] = o;
-      if (t == 0) {
-        out[D] = M;
-        out[D + 1] = lt;
-      }
+    for (int w = 0; w < WARPS; ++w) {
+      const float wt = (red_m[row][w] == -INFINITY) ? 0.f : ex2_approx(red_m[row][w] - M);
+      acc = fmaf(wt, red_o[row][w][t], acc);
+      lt = fmaf(wt, red_l[row][w], lt);
+    }
+    float* out = part + ((static_cast<size_t>(b) * H + h0 + row) * S + split) * (D + 2);
+    out[t] = acc;
+    if (t == 0) {
+      out[D] = M;
+      out[D + 1] = lt;
     }
   }
 }
@@ -440,20 +573,24 @@ void launch_split(const __nv_bfloat16* qq, const __nv_bfloat16* kk, const __nv_b
                   const int* seqlens, float* part, int B, int H, int group, int Lmax, int S,
                   float sl2, const Pages& pg, cudaStream_t stream) {
   const int Hkv = H / group;
-  // groups of 2, 4 or 8 query heads share one pass over their cache head;
-  // other group sizes (and plain multi-head attention) use one CTA per head
-  if (group == 2)
-    fa_decode_group_split_kernel<D, 2, PAGED><<<dim3(S, Hkv, B), THREADS, 0, stream>>>(
-        qq, kk, vv, seqlens, part, H, Hkv, Lmax, S, sl2, pg);
-  else if (group == 4)
-    fa_decode_group_split_kernel<D, 4, PAGED><<<dim3(S, Hkv, B), THREADS, 0, stream>>>(
-        qq, kk, vv, seqlens, part, H, Hkv, Lmax, S, sl2, pg);
-  else if (group == 8)
-    fa_decode_group_split_kernel<D, 8, PAGED><<<dim3(S, Hkv, B), THREADS, 0, stream>>>(
-        qq, kk, vv, seqlens, part, H, Hkv, Lmax, S, sl2, pg);
-  else
+  // Grouped heads run on the tensor cores: one CTA per (split, run of qh
+  // query heads, batch) where qh is the whole group when it has at most 16
+  // heads, else 16 or 8 of them (the cache head is then read by several
+  // CTAs).  Plain multi-head attention and other group sizes use one CTA per
+  // query head.
+  const int qh = group <= 16 ? group : (group % 16 == 0 ? 16 : (group % 8 == 0 ? 8 : 0));
+  if (group > 1 && qh > 0) {
+    const dim3 grid(S, H / qh, B);
+    if (qh > 8)
+      fa_decode_group_mma_kernel<D, true, PAGED><<<grid, THREADS, 0, stream>>>(
+          qq, kk, vv, seqlens, part, H, Hkv, group, qh, Lmax, S, sl2, pg);
+    else
+      fa_decode_group_mma_kernel<D, false, PAGED><<<grid, THREADS, 0, stream>>>(
+          qq, kk, vv, seqlens, part, H, Hkv, group, qh, Lmax, S, sl2, pg);
+  } else {
     fa_decode_split_kernel<D, PAGED><<<dim3(S, H, B), THREADS, 0, stream>>>(
         qq, kk, vv, seqlens, part, H, group, Lmax, S, sl2, pg);
+  }
 }
 
 template <int D>

@@ -63,6 +63,26 @@ def test_gqa_decode(fa_mod, cuda_device, Hkv, d):
     check_lse(lse.cpu(), ref_l)
 
 
+@pytest.mark.parametrize("d", [128, 64])
+@pytest.mark.parametrize("H,Hkv", [(9, 3), (12, 2), (48, 3), (32, 1), (24, 1), (20, 1)],
+                         ids=lambda x: str(x))
+def test_gqa_decode_group_sizes(fa_mod, cuda_device, H, Hkv, d):
+    """Groups of 3, 6 and 16 query heads (one CTA per cached head, padded
+    head rows), 32 and 24 (16 or 8 heads per CTA, several CTAs per cached
+    head) and 20 (one CTA per query head); lengths inside and across 16-key
+    steps and 512-key splits."""
+    sl = [0, 1, 15, 16, 17, 100, 513, 1300]
+    q, kc, vc, sl = inputs.decode_inputs(len(sl), H, d, 0, 1300, seed=600 + H + Hkv + d,
+                                         Hkv=Hkv, seqlens=sl, Lcap=1300)
+    o, lse = fa_mod.decode(q.cuda(), kc.cuda(), vc.cuda(), sl.cuda())
+    torch.cuda.synchronize()
+    assert fa_mod.get_device_error() == 0
+    ref_o, ref_l = oracle.decode_forward(inputs.to_f64(q), inputs.to_f64(kc), inputs.to_f64(vc),
+                                         sl.tolist(), 1 / np.sqrt(d))
+    check_o(o.cpu(), ref_o)
+    check_lse(lse.cpu(), ref_l)
+
+
 def test_gqa_workload_forward_B4_H32_Hkv8_N2048_sampled(fa_mod, cuda_device):
     w = inputs.WORKLOADS["fwd_causal_gqa_B4_H32_Hkv8_N2048_d128"]
     q, k, v = inputs.workload_inputs(w)
