@@ -6,8 +6,10 @@
 One step is one call of the library on one batch of synthetic input of the
 chosen workload (default: the causal 2K-context prefill, B=4 H=16 N=2048
 d=128).  The timed region is exactly K steps bracketed by a barrier and a
-device synchronisation; each launch is timed with CUDA events on the stream it
-runs on.  Rank 0 prints one JSON line.  Under torchrun every rank runs the
+device synchronisation; each step is timed with CUDA events on the stream it
+runs on, and the library records a second pair of events around the step's
+dominant kernel (fa_set_timing_events), which gives the roofline's achieved
+rate.  Rank 0 prints one JSON line.  Under torchrun every rank runs the
 same workload on its own GPU (independent (batch, head) partitions, weak
 scaling, no data-path collective) and the time is the maximum over ranks.
 
@@ -305,6 +307,12 @@ def time_device(r, steps, warmup, world, dev):
         r.step()
     starts = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
     ends = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    # the library records these around its dominant kernel of each step
+    kstarts = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    kends = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    for ev in kstarts + kends:
+        ev.record(stream)  # creates the CUDA event behind it
+    torch.cuda.synchronize()
     sampler = ClockSampler(dev.index or 0)
     sampler.start()
     time.sleep(0.3)
@@ -313,15 +321,19 @@ def time_device(r, steps, warmup, world, dev):
     for i in range(steps):
         if r.flush is not None:
             r.flush.zero_()
+        r.fa.set_timing_events(kstarts[i], kends[i])
         starts[i].record(stream)
         r.step()
         ends[i].record(stream)
     barrier(world)
     wall = time.perf_counter() - t0
     clocks = sampler.stop()
+    r.fa.set_timing_events(None, None)
     per = [s.elapsed_time(e) * 1e-3 for s, e in zip(starts, ends)]
     mean_s = max_over_ranks(float(np.mean(per)), world, dev)
-    return mean_s, per, wall, clocks
+    kern = [s.elapsed_time(e) * 1e-3 for s, e in zip(kstarts, kends)]
+    kern_s = max_over_ranks(float(np.mean(kern)), world, dev)
+    return mean_s, per, wall, clocks, kern_s
 
 
 def time_e2e(r, steps, warmup, world, dev):
@@ -511,7 +523,7 @@ def main():
     fa.lib()
 
     r = Runner(w, dev)
-    mean_s, per, wall, clocks = time_device(r, args.steps, args.warmup, world, dev)
+    mean_s, per, wall, clocks, kern_s = time_device(r, args.steps, args.warmup, world, dev)
     if args.skip_baselines:
         e2e_s, h2d, d2h = float("nan"), 0, 0
     else:
@@ -521,7 +533,7 @@ def main():
     value = r.value(mean_s) * world
     if r.kind_bound == "tensor":
         peak = float(peaks["bf16_tflops"])
-        ach = r.work / mean_s / 1e12
+        ach = r.work / kern_s / 1e12
         traffic = profiled_traffic(r.kernel_key, r.w.kind)
         roof = {"bound": "tensor", "achieved": ach, "peak": peak, "unit": "TFLOP/s",
                 "frac": ach / peak, "traffic": traffic,
@@ -530,18 +542,19 @@ def main():
         # the 8-bit contraction's peak: the measured bf16 peak x the nominal
         # fp8 / bf16 ratio (4.5 / 2.25 PFLOP/s dense)
         peak = 2.0 * float(peaks["bf16_tflops"])
-        ach = r.work / mean_s / 1e12
+        ach = r.work / kern_s / 1e12
         traffic = profiled_traffic(r.kernel_key, r.w.kind)
         roof = {"bound": "tensor", "achieved": ach, "peak": peak, "unit": "TFLOP/s",
                 "frac": ach / peak, "traffic": traffic,
                 "peak_source": f"{peak_src} bf16_tflops (burst) x 2 (nominal e4m3 / bf16)"}
     else:
         peak = float(peaks["hbm_gbs"])
-        ach = r.work / mean_s / 1e9
+        ach = r.work / kern_s / 1e9
         traffic = profiled_traffic(r.kernel_key, r.w.kind)
         roof = {"bound": "hbm", "achieved": ach, "peak": peak, "unit": "GB/s",
                 "frac": ach / peak, "traffic": traffic,
                 "peak_source": f"{peak_src} hbm_gbs"}
+    roof["kernel_ms"] = kern_s * 1e3  # mean device time of the dominant kernel per step
     line = {
         "metric": METRIC, "value": value, "unit": r.unit, "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": mean_s * 1e3,

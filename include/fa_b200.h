@@ -54,6 +54,7 @@ extern "C" {
 #endif
 
 typedef struct CUstream_st* fa_stream_t; /* same type as cudaStream_t */
+typedef struct CUevent_st* fa_event_t;   /* same type as cudaEvent_t  */
 
 typedef enum {
     FA_OK = 0,
@@ -343,6 +344,18 @@ fa_status fa_decode_static(const void* q, const void* kcache, const void* vcache
                            const int* seqlens, void* o, float* lse,
                            int B, int H, int Lmax, int d, float scale,
                            fa_stream_t stream);
+
+/*
+ * Measurement hook.  With non-NULL events, every later call records `start`
+ * on its stream just before launching its dominant kernel and `stop` just
+ * after it: the attention kernel of fa_fwd*, the main kernel of fa_bwd*
+ * (not the D = rowsum(dO o O) preprocess or the dQ conversion), the split-KV
+ * kernel of fa_decode* (not the combine).  cudaEventElapsedTime(start, stop)
+ * then times that kernel alone.  The events are created and owned by the
+ * caller; pass NULL, NULL to turn the hook off.  Process-wide and not
+ * thread-safe.  Always returns FA_OK.
+ */
+fa_status fa_set_timing_events(fa_event_t start, fa_event_t stop);
 
 /*
  * Synchronises `stream`, then reads and clears the current device's error

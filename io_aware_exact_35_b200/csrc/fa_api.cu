@@ -9,6 +9,8 @@
 
 namespace fa {
 
+MainKernelEvents g_main_events = {nullptr, nullptr};
+
 namespace {
 
 using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
@@ -413,6 +415,12 @@ fa_status fa_decode_paged(const void* q, const void* kpages, const void* vpages,
   return launch_decode(q, kpages, vpages, seqlens, o, lse, B, H, Hkv, Lmax, d, scale,
                        static_cast<float*>(workspace), reinterpret_cast<cudaStream_t>(stream),
                        table, pages_per_seq, log2_page, num_pages);
+}
+
+fa_status fa_set_timing_events(fa_event_t start, fa_event_t stop) {
+  fa::g_main_events.start = reinterpret_cast<cudaEvent_t>(start);
+  fa::g_main_events.stop = reinterpret_cast<cudaEvent_t>(stop);
+  return FA_OK;
 }
 
 fa_status fa_get_device_error(fa_stream_t stream) {

@@ -702,8 +702,10 @@ fa_status launch_main(const CUtensorMap* maps, const Params& prm, int BH, cudaSt
     configured = true;
   }
   dim3 grid(prm.n_kt * BH);
+  main_kernel_begin(stream);
   kern<<<grid, NUM_THREADS, Smem<D>::ALLOC, stream>>>(maps[0], maps[1], maps[2], maps[3], maps[4],
                                                       maps[5], maps[6], prm);
+  main_kernel_end(stream);
   return cuda_status(cudaGetLastError());
 }
 

@@ -542,6 +542,28 @@ __global__ void __launch_bounds__(THREADS)
   }
 }
 
+// Block-wide max / sum over the D threads of a combine CTA (`red` holds one
+// value per warp; every thread gets the result).
+template <int D, bool MAX>
+__device__ __forceinline__ float block_reduce(float v, float* red) {
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) {
+    const float u = __shfl_xor_sync(0xffffffffu, v, off);
+    v = MAX ? fmaxf(v, u) : v + u;
+  }
+  __syncthreads();  // `red` may still be read from a previous reduction
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = v;
+  __syncthreads();
+  v = red[0];
+#pragma unroll
+  for (int w = 1; w < D / 32; ++w) v = MAX ? fmaxf(v, red[w]) : v + red[w];
+  return v;
+}
+
+// One CTA per (b, h), thread t owns output column t.  The split weights
+// w_s = 2^(m_s - M) are computed once per split (one thread each) and shared
+// through shared memory; the column sums then read the partials of up to D
+// splits with independent, coalesced loads.
 template <int D>
 __global__ void __launch_bounds__(D)
     fa_decode_combine_kernel(const float* __restrict__ part, const int* __restrict__ seqlens,
@@ -553,15 +575,36 @@ __global__ void __launch_bounds__(D)
   const int L = min(max(seqlens[b], 0), Lmax);
   const int n = (L + CHUNK - 1) / CHUNK;
   const float* base = part + static_cast<size_t>(bh) * S * (D + 2);
+  __shared__ float red[D / 32];
+  __shared__ float wts[D];
   float M = -INFINITY;
-  for (int s = 0; s < n; ++s) M = fmaxf(M, base[s * (D + 2) + D]);
-  float acc = 0.f, lt = 0.f;
-  for (int s = 0; s < n; ++s) {
-    const float ms = base[s * (D + 2) + D];
-    const float w = (ms == -INFINITY) ? 0.f : ex2_approx(ms - M);
-    acc = fmaf(w, base[s * (D + 2) + t], acc);
-    lt = fmaf(w, base[s * (D + 2) + D + 1], lt);
+  for (int s = t; s < n; s += D) M = fmaxf(M, base[static_cast<size_t>(s) * (D + 2) + D]);
+  M = block_reduce<D, true>(M, red);
+  float acc = 0.f, lpart = 0.f;
+  for (int s0 = 0; s0 < n; s0 += D) {
+    float w = 0.f;
+    if (s0 + t < n) {
+      const float* ps = base + static_cast<size_t>(s0 + t) * (D + 2);
+      const float ms = ps[D];
+      w = (ms == -INFINITY) ? 0.f : ex2_approx(ms - M);
+      lpart = fmaf(w, ps[D + 1], lpart);
+    }
+    __syncthreads();  // the previous chunk's weights have been used
+    wts[t] = w;
+    __syncthreads();
+    const int cnt = min(D, n - s0);
+    const float* ob = base + static_cast<size_t>(s0) * (D + 2) + t;
+    int k = 0;
+    for (; k + 8 <= cnt; k += 8) {
+      float v[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) v[u] = ob[static_cast<size_t>(k + u) * (D + 2)];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) acc = fmaf(wts[k + u], v[u], acc);
+    }
+    for (; k < cnt; ++k) acc = fmaf(wts[k], ob[static_cast<size_t>(k) * (D + 2)], acc);
   }
+  const float lt = block_reduce<D, false>(lpart, red);
   const float val = (lt > 0.f) ? acc / lt : 0.f;
   o[static_cast<size_t>(bh) * D + t] = __float2bfloat16_rn(val);
   if (t == 0 && lse != nullptr)
@@ -603,10 +646,12 @@ fa_status launch(const void* q, const void* kc, const void* vc, const int* seqle
     const auto* kk = static_cast<const __nv_bfloat16*>(kc);
     const auto* vv = static_cast<const __nv_bfloat16*>(vc);
     const float sl2 = scale * 1.4426950408889634f;
+    main_kernel_begin(stream);
     if (pg.table != nullptr)
       launch_split<D, true>(qq, kk, vv, seqlens, part, B, H, group, Lmax, S, sl2, pg, stream);
     else
       launch_split<D, false>(qq, kk, vv, seqlens, part, B, H, group, Lmax, S, sl2, pg, stream);
+    main_kernel_end(stream);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return FA_ERR_CUDA;
   }

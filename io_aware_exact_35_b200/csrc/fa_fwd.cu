@@ -666,7 +666,9 @@ fa_status launch(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap
     if (e != cudaSuccess) return FA_ERR_CUDA;
     configured = true;
   }
+  main_kernel_begin(stream);
   kern<<<grid_size, NUM_THREADS, SMEM, stream>>>(tq, tk, tv, prm);
+  main_kernel_end(stream);
   return cuda_status(cudaGetLastError());
 }
 

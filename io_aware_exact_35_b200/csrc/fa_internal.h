@@ -96,6 +96,21 @@ fa_status launch_decode(const void* q, const void* kc, const void* vc, const int
 
 inline fa_status cuda_status(cudaError_t e) { return e == cudaSuccess ? FA_OK : FA_ERR_CUDA; }
 
+// Caller-owned events recorded on the launch stream just before and just
+// after the dominant kernel of every call (fa_set_timing_events); null when
+// unset.
+struct MainKernelEvents {
+  cudaEvent_t start;
+  cudaEvent_t stop;
+};
+extern MainKernelEvents g_main_events;
+inline void main_kernel_begin(cudaStream_t s) {
+  if (g_main_events.start != nullptr) cudaEventRecord(g_main_events.start, s);
+}
+inline void main_kernel_end(cudaStream_t s) {
+  if (g_main_events.stop != nullptr) cudaEventRecord(g_main_events.stop, s);
+}
+
 inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
 }  // namespace fa

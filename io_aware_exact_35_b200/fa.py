@@ -51,6 +51,7 @@ SIGNATURES = {
                              _P]),
     "fa_get_device_error": (_I, [_P]),
     "fa_check_bounded_wait": (_I, [_P, _P]),
+    "fa_set_timing_events": (_I, [_P, _P]),
     "fa_status_string": (ctypes.c_char_p, [_I]),
     "fa_version": (_I, []),
 }
@@ -405,3 +406,16 @@ def check_bounded_wait(gave_up: torch.Tensor, stream=None) -> None:
     _req(gave_up, "gave_up", torch.int32, 1)
     _check("fa_check_bounded_wait", lib().fa_check_bounded_wait(gave_up.data_ptr(),
                                                                 _stream_ptr(stream)))
+
+
+def set_timing_events(start=None, stop=None) -> None:
+    """Record ``start`` / ``stop`` (torch.cuda.Event, already recorded once so
+    that their CUDA events exist) around the dominant kernel of every later
+    call; ``None, None`` turns this off."""
+    def handle(ev):
+        if ev is None:
+            return None
+        if not ev.cuda_event:
+            raise ValueError("record the event once before passing it")
+        return ev.cuda_event
+    _check("fa_set_timing_events", lib().fa_set_timing_events(handle(start), handle(stop)))
