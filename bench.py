@@ -290,7 +290,8 @@ class Runner:
 def barrier(world):
     if world > 1:
         torch.distributed.barrier()
-    torch.cuda.synchronize()
+    if torch.cuda.is_available():
+        torch.cuda.synchronize()
 
 
 def max_over_ranks(x, world, dev):
@@ -299,6 +300,13 @@ def max_over_ranks(x, world, dev):
     t = torch.tensor([x], dtype=torch.float64, device=dev)
     torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
     return float(t.item())
+
+
+def job_value(per_rank_value, world):
+    """Whole-job throughput: every rank processes the same units (weak
+    scaling) and the time is the maximum over ranks, so the job's rate is the
+    slowest rank's rate times the number of ranks."""
+    return per_rank_value * world
 
 
 def time_device(r, steps, warmup, world, dev):
@@ -547,7 +555,7 @@ def main():
         e2e_s, h2d, d2h = time_e2e(r, max(3, min(args.steps, 50)), 2, world, dev)
     err = fa.get_device_error()
     peaks, peak_src = load_peaks()
-    value = r.value(mean_s) * world
+    value = job_value(r.value(mean_s), world)
     if r.kind_bound == "tensor":
         peak = float(peaks["bf16_tflops"])
         ach = r.work / kern_s / 1e12
