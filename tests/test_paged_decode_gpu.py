@@ -47,6 +47,23 @@ def test_paged_decode_matches_oracle_and_contiguous(fa_mod, cuda_device, page_si
     check_lse(lse_p, lse_ref)
 
 
+@pytest.mark.parametrize("page_size", [1, 16, 128])
+@pytest.mark.parametrize("H,hkv,d", [(16, 1, 128), (12, 2, 64)])
+def test_paged_grouped_decode_large_groups(fa_mod, cuda_device, page_size, H, hkv, d):
+    """Groups of 16 and 6 query heads per cached head (all 16 head rows of the
+    tensor-core decode in use, and a padded group) over pages."""
+    B, Lcap = 3, 1300
+    seqlens = [17, 1300, 529]
+    (q, kc, vc, sl), (o_p, lse_p), (o_c, lse_c) = _decode_both(
+        fa_mod, B, H, hkv, d, seqlens, Lcap, page_size, seed=700 + page_size + H + d)
+    assert torch.equal(o_p, o_c), "paged and contiguous decode differ"
+    assert torch.equal(lse_p, lse_c)
+    o_ref, lse_ref = oracle.decode_forward(inputs.to_f64(q), inputs.to_f64(kc), inputs.to_f64(vc),
+                                           sl.tolist(), 1.0 / np.sqrt(d))
+    check_o(o_p, o_ref)
+    check_lse(lse_p, lse_ref)
+
+
 def test_paged_decode_workload_shape(fa_mod, cuda_device):
     """B16 H32 (and 8 shared K/V heads) d128, lengths U{4096..16384}, 16-row
     pages: bit-exact against the contiguous kernel on the full batch, and
