@@ -32,7 +32,13 @@ namespace fa {
 
 namespace dec {
 
-constexpr int CHUNK = 512;   // keys per split
+// Keys per split: CHUNK, or for the grouped kernel CHUNK_MAX when the
+// problem has enough splits of that length to fill the GPU several times
+// over (longer splits amortise each CTA's start and its merge, which pays
+// off with its two steps in flight per warp).  Workspaces are sized for
+// CHUNK.
+constexpr int CHUNK = 512;
+constexpr int CHUNK_MAX = 1024;
 constexpr int WARPS = 4;
 constexpr int THREADS = WARPS * 32;
 constexpr int UNROLL = 8;
@@ -310,8 +316,8 @@ __global__ void __launch_bounds__(THREADS)
                                const __nv_bfloat16* __restrict__ kc,
                                const __nv_bfloat16* __restrict__ vc,
                                const int* __restrict__ seqlens, float* __restrict__ part, int H,
-                               int Hkv, int group, int qh, int Lmax, int S, float scale_log2,
-                               const Pages pg) {
+                               int Hkv, int group, int qh, int Lmax, int S, int chunk,
+                               float scale_log2, const Pages pg) {
   constexpr int ROWS = HI ? 16 : 8;  // head rows that can be real
   constexpr int NH = HI ? 2 : 1;     // 8-head column tiles of O^T
   constexpr int KS = D / 16;         // k-steps of S = Q K^T
@@ -323,9 +329,9 @@ __global__ void __launch_bounds__(THREADS)
   const int b = blockIdx.z;
   const int hk = h0 / group;
   const int L = min(max(seqlens[b], 0), Lmax);
-  const int c0 = split * CHUNK;
+  const int c0 = split * chunk;
   if (c0 >= L) return;
-  const int c1 = min(c0 + CHUNK, L);
+  const int c1 = min(c0 + chunk, L);
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const int g = lane >> 2;
@@ -350,7 +356,7 @@ __global__ void __launch_bounds__(THREADS)
   const size_t bkv = static_cast<size_t>(b) * Hkv + hk;
   const __nv_bfloat16* kbase = kc + bkv * static_cast<size_t>(Lmax) * D;
   const __nv_bfloat16* vbase = vc + bkv * static_cast<size_t>(Lmax) * D;
-  __shared__ int spages[PAGED ? CHUNK : 1];
+  __shared__ int spages[PAGED ? CHUNK_MAX : 1];
   const auto rows = kv_rows<D, PAGED>(kc, vc, pg, spages, b, hk, Hkv, Lmax, c0, c1, 0);
   // element offset of a key's row; -1 when the key is masked (past the
   // prefix, or an invalid page entry)
@@ -360,34 +366,39 @@ __global__ void __launch_bounds__(THREADS)
     else return static_cast<long long>(key) * D;
   };
 
-  uint4 kr[2][NKL];  // K rows kb + g and kb + 8 + g
-  uint4 vr[4][NVL];  // V rows kb + 2c, kb + 2c + 1, kb + 8 + 2c, kb + 9 + 2c
-  bool klive[2];
-  auto load_k = [&](int kb) {
+  // DEPTH 16-key steps in flight per warp (two with 8 head rows; one with 16,
+  // whose accumulators leave no registers for a second): buffer bs holds the
+  // step being computed or a later one, and is refilled DEPTH steps ahead as
+  // soon as its K (after S) or V (after P V) has been used.
+  constexpr int DEPTH = HI ? 1 : 2;
+  uint4 kr[DEPTH][2][NKL];  // K rows kb + g and kb + 8 + g
+  uint4 vr[DEPTH][4][NVL];  // V rows kb + 2c, kb + 2c + 1, kb + 8 + 2c, kb + 9 + 2c
+  bool klive[DEPTH][2];
+  auto load_k = [&](const int bs, int kb) {
 #pragma unroll
     for (int t = 0; t < 2; ++t) {
       const long long off = row_off(kb + 8 * t + g);
-      klive[t] = off >= 0;
+      klive[bs][t] = off >= 0;
 #pragma unroll
       for (int i = 0; i < NKL; ++i)
-        kr[t][i] = off >= 0 ? ld_stream((PAGED ? rows.k : kbase) + off + 32 * i + 8 * c)
+        kr[bs][t][i] = off >= 0 ? ld_stream((PAGED ? rows.k : kbase) + off + 32 * i + 8 * c)
                             : make_uint4(0, 0, 0, 0);
     }
   };
-  auto load_v = [&](int kb) {
+  auto load_v = [&](const int bs, int kb) {
 #pragma unroll
     for (int r = 0; r < 4; ++r) {
       const long long off = row_off(kb + 8 * (r >> 1) + 2 * c + (r & 1));
 #pragma unroll
       for (int i = 0; i < NVL; ++i)
-        vr[r][i] = off >= 0 ? ld_stream((PAGED ? rows.v : vbase) + off + 64 * i + 8 * g)
+        vr[bs][r][i] = off >= 0 ? ld_stream((PAGED ? rows.v : vbase) + off + 64 * i + 8 * g)
                             : make_uint4(0, 0, 0, 0);
     }
   };
   // bf16 pair (key a, key b) at entry e of the lane's V list
-  auto vpair = [&](int ra, int rb, int e) -> uint32_t {
-    const uint4& ua = vr[ra][e >> 3];
-    const uint4& ub = vr[rb][e >> 3];
+  auto vpair = [&](const int bs, int ra, int rb, int e) -> uint32_t {
+    const uint4& ua = vr[bs][ra][e >> 3];
+    const uint4& ub = vr[bs][rb][e >> 3];
     const int w = (e & 7) >> 1;
     const uint32_t wa = w == 0 ? ua.x : w == 1 ? ua.y : w == 2 ? ua.z : ua.w;
     const uint32_t wb = w == 0 ? ub.x : w == 1 ? ub.y : w == 2 ? ub.z : ub.w;
@@ -402,13 +413,17 @@ __global__ void __launch_bounds__(THREADS)
   float m[2] = {-INFINITY, -INFINITY};  // heads g, g + 8 (log2 units, stale)
   float l[2] = {0.f, 0.f};              // this lane's share of their sums
 
-  int kb = c0 + 16 * warp;
-  if (kb < c1) {
-    load_k(kb);
-    load_v(kb);
+  const int kb0 = c0 + 16 * warp;  // this warp's steps: kb0, kb0 + 64, ...
+  if (kb0 < c1) {
+    load_k(0, kb0);
+    load_v(0, kb0);
   }
-  for (; kb < c1; kb += 16 * WARPS) {
-    const int nb = kb + 16 * WARPS;
+  if (DEPTH > 1 && kb0 + 16 * WARPS < c1) {
+    load_k(DEPTH - 1, kb0 + 16 * WARPS);
+    load_v(DEPTH - 1, kb0 + 16 * WARPS);
+  }
+  auto step = [&](const int bs, const int kb) {
+    const int nb = kb + DEPTH * 16 * WARPS;  // the next step held by buffer bs
     // S = Q K^T for keys kb .. kb+7 (half 0) and kb+8 .. kb+15 (half 1)
     float sc[2][4];
 #pragma unroll
@@ -416,7 +431,7 @@ __global__ void __launch_bounds__(THREADS)
       sc[t][0] = sc[t][1] = sc[t][2] = sc[t][3] = 0.f;
 #pragma unroll
       for (int s = 0; s < KS; ++s) {
-        const uint4& u = kr[t][s >> 1];
+        const uint4& u = kr[bs][t][s >> 1];
         mma_bf16_16816(sc[t], qa[s][0], qb[s][0], qa[s][1], qb[s][1], (s & 1) ? u.z : u.x,
                        (s & 1) ? u.w : u.y);
       }
@@ -428,8 +443,8 @@ __global__ void __launch_bounds__(THREADS)
     for (int t = 0; t < 2; ++t)
 #pragma unroll
       for (int j = 0; j < 2; ++j)
-        live[t][j] = __shfl_sync(0xffffffffu, static_cast<int>(klive[t]), 4 * (2 * c + j)) != 0;
-    if (nb < c1) load_k(nb);
+        live[t][j] = __shfl_sync(0xffffffffu, static_cast<int>(klive[bs][t]), 4 * (2 * c + j)) != 0;
+    if (nb < c1) load_k(bs, nb);
 
     uint32_t pb[2][2] = {{0u, 0u}, {0u, 0u}};  // P^T as the B operand: [head half][key half]
     float alpha[2] = {1.f, 1.f};
@@ -483,14 +498,18 @@ __global__ void __launch_bounds__(THREADS)
     // O^T += V^T P^T
 #pragma unroll
     for (int t = 0; t < MT; ++t) {
-      const uint32_t a0 = vpair(0, 1, t);
-      const uint32_t a1 = vpair(0, 1, t + MT);
-      const uint32_t a2 = vpair(2, 3, t);
-      const uint32_t a3 = vpair(2, 3, t + MT);
+      const uint32_t a0 = vpair(bs, 0, 1, t);
+      const uint32_t a1 = vpair(bs, 0, 1, t + MT);
+      const uint32_t a2 = vpair(bs, 2, 3, t);
+      const uint32_t a3 = vpair(bs, 2, 3, t + MT);
 #pragma unroll
       for (int n = 0; n < NH; ++n) mma_bf16_16816(o[n][t], a0, a1, a2, a3, pb[n][0], pb[n][1]);
     }
-    if (nb < c1) load_v(nb);
+    if (nb < c1) load_v(bs, nb);
+  };
+  for (int kb = kb0; kb < c1; kb += DEPTH * 16 * WARPS) {
+    step(0, kb);
+    if (DEPTH > 1 && kb + 16 * WARPS < c1) step(DEPTH - 1, kb + 16 * WARPS);
   }
 
   // Merge the four warps of the CTA: per head, M = max m_w, then
@@ -568,12 +587,12 @@ template <int D>
 __global__ void __launch_bounds__(D)
     fa_decode_combine_kernel(const float* __restrict__ part, const int* __restrict__ seqlens,
                              __nv_bfloat16* __restrict__ o, float* __restrict__ lse, int H,
-                             int Lmax, int S) {
+                             int Lmax, int S, int chunk) {
   const int bh = blockIdx.x;
   const int b = bh / H;
   const int t = threadIdx.x;
   const int L = min(max(seqlens[b], 0), Lmax);
-  const int n = (L + CHUNK - 1) / CHUNK;
+  const int n = (L + chunk - 1) / chunk;
   const float* base = part + static_cast<size_t>(bh) * S * (D + 2);
   __shared__ float red[D / 32];
   __shared__ float wts[D];
@@ -611,25 +630,29 @@ __global__ void __launch_bounds__(D)
     lse[bh] = (lt > 0.f) ? (M + lg2_approx(lt)) * 0.6931471805599453f : -INFINITY;
 }
 
+// Query heads per CTA of the grouped (tensor-core) kernel, 0 for the
+// per-head kernel: the whole group when it has at most 16 heads, else 16 or
+// 8 of them (the cache head is then read by several CTAs).  Plain multi-head
+// attention and other group sizes use one CTA per query head.
+inline int group_heads_per_cta(int group) {
+  if (group <= 1) return 0;
+  return group <= 16 ? group : (group % 16 == 0 ? 16 : (group % 8 == 0 ? 8 : 0));
+}
+
 template <int D, bool PAGED>
 void launch_split(const __nv_bfloat16* qq, const __nv_bfloat16* kk, const __nv_bfloat16* vv,
                   const int* seqlens, float* part, int B, int H, int group, int Lmax, int S,
-                  float sl2, const Pages& pg, cudaStream_t stream) {
+                  int chunk, float sl2, const Pages& pg, cudaStream_t stream) {
   const int Hkv = H / group;
-  // Grouped heads run on the tensor cores: one CTA per (split, run of qh
-  // query heads, batch) where qh is the whole group when it has at most 16
-  // heads, else 16 or 8 of them (the cache head is then read by several
-  // CTAs).  Plain multi-head attention and other group sizes use one CTA per
-  // query head.
-  const int qh = group <= 16 ? group : (group % 16 == 0 ? 16 : (group % 8 == 0 ? 8 : 0));
-  if (group > 1 && qh > 0) {
+  const int qh = group_heads_per_cta(group);
+  if (qh > 0) {
     const dim3 grid(S, H / qh, B);
     if (qh > 8)
       fa_decode_group_mma_kernel<D, true, PAGED><<<grid, THREADS, 0, stream>>>(
-          qq, kk, vv, seqlens, part, H, Hkv, group, qh, Lmax, S, sl2, pg);
+          qq, kk, vv, seqlens, part, H, Hkv, group, qh, Lmax, S, chunk, sl2, pg);
     else
       fa_decode_group_mma_kernel<D, false, PAGED><<<grid, THREADS, 0, stream>>>(
-          qq, kk, vv, seqlens, part, H, Hkv, group, qh, Lmax, S, sl2, pg);
+          qq, kk, vv, seqlens, part, H, Hkv, group, qh, Lmax, S, chunk, sl2, pg);
   } else {
     fa_decode_split_kernel<D, PAGED><<<dim3(S, H, B), THREADS, 0, stream>>>(
         qq, kk, vv, seqlens, part, H, group, Lmax, S, sl2, pg);
@@ -640,7 +663,19 @@ template <int D>
 fa_status launch(const void* q, const void* kc, const void* vc, const int* seqlens, void* o,
                  float* lse, int B, int H, int group, int Lmax, float scale, float* part,
                  const Pages& pg, cudaStream_t stream) {
-  const int S = decode_num_splits(Lmax);
+  // Split length: CHUNK for the per-head kernel; for the grouped kernel
+  // CHUNK_MAX once its splits alone give at least 8 CTAs per SM (by the
+  // cache capacity Lmax), else CHUNK.  The partials then take
+  // ceil(Lmax / chunk) <= ceil(Lmax / CHUNK) slots per head.
+  int dev = 0, sms = 148;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+    return FA_ERR_CUDA;
+  const int qh = group_heads_per_cta(group);
+  const long long rows = static_cast<long long>(B) * (qh > 0 ? H / qh : H);
+  const long long long_splits = (static_cast<long long>(Lmax) + CHUNK_MAX - 1) / CHUNK_MAX;
+  const int chunk = (qh > 0 && rows * long_splits >= 8LL * sms) ? CHUNK_MAX : CHUNK;
+  const int S = (Lmax + chunk - 1) / chunk;
   if (S > 0) {
     const auto* qq = static_cast<const __nv_bfloat16*>(q);
     const auto* kk = static_cast<const __nv_bfloat16*>(kc);
@@ -648,16 +683,18 @@ fa_status launch(const void* q, const void* kc, const void* vc, const int* seqle
     const float sl2 = scale * 1.4426950408889634f;
     main_kernel_begin(stream);
     if (pg.table != nullptr)
-      launch_split<D, true>(qq, kk, vv, seqlens, part, B, H, group, Lmax, S, sl2, pg, stream);
+      launch_split<D, true>(qq, kk, vv, seqlens, part, B, H, group, Lmax, S, chunk, sl2, pg,
+                            stream);
     else
-      launch_split<D, false>(qq, kk, vv, seqlens, part, B, H, group, Lmax, S, sl2, pg, stream);
+      launch_split<D, false>(qq, kk, vv, seqlens, part, B, H, group, Lmax, S, chunk, sl2, pg,
+                             stream);
     main_kernel_end(stream);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return FA_ERR_CUDA;
   }
   fa_decode_combine_kernel<D><<<B * H, D, 0, stream>>>(part, seqlens,
                                                        static_cast<__nv_bfloat16*>(o), lse, H,
-                                                       Lmax, S > 0 ? S : 1);
+                                                       Lmax, S > 0 ? S : 1, chunk);
   return cuda_status(cudaGetLastError());
 }
 
