@@ -37,6 +37,21 @@ def test_decode_edge_lengths(fa_mod, cuda_device, d):
     check_lse(lse, lse_ref)
 
 
+@pytest.mark.parametrize("d,H,Hkv,L", [(64, 2, 2, 40000), (128, 2, 2, 70000),
+                                         (128, 8, 1, 70000), (64, 16, 1, 33000)])
+def test_decode_more_splits_than_combine_threads(fa_mod, cuda_device, d, H, Hkv, L):
+    """Long contexts give more 512-key splits than the combine kernel has
+    threads (d), so its weights are gathered in several chunks; per head,
+    grouped (8 and 16 query heads per cached head) and not."""
+    seqlens = [L, L // 3 + 5]
+    q, kc, vc, sl = inputs.decode_inputs(2, H, d, 0, L, seed=900 + d + H + L % 97, Lcap=L,
+                                         seqlens=seqlens, Hkv=Hkv)
+    o, lse = _run(fa_mod, q, kc, vc, sl, 1 / np.sqrt(d))
+    o_ref, lse_ref = _oracle(q, kc, vc, sl, 1 / np.sqrt(d))
+    check_o(o, o_ref)
+    check_lse(lse, lse_ref)
+
+
 def test_decode_small_random(fa_mod, cuda_device):
     q, kc, vc, sl = inputs.decode_inputs(4, 8, 128, 100, 3000, seed=5)
     o, lse = _run(fa_mod, q, kc, vc, sl, 0.1)
