@@ -90,6 +90,14 @@ constexpr int NUM_THREADS = 320;
 constexpr int PANEL_BYTES = 128 * 128;   // 128 rows x 64 bf16 (one swizzle panel)
 constexpr uint32_t TMEM_COLS = 512;
 constexpr float RESCALE_THRESHOLD = 8.0f;  // log2 units
+
+// max(a, b, c) in one instruction (three-input max.f32, sm_100).  Inputs
+// here are finite or -inf, never NaN.
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
 #ifndef FA_FWD_EMU_PAIRS
 #define FA_FWD_EMU_PAIRS 0
 #endif
@@ -510,7 +518,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         const int key0 = j * BLOCK_N;
         const bool need_mask = (key0 + BLOCK_N > g.Nk) ||
                                (CAUSAL && key0 + BLOCK_N - 1 > q_row0 + g.off);
-        // four independent max chains (latency, not throughput, bounds this loop)
+        // four independent max chains (latency, not throughput, bounds this
+        // loop), each taking two new values per three-input max
         float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
         if (need_mask) {
           // last admissible key (below 0: none, the row stays at -inf)
@@ -519,12 +528,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           for (int c = 0; c < 128; ++c) {
             const float s = (key0 + c <= lim) ? __uint_as_float(sr[c]) : -INFINITY;
             sr[c] = __float_as_uint(s);
-            mx[c & 3] = fmaxf(mx[c & 3], s);
           }
-        } else {
-#pragma unroll
-          for (int c = 0; c < 128; ++c) mx[c & 3] = fmaxf(mx[c & 3], __uint_as_float(sr[c]));
         }
+#pragma unroll
+        for (int c = 0; c < 128; c += 2)
+          mx[(c >> 1) & 3] = fmax3(mx[(c >> 1) & 3], __uint_as_float(sr[c]), __uint_as_float(sr[c + 1]));
         // scale * log2(e) > 0, so the maximum of the scaled row is the scaled maximum
         const float m_new = fmaxf(m, fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])) * sl2);
         // true when m = -inf < m_new; false while the whole row is masked
