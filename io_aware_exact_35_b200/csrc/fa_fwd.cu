@@ -91,6 +91,21 @@ constexpr int PANEL_BYTES = 128 * 128;   // 128 rows x 64 bf16 (one swizzle pane
 constexpr uint32_t TMEM_COLS = 512;
 constexpr float RESCALE_THRESHOLD = 8.0f;  // log2 units
 
+// Two f32 values as one 64-bit operand of the packed f32x2 instructions
+// (sm_100), and (x0, x1) = (a0, a1) * b + c lane by lane.  ftz, as the
+// scalar FFMA it replaces under fast-math.
+__device__ __forceinline__ uint64_t pack_f32x2(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ void fma_f32x2(float& x0, float& x1, float a0, float a1, uint64_t b,
+                                          uint64_t c) {
+  uint64_t d;
+  asm("fma.rn.ftz.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(pack_f32x2(a0, a1)), "l"(b), "l"(c));
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(x0), "=f"(x1) : "l"(d));
+}
+
 // max(a, b, c) in one instruction (three-input max.f32, sm_100).  Inputs
 // here are finite or -inf, never NaN.
 __device__ __forceinline__ float fmax3(float a, float b, float c) {
@@ -545,14 +560,18 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         // Exponentials: MUFU ex2; in unmasked tiles EMU_PAIRS of every 4 pairs
         // may go to the FMA-pipe polynomial.  Masked tiles use ex2 only, so
         // excluded keys give exactly 0.
+        // x = s * scale * log2(e) - m for two keys per packed f32x2 FMA
+        const uint64_t sl2_2 = pack_f32x2(sl2, sl2);
+        const uint64_t negm_2 = pack_f32x2(-m_ref, -m_ref);
 #pragma unroll
         for (int c = 0; c < 128; c += 32) {
           uint32_t pk[16];
           float pf[32];
 #pragma unroll
           for (int e = 0; e < 32; e += 2) {
-            const float x0 = fmaf(__uint_as_float(sr[c + e]), sl2, -m_ref);
-            const float x1 = fmaf(__uint_as_float(sr[c + e + 1]), sl2, -m_ref);
+            float x0, x1;
+            fma_f32x2(x0, x1, __uint_as_float(sr[c + e]), __uint_as_float(sr[c + e + 1]), sl2_2,
+                      negm_2);
             float p0, p1;
             if (((e >> 1) & 3) >= 4 - EMU_PAIRS && !need_mask) {
               p0 = ex2_poly3(x0);
