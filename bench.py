@@ -152,6 +152,17 @@ class ClockSampler:
 
 
 # ----------------------------------------------------------------------------- workloads
+def decode_kernel_key(d, group, paged):
+    """Name of the split kernel the library launches for decode: the grouped
+    tensor-core kernel with qh query heads per CTA (the whole group up to 16
+    heads, else 16 or 8 of them), or the per-head kernel."""
+    qh = group if group <= 16 else (16 if group % 16 == 0 else (8 if group % 8 == 0 else 0))
+    suffix = ",paged" if paged else ""
+    if group > 1 and qh > 0:
+        return f"fa_decode_group_mma_kernel<{d},{qh}{suffix}>"
+    return f"fa_decode_split_kernel<{d}{suffix}>"
+
+
 def workload_config(w, parallelism):
     cfg = {"workload": w.name, "B": w.B, "H": w.H, "Hkv": w.kv_heads, "N": w.N or None,
            "d": w.d, "causal": w.causal, "parallelism": parallelism}
@@ -244,12 +255,7 @@ class Runner:
             self.work = decode_bytes(w, self.host[-1].tolist())
             self.unit, self.kind_bound = "GB/s", "hbm"
             self.launches_per_step = 2
-            group = w.H // w.kv_heads
-            paged = ",paged" if w.page else ""
-            # heads per CTA of the grouped (tensor-core) decode kernel
-            qh = group if group <= 16 else (16 if group % 16 == 0 else (8 if group % 8 == 0 else 0))
-            self.kernel_key = (f"fa_decode_group_mma_kernel<{w.d},{qh}{paged}>"
-                               if group > 1 and qh > 0 else f"fa_decode_split_kernel<{w.d}{paged}>")
+            self.kernel_key = decode_kernel_key(w.d, w.H // w.kv_heads, bool(w.page))
             self.out_host = torch.empty(self.o.shape, dtype=torch.bfloat16).pin_memory()
         self.working_set = sum(t.numel() * t.element_size() for t in self.dbuf)
         self.flush = None
