@@ -450,3 +450,105 @@ def test_unequal_lengths_backward_matches_autograd():
         dq, dk, dv, _ = A.attention_backward(q, k, v, do, True, 0.4)
         assert np.allclose(dq[..., keep.numpy(), :], tq.grad.numpy()[..., keep.numpy(), :], atol=1e-11)
         assert np.allclose(dk, tk.grad.numpy(), atol=1e-11) and np.allclose(dv, tv.grad.numpy(), atol=1e-11)
+
+
+# --------------------------------------------------------------------------
+# softmax_rows: the stable softmax of "Flash Attention: principle & practice",
+# section 2.1, pinned against torch's float64 softmax, closed forms and
+# invariants; planted mistakes in copies of it must each fail a pin.
+# --------------------------------------------------------------------------
+
+def pin_softmax_library(sm):
+    s = RNG.standard_normal((5, 13)) * 3.0
+    ref = torch.softmax(torch.from_numpy(s), dim=-1).numpy()
+    assert np.allclose(sm(s), ref, rtol=0, atol=1e-15), "must equal torch.softmax in float64"
+
+
+def pin_softmax_rows_sum_to_one(sm):
+    s = RNG.standard_normal((4, 3, 9)) * 5.0
+    p = sm(s)
+    assert p.shape == s.shape and np.all(p >= 0)
+    assert np.allclose(p.sum(-1), 1.0, atol=1e-14), "each row must sum to 1"
+
+
+def pin_softmax_logistic(sm):
+    # two entries a, b: p_0 = 1 / (1 + e^(b - a)) (closed form)
+    for a, b in ((0.3, -1.2), (2.0, 2.0), (-4.0, 1.5)):
+        p = sm(np.array([[a, b]]))
+        assert abs(p[0, 0] - 1.0 / (1.0 + math.exp(b - a))) < 1e-15
+        assert abs(p[0, 1] - 1.0 / (1.0 + math.exp(a - b))) < 1e-15
+
+
+def pin_softmax_large_scores(sm):
+    # stability: the maximum is subtracted first, so scores of 1000 and 999
+    # give the logistic weights instead of inf / inf
+    with np.errstate(all="ignore"):
+        p = sm(np.array([[1000.0, 999.0]]))
+    assert np.all(np.isfinite(p)) and abs(p[0, 0] - 1.0 / (1.0 + math.exp(-1.0))) < 1e-15
+
+
+def pin_softmax_masked(sm):
+    # -inf entries get probability 0; the rest is the softmax of the others;
+    # a row that is entirely -inf gives zeros
+    s = np.array([[0.5, -np.inf, 1.5, -np.inf], [-np.inf] * 4])
+    with np.errstate(all="ignore"):
+        p = sm(s)
+    assert np.all(np.isfinite(p))
+    assert p[0, 1] == 0.0 and p[0, 3] == 0.0
+    assert abs(p[0, 0] - 1.0 / (1.0 + math.exp(1.0))) < 1e-15
+    assert np.all(p[1] == 0.0), "a fully masked row must be all zeros"
+
+
+def pin_softmax_shift_invariant(sm):
+    s = RNG.standard_normal((3, 11))
+    assert np.allclose(sm(s), sm(s + 7.25), atol=1e-15), "adding a constant to a row changes nothing"
+    assert not np.allclose(sm(s), sm(2.0 * s), atol=1e-6), "scaling the scores must change P"
+
+
+SOFTMAX_PINS = [pin_softmax_library, pin_softmax_rows_sum_to_one, pin_softmax_logistic,
+                pin_softmax_large_scores, pin_softmax_masked, pin_softmax_shift_invariant]
+
+
+@pytest.mark.parametrize("pin", SOFTMAX_PINS, ids=lambda f: f.__name__)
+def test_softmax_rows_pins(pin):
+    pin(oracle.softmax_rows)
+
+
+def _mutant_softmax(kind):
+    def sm(s):
+        if kind == "no_max":
+            e = np.exp(s)
+            return e / e.sum(-1, keepdims=True)
+        if kind == "wrong_axis":
+            m = np.max(s, axis=0, keepdims=True)
+            e = np.exp(s - np.where(np.isfinite(m), m, 0.0))
+            tot = e.sum(0, keepdims=True)
+            return np.where(tot > 0, e / np.where(tot > 0, tot, 1.0), 0.0)
+        if kind == "sum_with_max":  # divides by the sum plus the (unshifted) max
+            m = np.max(s, axis=-1, keepdims=True)
+            e = np.exp(s - np.where(np.isfinite(m), m, 0.0))
+            return e / (e.sum(-1, keepdims=True) + 1.0)
+        if kind == "masked_row_nan":  # no guard for a fully masked row
+            m = np.max(s, axis=-1, keepdims=True)
+            e = np.exp(s - m)
+            return e / e.sum(-1, keepdims=True)
+        if kind == "exp_not_shifted_back":  # uses exp(s) / sum exp(s - m)
+            m = np.max(s, axis=-1, keepdims=True)
+            m0 = np.where(np.isfinite(m), m, 0.0)
+            return np.exp(s) / np.exp(s - m0).sum(-1, keepdims=True)
+        raise ValueError(kind)
+    return sm
+
+
+@pytest.mark.parametrize("kind", ["no_max", "wrong_axis", "sum_with_max", "masked_row_nan",
+                                  "exp_not_shifted_back"])
+def test_softmax_pins_reject_planted_mistakes(kind):
+    sm = _mutant_softmax(kind)
+    failures = 0
+    for pin in SOFTMAX_PINS:
+        try:
+            with np.errstate(all="ignore"):
+                pin(sm)
+        except (AssertionError, ValueError, FloatingPointError):
+            failures += 1
+    assert failures >= 1, f"no pin caught the planted softmax mistake {kind!r}"
