@@ -358,6 +358,30 @@ fa_status fa_decode_static(const void* q, const void* kcache, const void* vcache
 fa_status fa_set_timing_events(fa_event_t start, fa_event_t stop);
 
 /*
+ * Work-distribution override, for tests and measurements that must exercise
+ * one particular schedule.  It changes only how work is spread over the SMs,
+ * never a result.  Process-wide (it applies to every later call on every
+ * device and host thread) until changed again.
+ *   fwd_schedule : FA_SCHEDULE_AUTO lets the library choose per call;
+ *                  FA_SCHEDULE_GRID launches the forward with one CTA per
+ *                  256-row query tile; FA_SCHEDULE_PERSISTENT launches about
+ *                  one CTA per SM (at most a third of the tiles), each looping
+ *                  over several tiles.
+ *   bwd_order    : FA_SCHEDULE_AUTO; FA_SCHEDULE_GRID orders the backward's
+ *                  CTAs head-major (a head's key tiles adjacent);
+ *                  FA_SCHEDULE_PERSISTENT launches the longest causal key
+ *                  tiles of every head first.
+ * Returns FA_ERR_INVALID_ARG for any other value (nothing is changed), else
+ * FA_OK.
+ */
+enum {
+    FA_SCHEDULE_AUTO = 0,
+    FA_SCHEDULE_GRID = 1,
+    FA_SCHEDULE_PERSISTENT = 2
+};
+fa_status fa_set_schedule(int fwd_schedule, int bwd_order);
+
+/*
  * Synchronises `stream`, then reads and clears the current device's error
  * word.  Returns FA_OK, FA_ERR_TIMEOUT (a kernel gave up a bounded wait and
  * returned without finishing) or FA_ERR_CUDA (the synchronisation failed).

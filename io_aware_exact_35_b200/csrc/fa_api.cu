@@ -10,6 +10,8 @@
 namespace fa {
 
 MainKernelEvents g_main_events = {nullptr, nullptr};
+std::atomic<int> g_fwd_schedule{FA_SCHEDULE_AUTO};
+std::atomic<int> g_bwd_order{FA_SCHEDULE_AUTO};
 
 namespace {
 
@@ -420,6 +422,16 @@ fa_status fa_decode_paged(const void* q, const void* kpages, const void* vpages,
 fa_status fa_set_timing_events(fa_event_t start, fa_event_t stop) {
   fa::g_main_events.start = reinterpret_cast<cudaEvent_t>(start);
   fa::g_main_events.stop = reinterpret_cast<cudaEvent_t>(stop);
+  return FA_OK;
+}
+
+fa_status fa_set_schedule(int fwd_schedule, int bwd_order) {
+  auto valid = [](int v) {
+    return v == FA_SCHEDULE_AUTO || v == FA_SCHEDULE_GRID || v == FA_SCHEDULE_PERSISTENT;
+  };
+  if (!valid(fwd_schedule) || !valid(bwd_order)) return FA_ERR_INVALID_ARG;
+  fa::g_fwd_schedule.store(fwd_schedule, std::memory_order_relaxed);
+  fa::g_bwd_order.store(bwd_order, std::memory_order_relaxed);
   return FA_OK;
 }
 

@@ -694,13 +694,8 @@ __global__ void __launch_bounds__(256)
 template <int D, bool CAUSAL, bool VARLEN>
 fa_status launch_main(const CUtensorMap* maps, const Params& prm, int BH, cudaStream_t stream) {
   auto kern = fa_bwd_kernel<D, CAUSAL, VARLEN>;
-  static bool configured = false;
-  if (!configured) {
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Smem<D>::ALLOC) !=
-        cudaSuccess)
-      return FA_ERR_CUDA;
-    configured = true;
-  }
+  static SmemOptIn opt_in;  // one per instantiation of this kernel
+  if (const fa_status st = opt_in.ensure(kern, Smem<D>::ALLOC); st != FA_OK) return st;
   dim3 grid(prm.n_kt * BH);
   main_kernel_begin(stream);
   kern<<<grid, NUM_THREADS, Smem<D>::ALLOC, stream>>>(maps[0], maps[1], maps[2], maps[3], maps[4],
@@ -775,18 +770,14 @@ fa_status launch_bwd(const void* q, const void* k, const void* v, const void* o,
   {
     // Causal CTAs differ in length (later key tiles see fewer query tiles);
     // when there are only a few waves of them, launching the longest first
-    // shortens the tail.  FA_BWD_ORDER=head|lpt forces one.
-    static int mode = -1;
-    if (mode < 0) {
-      const char* env = std::getenv("FA_BWD_ORDER");
-      mode = (env && std::strcmp(env, "head") == 0) ? 1 : (env && std::strcmp(env, "lpt") == 0) ? 2 : 0;
-    }
+    // shortens the tail.  fa_set_schedule can force either order.
+    const int mode = g_bwd_order.load(std::memory_order_relaxed);
     int dev = 0, sms = 148;
     if (cudaGetDevice(&dev) != cudaSuccess ||
         cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
       return FA_ERR_CUDA;
     const long long ctas = static_cast<long long>(prm.n_kt) * BHkv;
-    prm.lpt_order = (mode == 2 || (mode == 0 && causal && ctas < 8LL * sms)) ? 1 : 0;
+    prm.lpt_order = (mode == FA_SCHEDULE_PERSISTENT || (mode == FA_SCHEDULE_AUTO && causal && ctas < 8LL * sms)) ? 1 : 0;
   }
   prm.scale_log2 = scale * bwd::LOG2E;
   prm.scale = scale;

@@ -687,12 +687,8 @@ fa_status launch(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap
                  const Params& prm, int grid_size, cudaStream_t stream) {
   auto kern = fa_fwd_kernel<D, CAUSAL, VARLEN, F8>;
   constexpr int SMEM = Smem<D, F8>::ALLOC;
-  static bool configured = false;  // per process; the attribute is per function
-  if (!configured) {
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM);
-    if (e != cudaSuccess) return FA_ERR_CUDA;
-    configured = true;
-  }
+  static SmemOptIn opt_in;  // one per instantiation of this kernel
+  if (const fa_status st = opt_in.ensure(kern, SMEM); st != FA_OK) return st;
   main_kernel_begin(stream);
   kern<<<grid_size, NUM_THREADS, SMEM, stream>>>(tq, tk, tv, prm);
   main_kernel_end(stream);
@@ -702,17 +698,9 @@ fa_status launch(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap
 // Work distribution.  Causal problems whose K and V all fit comfortably in L2
 // run persistently (one CTA per SM, longest tiles first, alternating rounds);
 // everything else runs one CTA per 256-row tile in head-major order, so the
-// resident CTAs share their heads' K/V tiles in L2.  FA_FWD_SCHEDULE=grid or
-// =persistent forces one of the two.
-int schedule_mode() {
-  static int mode = -1;
-  if (mode < 0) {
-    const char* env = std::getenv("FA_FWD_SCHEDULE");
-    mode = (env && std::strcmp(env, "grid") == 0) ? 1
-           : (env && std::strcmp(env, "persistent") == 0) ? 2 : 0;
-  }
-  return mode;
-}
+// resident CTAs share their heads' K/V tiles in L2.  fa_set_schedule can force
+// one of the two.
+int schedule_mode() { return g_fwd_schedule.load(std::memory_order_relaxed); }
 
 // Rows with no key at all (Nk = 0): O = 0, LSE = -inf, the same values the
 // main kernel gives a fully masked row.
@@ -758,10 +746,10 @@ fa_status launch_fwd(const void* q, const void* k, const void* v, void* o, float
   const int mode = fwd::schedule_mode();
   bool persistent = causal && items > sms && kv_bytes <= 96.0 * 1024 * 1024;
   int grid = persistent ? sms : static_cast<int>(items);
-  if (mode == 1) {
+  if (mode == FA_SCHEDULE_GRID) {
     persistent = false;
     grid = static_cast<int>(items);
-  } else if (mode == 2) {  // forced: about three items per CTA even for small problems
+  } else if (mode == FA_SCHEDULE_PERSISTENT) {  // forced: about three items per CTA even for small problems
     persistent = true;
     grid = static_cast<int>(std::min<long long>(sms, std::max<long long>(1, items / 3)));
   }
@@ -878,10 +866,10 @@ fa_status launch_fwd_fp8(const void* q, const void* k, const void* vt, void* o, 
   const int mode = fwd::schedule_mode();
   bool persistent = causal && items > sms && kv_bytes <= 96.0 * 1024 * 1024;
   int grid = persistent ? sms : static_cast<int>(items);
-  if (mode == 1) {
+  if (mode == FA_SCHEDULE_GRID) {
     persistent = false;
     grid = static_cast<int>(items);
-  } else if (mode == 2) {
+  } else if (mode == FA_SCHEDULE_PERSISTENT) {
     persistent = true;
     grid = static_cast<int>(std::min<long long>(sms, std::max<long long>(1, items / 3)));
   }

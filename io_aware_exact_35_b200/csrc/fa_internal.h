@@ -5,6 +5,7 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <atomic>
 #include <cstddef>
 #include <cstdint>
 
@@ -111,6 +112,32 @@ inline void main_kernel_end(cudaStream_t s) {
   if (g_main_events.stop != nullptr) cudaEventRecord(g_main_events.stop, s);
 }
 
+// Work-distribution overrides set by fa_set_schedule (FA_SCHEDULE_*).
+extern std::atomic<int> g_fwd_schedule;
+extern std::atomic<int> g_bwd_order;
+
 inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+// Dynamic shared memory above 48 KB must be enabled per kernel function and
+// per device (the attribute belongs to the function as loaded on each
+// device).  One flag per device records that the current device has been
+// configured; two threads racing here both set the same value, which is
+// harmless.  Devices beyond the table are configured on every call.
+struct SmemOptIn {
+  static constexpr int kMaxDevices = 64;
+  std::atomic<bool> done[kMaxDevices] = {};
+  template <typename Kern>
+  fa_status ensure(Kern kern, int bytes) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return FA_ERR_CUDA;
+    const bool cached = dev >= 0 && dev < kMaxDevices;
+    if (cached && done[dev].load(std::memory_order_acquire)) return FA_OK;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) !=
+        cudaSuccess)
+      return FA_ERR_CUDA;
+    if (cached) done[dev].store(true, std::memory_order_release);
+    return FA_OK;
+  }
+};
 
 }  // namespace fa

@@ -52,6 +52,7 @@ SIGNATURES = {
     "fa_get_device_error": (_I, [_P]),
     "fa_check_bounded_wait": (_I, [_P, _P]),
     "fa_set_timing_events": (_I, [_P, _P]),
+    "fa_set_schedule": (_I, [_I, _I]),
     "fa_status_string": (ctypes.c_char_p, [_I]),
     "fa_version": (_I, []),
 }
@@ -419,3 +420,15 @@ def set_timing_events(start=None, stop=None) -> None:
             raise ValueError("record the event once before passing it")
         return ev.cuda_event
     _check("fa_set_timing_events", lib().fa_set_timing_events(handle(start), handle(stop)))
+
+
+SCHEDULES = {"auto": 0, "grid": 1, "persistent": 2}
+
+
+def set_schedule(fwd: str = "auto", bwd: str = "auto") -> None:
+    """Force the work distribution of later calls (process-wide; results do
+    not change): forward ``"grid"`` (one CTA per 256-row query tile) or
+    ``"persistent"`` (CTAs looping over tiles); backward ``"grid"``
+    (head-major) or ``"persistent"`` (longest key tiles first); ``"auto"``
+    restores the library's own choice."""
+    _check("fa_set_schedule", lib().fa_set_schedule(SCHEDULES[fwd], SCHEDULES[bwd]))

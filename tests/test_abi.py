@@ -137,3 +137,15 @@ def test_bounded_wait_check_validates_pointer(fa_mod):
     INVALID = 1
     assert lib.fa_check_bounded_wait(None, None) == INVALID
     assert lib.fa_check_bounded_wait((1 << 20) + 2, None) == INVALID
+
+
+def test_set_schedule_validates_and_resets(fa_mod):
+    lib = fa_mod.lib()
+    assert lib.fa_set_schedule(3, 0) == 1 and lib.fa_set_schedule(0, -1) == 1
+    for f in (0, 1, 2):
+        for b in (0, 1, 2):
+            assert lib.fa_set_schedule(f, b) == 0
+    fa_mod.set_schedule("grid", "persistent")
+    fa_mod.set_schedule()  # back to the library's own choice
+    with pytest.raises(KeyError):
+        fa_mod.set_schedule("sideways")

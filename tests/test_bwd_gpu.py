@@ -48,9 +48,32 @@ def test_bwd_workload_causal_B2_H16_N8192_d128_sampled_heads(fa_mod, cuda_device
     dq, dk, dv = _run(fa_mod, q, k, v, do, w.causal, w.scale)
     for t in (dq, dk, dv):
         assert torch.isfinite(t.float()).all()
-    for (b, h) in ((0, 0), (1, 15), (1, 6)):
+    # eight (batch, head) pairs over both batches and the head-major launch order
+    for (b, h) in ((0, 0), (0, 5), (0, 10), (0, 15), (1, 0), (1, 6), (1, 11), (1, 15)):
         rq, rk, rv, _ = oracle.attention_backward(
             *(inputs.to_f64(t[b, h]) for t in (q, k, v, do)), True, w.scale)
         check_grad(dq[b, h], rq, f"dQ[{b},{h}]")
         check_grad(dk[b, h], rk, f"dK[{b},{h}]")
         check_grad(dv[b, h], rv, f"dV[{b},{h}]")
+
+
+@pytest.mark.parametrize("order", ["grid", "persistent"])
+def test_bwd_both_cta_orders(fa_mod, cuda_device, order):
+    """The backward launches its key-tile CTAs head-major or longest first;
+    both orders must give the oracle's gradients."""
+    fa_mod.set_schedule(bwd=order)
+    try:
+        for (B, H, N, d, causal) in ((2, 3, 700, 128, True), (1, 4, 1100, 64, True),
+                                     (2, 2, 513, 128, False)):
+            q, k, v, do = inputs.bwd_inputs(B, H, N, d, seed=3000 + N + d)
+            scale = 1.0 / np.sqrt(d)
+            dq, dk, dv = _run(fa_mod, q, k, v, do, causal, scale)
+            for b in range(B):
+                for h in range(H):
+                    rq, rk, rv, _ = oracle.attention_backward(
+                        *(inputs.to_f64(t[b, h]) for t in (q, k, v, do)), causal, scale)
+                    check_grad(dq[b, h], rq, f"dQ[{b},{h}]")
+                    check_grad(dk[b, h], rk, f"dK[{b},{h}]")
+                    check_grad(dv[b, h], rv, f"dV[{b},{h}]")
+    finally:
+        fa_mod.set_schedule()

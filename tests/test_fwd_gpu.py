@@ -105,40 +105,29 @@ def test_fwd_output_buffers_and_streams(fa_mod, cuda_device):
     check_o(o.cpu(), o_ref)
 
 
-_SCHEDULE_SCRIPT = r"""
-import sys, numpy as np, torch
-sys.path.insert(0, {root!r})
-import oracle
-from io_aware_exact_35_b200 import fa, inputs
-from tests._parity import check_o, check_lse
 # (B, H, Hkv, Nq, Nk, d, causal); with Nq > Nk many work items have halves
 # that see the same number of key tiles, with Nq < Nk none do
-for (B, H, Hkv, N, Nk, d, causal) in [(2, 3, 3, 1000, 1000, 128, True), (1, 5, 5, 777, 777, 64, True),
-                                      (3, 2, 2, 513, 513, 128, False), (2, 4, 4, 2048, 2048, 128, True),
-                                      (1, 4, 2, 3000, 1000, 128, True), (2, 2, 1, 1500, 4000, 64, True),
-                                      (1, 3, 3, 2900, 2900, 128, True)]:
-    q, k, v = inputs.fwd_inputs(B, H, N, d, seed=N + d, Hkv=Hkv, Nk=Nk)
-    o, lse = fa.fwd(q.cuda(), k.cuda(), v.cuda(), causal=causal)
-    torch.cuda.synchronize()
-    assert fa.get_device_error() == 0
-    ref_o, ref_l = oracle.attention_forward(*(inputs.to_f64(t) for t in (q, k, v)), causal, 1 / np.sqrt(d))
-    check_o(o.cpu(), ref_o)
-    check_lse(lse.cpu(), ref_l)
-print("ok")
-"""
+_SCHEDULE_CASES = [(2, 3, 3, 1000, 1000, 128, True), (1, 5, 5, 777, 777, 64, True),
+                   (3, 2, 2, 513, 513, 128, False), (2, 4, 4, 2048, 2048, 128, True),
+                   (1, 4, 2, 3000, 1000, 128, True), (2, 2, 1, 1500, 4000, 64, True),
+                   (1, 3, 3, 2900, 2900, 128, True)]
 
 
 @pytest.mark.parametrize("schedule", ["persistent", "grid"])
 def test_fwd_both_work_schedules(fa_mod, cuda_device, schedule):
     """The forward runs either one CTA per 256-row tile or persistently (each
-    CTA loops over several tiles, barrier phases carried across them, the
-    two query-tile streams running into the next tile independently); both
+    CTA loops over several tiles, barrier phases carried across them); both
     must give the oracle's result, also for unequal query / key lengths."""
-    import os
-    import subprocess
-    import sys
-    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
-    env = dict(os.environ, FA_FWD_SCHEDULE=schedule)
-    r = subprocess.run([sys.executable, "-c", _SCHEDULE_SCRIPT.format(root=root)], env=env,
-                       capture_output=True, text=True, timeout=600, cwd=root)
-    assert r.returncode == 0 and r.stdout.strip().endswith("ok"), r.stdout + r.stderr
+    fa_mod.set_schedule(fwd=schedule)
+    try:
+        for (B, H, Hkv, N, Nk, d, causal) in _SCHEDULE_CASES:
+            q, k, v = inputs.fwd_inputs(B, H, N, d, seed=N + d, Hkv=Hkv, Nk=Nk)
+            o, lse = fa_mod.fwd(q.cuda(), k.cuda(), v.cuda(), causal=causal)
+            torch.cuda.synchronize()
+            assert fa_mod.get_device_error() == 0
+            ref_o, ref_l = oracle.attention_forward(*(inputs.to_f64(t) for t in (q, k, v)),
+                                                    causal, 1 / np.sqrt(d))
+            check_o(o.cpu(), ref_o)
+            check_lse(lse.cpu(), ref_l)
+    finally:
+        fa_mod.set_schedule()
