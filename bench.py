@@ -205,7 +205,6 @@ class Runner:
             self.unit, self.kind_bound = "TFLOP/s", "tensor"
             self.launches_per_step = 1
             self.kernel_key = f"fa_fwd_kernel<{w.d},{str(w.causal).lower()}>"
-            self.out_host = torch.empty(self.o.shape, dtype=torch.bfloat16).pin_memory()
         elif w.kind == "fwd_fp8":
             q8 = self.host[0]
             self.o = torch.empty(q8.shape, dtype=torch.bfloat16, device=dev)
@@ -214,7 +213,6 @@ class Runner:
             self.unit, self.kind_bound = "TFLOP/s", "tensor_fp8"
             self.launches_per_step = 1
             self.kernel_key = f"fa_fwd_kernel<{w.d},{str(w.causal).lower()},e4m3>"
-            self.out_host = torch.empty(self.o.shape, dtype=torch.bfloat16).pin_memory()
         elif w.kind == "fwd_varlen":
             q, k, v, cu_q, cu_k = self.dbuf
             lens = (self.host[3][1:] - self.host[3][:-1]).tolist()
@@ -225,10 +223,12 @@ class Runner:
             self.unit, self.kind_bound = "TFLOP/s", "tensor"
             self.launches_per_step = 1
             self.kernel_key = f"fa_fwd_kernel<{w.d},{str(w.causal).lower()},varlen>"
-            self.out_host = torch.empty(self.o.shape, dtype=torch.bfloat16).pin_memory()
         elif w.kind == "bwd":
             q, k, v, do = self.dbuf
             self.o, self.lse = fa.fwd(q, k, v, causal=w.causal, scale=w.scale)
+            # O and LSE are inputs of the backward too (from the forward pass)
+            self.host = list(self.host) + [self.o.cpu(), self.lse.cpu()]
+            self.dbuf = list(self.dbuf) + [self.o, self.lse]
             self.dq, self.dk, self.dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
             self.ws = torch.empty(fa.bwd_workspace_size(w.B, w.H, w.N, w.d), dtype=torch.uint8,
                                   device=dev)
@@ -236,7 +236,6 @@ class Runner:
             self.unit, self.kind_bound = "TFLOP/s", "tensor"
             self.launches_per_step = 3
             self.kernel_key = f"fa_bwd_kernel<{w.d},{str(w.causal).lower()}>"
-            self.out_host = torch.empty(self.dq.shape, dtype=torch.bfloat16).pin_memory()
         else:
             q, kc, vc, sl = self.dbuf
             lcap = kc.shape[2]
@@ -256,38 +255,43 @@ class Runner:
             self.unit, self.kind_bound = "GB/s", "hbm"
             self.launches_per_step = 2
             self.kernel_key = decode_kernel_key(w.d, w.H // w.kv_heads, bool(w.page))
-            self.out_host = torch.empty(self.o.shape, dtype=torch.bfloat16).pin_memory()
+        # every output of a step, copied back to pinned host memory by the
+        # end-to-end measurement
+        outs = self.outputs()
+        self.out_host = [torch.empty(t.shape, dtype=t.dtype).pin_memory() for t in outs]
         self.working_set = sum(t.numel() * t.element_size() for t in self.dbuf)
         self.flush = None
         if self.working_set < 2 * L2_BYTES:
             self.flush = torch.empty(2 * L2_BYTES, dtype=torch.uint8, device=dev)
+
+    def outputs(self):
+        """The tensors one step writes (all of them are results)."""
+        if self.w.kind == "bwd":
+            return [self.dq, self.dk, self.dv]
+        return [self.o, self.lse]
 
     def step(self, bufs=None):
         w, fa = self.w, self.fa
         b = bufs if bufs is not None else self.dbuf
         if w.kind == "fwd":
             fa.fwd(b[0], b[1], b[2], causal=w.causal, scale=w.scale, out=self.o, lse=self.lse)
-            return self.o
-        if w.kind == "fwd_fp8":
+        elif w.kind == "fwd_fp8":
             qs, ks, vs = self.fp8_scales
             fa.fwd_fp8(b[0], b[1], b[2], qs, ks, vs, causal=w.causal, scale=w.scale, out=self.o,
                        lse=self.lse)
-            return self.o
-        if w.kind == "fwd_varlen":
+        elif w.kind == "fwd_varlen":
             fa.fwd_varlen(b[0], b[1], b[2], b[3], b[4], self.max_len, causal=w.causal,
                           scale=w.scale, out=self.o, lse=self.lse)
-            return self.o
-        if w.kind == "bwd":
-            fa.bwd(b[0], b[1], b[2], self.o, b[3], self.lse, causal=w.causal, scale=w.scale,
+        elif w.kind == "bwd":
+            fa.bwd(b[0], b[1], b[2], b[4], b[3], b[5], causal=w.causal, scale=w.scale,
                    dq=self.dq, dk=self.dk, dv=self.dv, workspace=self.ws)
-            return self.dq
-        if w.page:
+        elif w.page:
             fa.decode_paged(b[0], b[1], b[2], b[3], b[4], scale=w.scale, out=self.o,
                             lse=self.lse, workspace=self.ws)
-            return self.o
-        fa.decode(b[0], b[1], b[2], b[3], scale=w.scale, out=self.o, lse=self.lse,
-                  workspace=self.ws)
-        return self.o
+        else:
+            fa.decode(b[0], b[1], b[2], b[3], scale=w.scale, out=self.o, lse=self.lse,
+                      workspace=self.ws)
+        return self.outputs()
 
     def value(self, seconds):
         return self.work / seconds / 1e12 if self.unit == "TFLOP/s" else self.work / seconds / 1e9
@@ -373,13 +377,13 @@ def time_e2e(r, steps, warmup, world, dev):
     host = [t.pin_memory() for t in r.host]
     dbufs = [torch.empty_like(t, device=dev) for t in r.host]
     h2d = sum(t.numel() * t.element_size() for t in host)
-    d2h = r.out_host.numel() * r.out_host.element_size()
+    d2h = sum(t.numel() * t.element_size() for t in r.out_host)
 
     def one():
         for hb, db in zip(host, dbufs):
             db.copy_(hb, non_blocking=True)
-        out = r.step(dbufs)
-        r.out_host.copy_(out, non_blocking=True)
+        for out, oh in zip(r.step(dbufs), r.out_host):
+            oh.copy_(out, non_blocking=True)
 
     for _ in range(max(1, warmup)):
         one()
@@ -435,7 +439,25 @@ def run_reference(args, w, total_budget=150.0, emit=True):
             return dt, 4.0 * keys * w.d, 1.0
         unit = "TFLOP/s"
         scale_out = 1e12
-    elif w.kind in ("fwd", "bwd", "fwd_fp8"):
+    elif w.kind == "bwd":
+        # the oracle's backward of whole (batch, head) problems: it recomputes
+        # S and P from q, k, v and forms dV, dP, dS, dQ, dK in fp64
+        q, k, v, do = host[:4]
+        heads = [(b, h) for b in range(w.B) for h in range(w.H)]
+        group = w.H // w.kv_heads
+        sample = "one whole (batch, head) backward (all N query and key rows) per step"
+
+        def step(i):
+            b, h = heads[i % len(heads)]
+            args_ = (f64(q[b, h]), f64(k[b, h // group]), f64(v[b, h // group]), f64(do[b, h]))
+            t = time.perf_counter()
+            oracle.attention_backward(*args_, w.causal, w.scale)
+            dt = time.perf_counter() - t
+            f = 4.0 * w.N * w.N * w.d * (0.5 if w.causal else 1.0)
+            return dt, 2.5 * f, 1.0
+        unit = "TFLOP/s"
+        scale_out = 1e12
+    elif w.kind in ("fwd", "fwd_fp8"):
         if w.kind == "fwd_fp8":  # the oracle takes the real (descaled) values
             q8, k8, vt8, (qs, ks, vs) = host
             q = torch.from_numpy(inputs.fp8_to_f64(q8, qs))
@@ -452,7 +474,6 @@ def run_reference(args, w, total_budget=150.0, emit=True):
         per_row = (time.perf_counter() - t0) / min(64, w.N)
         rows_per_step = int(max(1, min(w.N, budget / max(per_row, 1e-9))))
         sample = f"{rows_per_step} query rows of one (batch, head) per step, rows drawn uniformly"
-        mult = 3.5 if w.kind == "bwd" else 1.0  # bwd oracle is not timed; fwd rows scaled
 
         group = w.H // w.kv_heads
 
@@ -464,7 +485,7 @@ def run_reference(args, w, total_budget=150.0, emit=True):
             oracle.attention_forward_rows(qh, kh, vh, w.causal, w.scale, rows)
             dt = time.perf_counter() - t
             keys = (rows + 1).sum() if w.causal else rows.size * w.N
-            return dt, 4.0 * keys * w.d * (2.5 if w.kind == "bwd" else 1.0), mult
+            return dt, 4.0 * keys * w.d, 1.0
         unit = "TFLOP/s"
         scale_out = 1e12
     else:
@@ -497,7 +518,7 @@ def run_reference(args, w, total_budget=150.0, emit=True):
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": workload_config(w, "cpu"),
         "cpu_baseline": {"value": value, "unit": unit, "cores": cores, "kind": "oracle",
-                         "sample": sample + (" (bwd: forward-row oracle time x3.5)" if w.kind == "bwd" else "")},
+                         "sample": sample},
         "e2e": {"value": value, "unit": unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     if emit:
@@ -521,6 +542,8 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--skip-baselines", action="store_true",
                     help="profiling runs: skip the end-to-end and CPU-oracle legs")
+    ap.add_argument("--no-extra", action="store_true",
+                    help="report only the chosen workload (no `workloads` object)")
     ap.add_argument("--B", type=int, default=None,
                     help="profiling runs: override the workload's batch size")
     args = ap.parse_args()
@@ -554,54 +577,39 @@ def main():
     fa.lib()
 
     r = Runner(w, dev)
-    mean_s, per, wall, clocks, kern_s = time_device(r, args.steps, args.warmup, world, dev)
-    if args.skip_baselines:
-        e2e_s, h2d, d2h = float("nan"), 0, 0
-    else:
-        e2e_s, h2d, d2h = time_e2e(r, max(3, min(args.steps, 50)), 2, world, dev)
+    res = measure(r, args.steps, args.warmup, world, dev, e2e=not args.skip_baselines)
     err = fa.get_device_error()
-    peaks, peak_src = load_peaks()
-    value = job_value(r.value(mean_s), world)
-    if r.kind_bound == "tensor":
-        peak = float(peaks["bf16_tflops"])
-        ach = r.work / kern_s / 1e12
-        traffic = profiled_traffic(r.kernel_key, r.w.kind, r.w.name)
-        roof = {"bound": "tensor", "achieved": ach, "peak": peak, "unit": "TFLOP/s",
-                "frac": ach / peak, "traffic": traffic,
-                "peak_source": f"{peak_src} bf16_tflops (burst)"}
-    elif r.kind_bound == "tensor_fp8":
-        # the 8-bit contraction's peak: the measured bf16 peak x the nominal
-        # fp8 / bf16 ratio (4.5 / 2.25 PFLOP/s dense)
-        peak = 2.0 * float(peaks["bf16_tflops"])
-        ach = r.work / kern_s / 1e12
-        traffic = profiled_traffic(r.kernel_key, r.w.kind, r.w.name)
-        roof = {"bound": "tensor", "achieved": ach, "peak": peak, "unit": "TFLOP/s",
-                "frac": ach / peak, "traffic": traffic,
-                "peak_source": f"{peak_src} bf16_tflops (burst) x 2 (nominal e4m3 / bf16)"}
-    else:
-        peak = float(peaks["hbm_gbs"])
-        ach = r.work / kern_s / 1e9
-        traffic = profiled_traffic(r.kernel_key, r.w.kind, r.w.name)
-        roof = {"bound": "hbm", "achieved": ach, "peak": peak, "unit": "GB/s",
-                "frac": ach / peak, "traffic": traffic,
-                "peak_source": f"{peak_src} hbm_gbs"}
-    roof["kernel_ms"] = kern_s * 1e3  # mean device time of the dominant kernel per step
     line = {
-        "metric": METRIC, "value": value, "unit": r.unit, "n_gpus": world,
-        "steps": args.steps, "warmup": args.warmup, "ms_per_step": mean_s * 1e3,
+        "metric": METRIC, "value": res["value"], "unit": r.unit, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": res["ms_per_step"],
+        "ms_per_step_median": res["ms_per_step_median"],
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "e4m3" if w.kind == "fwd_fp8" else "bf16", "data": "synthetic",
         "config": dict(workload_config(w, f"replicas{world}" if world > 1 else "single"),
-                       l2="flushed (256 MB write) before every step" if r.flush is not None
-                       else "inputs larger than L2"),
-        "roofline": roof,
-        "e2e": {"value": r.value(e2e_s) * world, "unit": r.unit, "h2d_bytes_per_step": h2d,
-                "d2h_bytes_per_step": d2h},
+                       l2=res["l2"]),
+        "roofline": res["roofline"],
+        "e2e": res["e2e"],
         "gpu_launches": args.steps * r.launches_per_step,
-        "clocks": clocks,
+        "clocks": res["clocks"],
         "device_error": err,
-        "wall_s_timed_region": wall,
+        "wall_s_timed_region": res["wall_s"],
     }
+    del r
+    if not args.skip_baselines and not args.no_extra and w.name == DEFAULT_WORKLOAD:
+        # the other full-size configurations, each timed the same way (device
+        # time of whole steps, dominant kernel alone for the roofline)
+        line["workloads"] = {}
+        for name, steps in EXTRA_WORKLOADS:
+            rx = Runner(inputs.WORKLOADS[name], dev)
+            rr = measure(rx, steps, args.warmup, world, dev, e2e=False)
+            rr["device_error"] = fa.get_device_error()
+            rr.pop("e2e", None)
+            rr["steps"] = steps
+            rr["warmup"] = args.warmup
+            rr["unit"] = rx.unit
+            line["workloads"][name] = rr
+            del rx
+            torch.cuda.empty_cache()
     if rank == 0 and world == 1 and not args.skip_baselines:
         try:
             line["cpu_baseline"] = cpu_baseline(w)
@@ -611,6 +619,57 @@ def main():
         torch.distributed.destroy_process_group()
     if rank == 0:
         print(json.dumps(line), flush=True)
+
+
+# The other full-size configurations reported beside the default one, with
+# their timed steps: the 32K-context forward, the backward, the decode.
+EXTRA_WORKLOADS = (("fwd_causal_B1_H32_N32768_d128", 10),
+                   ("bwd_causal_B2_H16_N8192_d128", 30),
+                   ("decode_B16_H32_d128_L4096-16384", 100))
+NOMINAL = {"tensor": 2250.0, "tensor_fp8": 4500.0, "hbm": 8000.0}
+
+
+def measure(r, steps, warmup, world, dev, e2e=True):
+    """Times one workload: the step rate (`value`), the dominant kernel's
+    roofline, clocks and (optionally) the end-to-end rate."""
+    mean_s, per, wall, clocks, kern_s = time_device(r, steps, warmup, world, dev)
+    if e2e:
+        e2e_s, h2d, d2h = time_e2e(r, max(3, min(steps, 50)), 2, world, dev)
+    else:
+        e2e_s, h2d, d2h = float("nan"), 0, 0
+    peaks, peak_src = load_peaks()
+    if r.kind_bound == "tensor":
+        peak = float(peaks["bf16_tflops"])
+        src = f"{peak_src} bf16_tflops (burst)"
+    elif r.kind_bound == "tensor_fp8":
+        # the 8-bit contraction's peak: the measured bf16 peak x the nominal
+        # fp8 / bf16 ratio (4.5 / 2.25 PFLOP/s dense)
+        peak = 2.0 * float(peaks["bf16_tflops"])
+        src = f"{peak_src} bf16_tflops (burst) x 2 (nominal e4m3 / bf16)"
+    else:
+        peak = float(peaks["hbm_gbs"])
+        src = f"{peak_src} hbm_gbs (copy)"
+    ach = r.work / kern_s / (1e12 if r.unit == "TFLOP/s" else 1e9)
+    roof = {"bound": "hbm" if r.kind_bound == "hbm" else "tensor", "achieved": ach,
+            "peak": peak, "unit": r.unit, "frac": ach / peak,
+            "traffic": profiled_traffic(r.kernel_key, r.w.kind, r.w.name),
+            "peak_source": src, "kernel": r.kernel_key,
+            # mean device time of the dominant kernel per step
+            "kernel_ms": kern_s * 1e3,
+            # against the nominal dense bf16 (2.25 PFLOP/s) / e4m3 / HBM (8 TB/s) figure
+            "frac_nominal": ach / NOMINAL[r.kind_bound]}
+    return {
+        "value": job_value(r.value(mean_s), world),
+        "ms_per_step": mean_s * 1e3,
+        "ms_per_step_median": float(np.median(per)) * 1e3,
+        "roofline": roof,
+        "clocks": clocks,
+        "e2e": {"value": r.value(e2e_s) * world, "unit": r.unit, "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h},
+        "l2": "flushed (256 MB write) before every step" if r.flush is not None
+              else "inputs larger than L2",
+        "wall_s": wall,
+    }
 
 
 if __name__ == "__main__":
