@@ -41,9 +41,17 @@ def test_gqa_backward(fa_mod, cuda_device, shape, causal):
     assert dk.shape == k.shape and dv.shape == v.shape
     rq, rk, rv, _ = oracle.attention_backward(*(inputs.to_f64(t) for t in (q, k, v, do)), causal,
                                               1 / np.sqrt(d))
-    check_grad(dq.cpu(), rq, "dQ")
-    check_grad(dk.cpu(), rk, "dK")
-    check_grad(dv.cpu(), rv, "dV")
+    dq, dk, dv = dq.cpu(), dk.cpu(), dv.cpu()
+    check_grad(dq, rq, "dQ")
+    check_grad(dk, rk, "dK")
+    check_grad(dv, rv, "dV")
+    # per head as well: a wrong head must not hide under the others
+    for b in range(B):
+        for h in range(H):
+            check_grad(dq[b, h], rq[b, h], f"dQ[{b},{h}]")
+        for h in range(Hkv):
+            check_grad(dk[b, h], rk[b, h], f"dK[{b},{h}]")
+            check_grad(dv[b, h], rv[b, h], f"dV[{b},{h}]")
 
 
 @pytest.mark.parametrize("d", [128, 64])

@@ -126,6 +126,17 @@ def test_bwd_varlen_matches_oracle(fa_mod, cuda_device, case, causal):
     check_grad(dq, ref_q, "dQ")
     check_grad(dk, ref_k, "dK")
     check_grad(dv, ref_v, "dV")
+    # and per sequence and head, so that one wrong sequence or head cannot
+    # hide under the others
+    for b in range(len(lens_q)):
+        q0, q1, k0, k1 = int(cu_q[b]), int(cu_q[b + 1]), int(cu_k[b]), int(cu_k[b + 1])
+        for h in range(H):
+            if q1 > q0:
+                check_grad(dq[q0:q1, h], ref_q[q0:q1, h], f"dQ seq {b} head {h}")
+        for h in range(Hkv):
+            if k1 > k0:
+                check_grad(dk[k0:k1, h], ref_k[k0:k1, h], f"dK seq {b} head {h}")
+                check_grad(dv[k0:k1, h], ref_v[k0:k1, h], f"dV seq {b} head {h}")
 
 
 def test_bwd_varlen_equal_lengths_match_padded_kernel(fa_mod, cuda_device):

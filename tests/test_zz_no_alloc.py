@@ -5,14 +5,15 @@ host program has reserved nearly all device memory for its own pool, or a
 latency-critical loop that must not trigger the device-wide synchronisation
 an allocation can cause.  Its scratch is a fixed library-owned device array,
 shared by every call.  These tests compare it with fa_decode (caller-provided
-workspace) on two different problems in a row, so that a stale array from
-the first call would show up in the second.  This file is collected last on
+workspace) and with the fp64 oracle on two different problems in a row, so
+that a stale array from the first call would show up in the second.  This file is collected last on
 purpose: a failure here comes after every other test has run.
 """
 import numpy as np
 import pytest
 import torch
 
+import oracle
 from io_aware_exact_35_b200 import inputs
 from tests._parity import check_lse, check_o
 
@@ -47,3 +48,8 @@ def test_static_decode_matches_workspace_decode_twice(fa_mod, cuda_device):
         assert fa_mod.get_device_error() == 0
         check_o(o_st.cpu(), o_ref.cpu().double().numpy(), "static-scratch O")
         check_lse(lse_st.cpu(), lse_ref.cpu().double().numpy(), "static-scratch LSE")
+        # and against the fp64 oracle itself
+        o_or, lse_or = oracle.decode_forward(*(inputs.to_f64(t) for t in (q, kc, vc)),
+                                             sl.cpu().tolist(), 1 / np.sqrt(d))
+        check_o(o_st.cpu(), o_or, "static-scratch O vs oracle")
+        check_lse(lse_st.cpu(), lse_or, "static-scratch LSE vs oracle")
