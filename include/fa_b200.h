@@ -62,7 +62,9 @@ typedef enum {
     FA_ERR_UNSUPPORTED = 2,  /* head dimension other than 64 / 128, no sm_100   */
     FA_ERR_WORKSPACE = 3,    /* workspace missing or smaller than required      */
     FA_ERR_CUDA = 4,         /* a CUDA runtime / driver call failed             */
-    FA_ERR_TIMEOUT = 5       /* a kernel's bounded wait expired (device word)   */
+    FA_ERR_TIMEOUT = 5,      /* a kernel's bounded wait expired (device word)   */
+    FA_ERR_BOUNDS = 6        /* debug build only: a kernel's bounds check failed
+                                and the access was skipped (device word)        */
 } fa_status;
 
 /*

@@ -4,6 +4,8 @@
 #include <cstring>
 #include <mutex>
 
+#include <nvtx3/nvToolsExt.h>
+
 #include "fa_internal.h"
 #include "sm100.cuh"
 
@@ -35,6 +37,16 @@ EncodeTiledFn encode_fn() {
 }
 
 constexpr int kMaxDevices = 64;
+
+// NVTX range around one ABI call, so that a timeline (nsys, ncu's NVTX
+// filter) shows which entry point launched which kernels.  Without a tool
+// attached a push / pop is a call to an empty function.
+struct Range {
+  explicit Range(const char* name) { nvtxRangePushA(name); }
+  ~Range() { nvtxRangePop(); }
+  Range(const Range&) = delete;
+  Range& operator=(const Range&) = delete;
+};
 
 // 1 = sm_100 family, 0 = other, -1 = unknown (query failed).
 fa_status check_device() {
@@ -165,6 +177,7 @@ const char* fa_status_string(fa_status s) {
     case FA_ERR_WORKSPACE: return "workspace missing or too small";
     case FA_ERR_CUDA: return "CUDA error";
     case FA_ERR_TIMEOUT: return "a kernel's bounded wait expired";
+    case FA_ERR_BOUNDS: return "a bounds check of the debug build failed";
   }
   return "unknown status";
 }
@@ -184,6 +197,7 @@ fa_status fa_fwd_gqa(const void* q, const void* k, const void* v, void* o, float
 fa_status fa_fwd_ext(const void* q, const void* k, const void* v, void* o, float* lse, int B,
                      int H, int Hkv, int Nq, int Nk, int d, int causal, float scale,
                      fa_stream_t stream) {
+  Range nvtx_range("fa_fwd_ext");
   fa_status st = check_shape(B, H, Nq, d);
   if (st != FA_OK) return st;
   if ((st = check_shape(B, Hkv, Nk, d)) != FA_OK) return st;
@@ -205,6 +219,7 @@ fa_status fa_fwd_varlen(const void* q, const void* k, const void* v, void* o, fl
                         const int* cu_seqlens_q, const int* cu_seqlens_k, int B, int H, int Hkv,
                         int total_q, int total_k, int max_seqlen_q, int d, int causal,
                         float scale, fa_stream_t stream) {
+  Range nvtx_range("fa_fwd_varlen");
   if (B < 1 || H < 1 || Hkv < 1 || H % Hkv != 0) return FA_ERR_INVALID_ARG;
   if (total_q < 0 || total_k < 0 || max_seqlen_q < 0) return FA_ERR_INVALID_ARG;
   if (static_cast<long long>(B) * H > INT_MAX) return FA_ERR_INVALID_ARG;
@@ -229,6 +244,7 @@ fa_status fa_fwd_varlen(const void* q, const void* k, const void* v, void* o, fl
 fa_status fa_fwd_fp8(const void* q, const void* k, const void* vt, void* o, float* lse,
                      float q_scale, float k_scale, float v_scale, int B, int H, int Hkv, int Nq,
                      int Nk, int d, int causal, float scale, fa_stream_t stream) {
+  Range nvtx_range("fa_fwd_fp8");
   fa_status st = check_shape(B, H, Nq, d);
   if (st != FA_OK) return st;
   if ((st = check_shape(B, Hkv, Nk, d)) != FA_OK) return st;
@@ -278,6 +294,7 @@ fa_status fa_bwd_ext(const void* q, const void* k, const void* v, const void* o,
                      const void* dout, const float* lse, void* dq, void* dk, void* dv,
                      void* workspace, size_t ws_bytes, int B, int H, int Hkv, int Nq, int Nk,
                      int d, int causal, float scale, fa_stream_t stream) {
+  Range nvtx_range("fa_bwd_ext");
   fa_status st = check_shape(B, H, Nq, d);
   if (st != FA_OK) return st;
   if ((st = check_shape(B, Hkv, Nk, d)) != FA_OK) return st;
@@ -314,6 +331,7 @@ fa_status fa_bwd_varlen(const void* q, const void* k, const void* v, const void*
                         const int* cu_seqlens_q, const int* cu_seqlens_k, void* workspace,
                         size_t ws_bytes, int B, int H, int Hkv, int total_q, int total_k,
                         int max_seqlen_k, int d, int causal, float scale, fa_stream_t stream) {
+  Range nvtx_range("fa_bwd_varlen");
   if (B < 1 || H < 1 || Hkv < 1 || H % Hkv != 0) return FA_ERR_INVALID_ARG;
   if (total_q < 0 || total_k < 0 || max_seqlen_k < 0) return FA_ERR_INVALID_ARG;
   if (static_cast<long long>(B) * H > INT_MAX) return FA_ERR_INVALID_ARG;
@@ -357,6 +375,7 @@ fa_status fa_decode(const void* q, const void* kcache, const void* vcache, const
 fa_status fa_decode_gqa(const void* q, const void* kcache, const void* vcache, const int* seqlens,
                         void* o, float* lse, int B, int H, int Hkv, int Lmax, int d, float scale,
                         void* workspace, size_t ws_bytes, fa_stream_t stream) {
+  Range nvtx_range("fa_decode_gqa");
   if (B < 1 || H < 1 || Lmax < 0) return FA_ERR_INVALID_ARG;
   if (Hkv < 1 || H % Hkv != 0) return FA_ERR_INVALID_ARG;
   if (static_cast<long long>(B) * H > INT_MAX) return FA_ERR_INVALID_ARG;
@@ -380,6 +399,7 @@ fa_status fa_decode_paged(const void* q, const void* kpages, const void* vpages,
                           const int* block_table, const int* seqlens, void* o, float* lse, int B,
                           int H, int Hkv, int page_size, int pages_per_seq, int num_pages, int d,
                           float scale, void* workspace, size_t ws_bytes, fa_stream_t stream) {
+  Range nvtx_range("fa_decode_paged");
   if (B < 1 || H < 1 || pages_per_seq < 0 || num_pages < 0) return FA_ERR_INVALID_ARG;
   if (Hkv < 1 || H % Hkv != 0) return FA_ERR_INVALID_ARG;
   if (static_cast<long long>(B) * H > INT_MAX) return FA_ERR_INVALID_ARG;

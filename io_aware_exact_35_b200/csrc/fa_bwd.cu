@@ -103,6 +103,7 @@ struct Params {
   int total_q, total_k;
   // element strides of dK / dV: [head][row] at head * kv_head + row * kv_row
   size_t kv_head, kv_row;
+  size_t kv_elems;   // elements of dK (= of dV), for the debug build's checks
 };
 
 // First row of sequence b in the ragged LSE / D tables: a multiple of 4 (a
@@ -182,6 +183,7 @@ __device__ __forceinline__ void reduce_rows(const CUtensorMap* map, const void* 
 
 __device__ __forceinline__ void tma_load_2d(void* smem_dst, const void* desc, uint64_t* bar,
                                             int c0, int c1) {
+  if (!dbg_ok(c0 >= 0 && (c0 & 3) == 0 && c1 >= 0)) return;  // fp32 rows, 16-byte aligned
   asm volatile(
       "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
       " [%0], [%1, {%2, %3}], [%4];" ::"r"(smem_u32(smem_dst)),
@@ -493,7 +495,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             pk[e >> 1] = seen ? pack_bf16x2(__uint_as_float(r[e]) * mul,
                                             __uint_as_float(r[e + 1]) * mul)
                               : 0u;
-          if (key_ok) {
+          if (key_ok && dbg_ok(rowoff + c + 32 <= p.kv_elems)) {
             uint4* dst = reinterpret_cast<uint4*>(dst_row + c);
 #pragma unroll
             for (int v4 = 0; v4 < 4; ++v4)
@@ -788,6 +790,7 @@ fa_status launch_bwd(const void* q, const void* k, const void* v, const void* o,
   prm.total_k = 0;
   prm.kv_head = static_cast<size_t>(Nk) * d;
   prm.kv_row = static_cast<size_t>(d);
+  prm.kv_elems = static_cast<size_t>(BHkv) * Nk * d;
   if (d == 128)
     st = causal ? bwd::launch_main<128, true, false>(maps, prm, BHkv, stream)
                 : bwd::launch_main<128, false, false>(maps, prm, BHkv, stream);
@@ -884,6 +887,7 @@ fa_status launch_bwd_varlen(const void* q, const void* k, const void* v, const v
   prm.total_k = total_k;
   prm.kv_head = static_cast<size_t>(d);
   prm.kv_row = static_cast<size_t>(Hkv) * d;
+  prm.kv_elems = static_cast<size_t>(total_k) * Hkv * d;
   if (static_cast<long long>(prm.n_kt) * prm.BHkv > 0x7fffffffLL) return FA_ERR_INVALID_ARG;
   if (d == 128)
     st = causal ? bwd::launch_main<128, true, true>(maps, prm, prm.BHkv, stream)

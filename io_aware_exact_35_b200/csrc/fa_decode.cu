@@ -207,7 +207,7 @@ __global__ void __launch_bounds__(THREADS)
           vu[u] = make_uint4(0, 0, 0, 0);
         }
       } else {
-        if (key[u] < c1) {
+        if (key[u] < c1 && dbg_ok(key[u] < Lmax)) {
           ku[u] = ld_stream(kbase + static_cast<size_t>(key[u]) * D);
           vu[u] = ld_stream(vbase + static_cast<size_t>(key[u]) * D);
         } else {
@@ -262,6 +262,7 @@ __global__ void __launch_bounds__(THREADS)
   }
   __syncthreads();
   float* out = part + (bh * S + split) * (D + 2);
+  if (!dbg_ok(split < S)) return;
   for (int t = threadIdx.x; t < D; t += THREADS) {
     float M = -INFINITY;
 #pragma unroll
@@ -553,6 +554,7 @@ __global__ void __launch_bounds__(THREADS)
       lt = fmaf(wt, red_l[row][w], lt);
     }
     float* out = part + ((static_cast<size_t>(b) * H + h0 + row) * S + split) * (D + 2);
+    if (!dbg_ok(split < S && h0 + row < H)) continue;
     out[t] = acc;
     if (t == 0) {
       out[D] = M;

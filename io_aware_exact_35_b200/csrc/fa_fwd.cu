@@ -12,21 +12,27 @@
 // normalisation (MMA warp + softmax warpgroups), accumulate without the full
 // matrix (MMA warp, O in tensor memory), and the kernel schedule (grid order).
 //
-// Warp roles (320 threads):
+// Warp roles (512 threads, four warpgroups; registers are moved between the
+// warpgroups with setmaxnreg so that the softmax gets most of them):
 //   warps 0-3  softmax warpgroup 0: thread t owns row t of query tile 0.
 //   warps 4-7  softmax warpgroup 1: the same for query tile 1.
 //              Each reads its S from tensor memory, masks, keeps the running
 //              max m and sum l (log2 domain), writes P as bf16 into the same
-//              tensor-memory columns, rescales its O when m grows, and finally
-//              writes O / l and LSE.
-//   warp 8     TMA producer: the query pair of each work item, then K_j and
+//              tensor-memory columns, rescales its O when m grows, and at the
+//              end of a work item writes LSE and hands 1 / l to the epilogue.
+//   warps 8-11 epilogue warpgroup: once a tile's last O += P V has completed
+//              it reads O out of tensor memory (thread t: row t), multiplies
+//              by 1 / l and stores bf16 rows, while the softmax warpgroups
+//              already work on the next item.
+//   warp 12    TMA producer: the query pair of each work item, then K_j and
 //              V_j through one ring of NSLOT tile-sized slots that holds K and
 //              V tiles in the order they are consumed (K_0 V_0 K_1 V_1 ...), so
 //              loads run about two key tiles ahead of the tensor core.
-//   warp 9     tensor-memory allocator and MMA issuer (one thread).  The two
+//   warp 13    tensor-memory allocator and MMA issuer (one thread).  The two
 //              query tiles ping-pong: while warpgroup 0 exponentiates S_0,j the
 //              tensor core runs O_1 += P_1 V_{j-1} and S_1,j, and vice versa:
 //                S0(0) S1(0) | PV0(0) S0(1) PV1(0) S1(1) | PV0(1) S0(2) ...
+//   warps 14-15 idle (they complete the fourth warpgroup).
 //
 // Tensor memory (512 columns x 128 lanes, fp32): S_0 [0,128), S_1 [128,256),
 // O_0 [256,384), O_1 [384,512).  P_w overwrites the first 64 columns of S_w
@@ -80,13 +86,70 @@ __device__ __forceinline__ uint32_t pack_e4m3x4(float x0, float x1, float x2, fl
   return r;
 }
 
+// The same three tensor-core operations issued by a converged warp: every
+// lane holds the same (warp-uniform) operands and elect.sync picks the one
+// lane that issues, so the operands can stay in uniform registers.
+__device__ __forceinline__ void mma_bf16_ss_w(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                              uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p, e;\n\t"
+      "elect.sync _|e, 0xffffffff;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+__device__ __forceinline__ void mma_bf16_ts_w(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
+                                              uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p, e;\n\t"
+      "elect.sync _|e, 0xffffffff;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+__device__ __forceinline__ void mma_f8_ss_w(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                            uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p, e;\n\t"
+      "elect.sync _|e, 0xffffffff;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+__device__ __forceinline__ void mma_commit_w(uint64_t* bar) {
+  asm volatile(
+      "{\n\t.reg .pred e;\n\t"
+      "elect.sync _|e, 0xffffffff;\n\t"
+      "@e tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n\t}" ::"r"(
+          smem_u32(bar))
+      : "memory");
+}
+
 namespace fwd {
+
+#ifndef FA_FWD_MMA_WARP
+#define FA_FWD_MMA_WARP 0
+#endif
+// 1: the whole MMA warp runs the issue loop converged (elect.sync per
+// instruction); 0: lane 0 alone runs it.
+constexpr bool MMA_WARP = FA_FWD_MMA_WARP != 0;
 
 constexpr int TILE_M = 128;   // rows per softmax warpgroup
 constexpr int NQ = 2;         // query tiles per CTA
 constexpr int BLOCK_M = TILE_M * NQ;
 constexpr int BLOCK_N = 128;
-constexpr int NUM_THREADS = 320;
+constexpr int NUM_THREADS = 512;
+constexpr int WARP_PRODUCER = 12;
+constexpr int WARP_MMA = 13;
+// Registers per thread after setmaxnreg (launch: 65536 / 512 = 128 each):
+// 2 x 128 x 184 + 128 x 48 + 128 x 96 = 65536 (the producer / MMA warpgroup
+// needs more than the epilogue: its issue loops keep many descriptors live).
+constexpr int REGS_SOFTMAX = 184;
+constexpr int REGS_EPILOGUE = 48;
+constexpr int REGS_OTHER = 96;
 constexpr int PANEL_BYTES = 128 * 128;   // 128 rows x 64 bf16 (one swizzle panel)
 constexpr uint32_t TMEM_COLS = 512;
 constexpr float RESCALE_THRESHOLD = 8.0f;  // log2 units
@@ -105,6 +168,29 @@ __device__ __forceinline__ void fma_f32x2(float& x0, float& x1, float a0, float 
   asm("fma.rn.ftz.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(pack_f32x2(a0, a1)), "l"(b), "l"(c));
   asm("mov.b64 {%0, %1}, %2;" : "=f"(x0), "=f"(x1) : "l"(d));
 }
+// 32 lanes x 8 consecutive 32-bit columns of tensor memory (load / store).
+__device__ __forceinline__ void tmem_ld8(uint32_t taddr, uint32_t (&r)[8]) {
+  asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]),
+                 "=r"(r[6]), "=r"(r[7])
+               : "r"(taddr));
+}
+__device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t (&r)[8]) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};"
+               ::"r"(taddr), "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]),
+                 "r"(r[6]), "r"(r[7])
+               : "memory");
+}
+
+// acc += (a0, a1) lane by lane, one packed f32x2 addition.
+__device__ __forceinline__ void add_f32x2(uint64_t& acc, float a0, float a1) {
+  asm("add.rn.ftz.f32x2 %0, %0, %1;" : "+l"(acc) : "l"(pack_f32x2(a0, a1)));
+}
+__device__ __forceinline__ float sum_f32x2(uint64_t v) {
+  float a, b;
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(a), "=f"(b) : "l"(v));
+  return a + b;
+}
 
 // max(a, b, c) in one instruction (three-input max.f32, sm_100).  Inputs
 // here are finite or -inf, never NaN.
@@ -113,10 +199,40 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
   asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
   return r;
 }
+// 2^x0, 2^x1 on the FMA pipe, two lanes per packed f32x2 instruction: the
+// cubic of ex2_poly3 (sm100.cuh; Remez fit of
+// io_aware_exact_35_b200/exp2_poly.py) evaluated on the pair.  Inputs are
+// clamped at -125 (so masked scores must not come here).
+__device__ __forceinline__ void ex2_poly3_x2(float x0, float x1, float& y0, float& y1) {
+  const uint64_t x = pack_f32x2(fmaxf(x0, -125.f), fmaxf(x1, -125.f));
+  const uint64_t magic = pack_f32x2(12582912.f, 12582912.f);  // 1.5 * 2^23
+  uint64_t t, n, f, q;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(t) : "l"(x), "l"(magic));  // x rounded into t's mantissa
+  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(n) : "l"(t), "l"(magic));  // n = round(x)
+  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(f) : "l"(x), "l"(n));      // f in [-1/2, 1/2]
+  asm("fma.rn.f32x2 %0, %1, %2, %3;"
+      : "=l"(q) : "l"(pack_f32x2(kEx2C3, kEx2C3)), "l"(f), "l"(pack_f32x2(kEx2C2, kEx2C2)));
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(q) : "l"(q), "l"(f), "l"(pack_f32x2(kEx2C1, kEx2C1)));
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(q) : "l"(q), "l"(f), "l"(pack_f32x2(kEx2C0, kEx2C0)));
+  float q0, q1, t0, t1;
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(q0), "=f"(q1) : "l"(q));
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(t0), "=f"(t1) : "l"(t));
+  // n sits in the low mantissa bits of t: shifting it into the exponent
+  // field multiplies 2^f by 2^n
+  y0 = __int_as_float(__float_as_int(q0) + (__float_as_int(t0) << 23));
+  y1 = __int_as_float(__float_as_int(q1) + (__float_as_int(t1) << 23));
+}
+
 #ifndef FA_FWD_EMU_PAIRS
 #define FA_FWD_EMU_PAIRS 0
 #endif
 constexpr int EMU_PAIRS = FA_FWD_EMU_PAIRS;  // of every 4 exp pairs, on the FMA pipe
+#ifndef FA_FWD_P_SPLIT
+#define FA_FWD_P_SPLIT 0
+#endif
+// P handed to the tensor core in two halves (keys 0-63, then 64-127), so that
+// the first half of O += P V runs while the second half is exponentiated.
+constexpr bool P_SPLIT = FA_FWD_P_SPLIT != 0;
 
 // Shared-memory plan.  A panel is 128 rows x 128 bytes (64 bf16 or 128 e4m3
 // values per row).  With 8-bit inputs (F8) the ring carries K_j and V_j^T
@@ -132,9 +248,12 @@ struct Smem {
   static constexpr int P_OFF = RING_OFF + NSLOT * TILE;  // F8: NQ tiles of 128 x 128 e4m3
   static constexpr int BAR_OFF = P_OFF + (F8 ? NQ * PANEL_BYTES : 0);
   // barriers: q_full, q_empty, full[NSLOT], empty[NSLOT],
-  //           s_full[NQ], p_full[NQ], o_done[NQ], o_final[NQ], o_free[NQ], mma_final
-  static constexpr int NBAR = 2 + 2 * NSLOT + 5 * NQ + 1;
-  static constexpr int MISC_OFF = BAR_OFF + NBAR * 8;
+  //           s_full[NQ], p_full[NQ], o_done[NQ], o_final[NQ], o_free[NQ], mma_final,
+  //           l_ready[NQ][2], p_half[NQ]
+  static constexpr int NBAR = 2 + 2 * NSLOT + 5 * NQ + 1 + 2 * NQ + NQ;
+  // 1 / l of every row, per query tile, for work items of even / odd index
+  static constexpr int STAT_OFF = BAR_OFF + NBAR * 8;
+  static constexpr int MISC_OFF = STAT_OFF + 2 * NQ * TILE_M * 4;
   static constexpr int BYTES = MISC_OFF + 16;
   // at least 116 KB so that a single CTA (and its 512 tensor-memory columns)
   // occupies an SM.
@@ -165,6 +284,7 @@ struct Params {
   // element strides of O and LSE: O[head][row] at head * o_head + row * o_row,
   // LSE at head * lse_head + row, with head = b*H + h (padded) or h (ragged)
   size_t o_head, o_row, lse_head;
+  size_t o_elems, lse_elems;  // sizes of O and LSE, for the debug build's checks
 };
 
 // Work item -> (batch*head, 256-row tile).  In LPT order the longest tiles of
@@ -272,6 +392,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   uint64_t* o_final = o_done + NQ;  // [NQ] one phase per work item: its last O += P V
   uint64_t* o_free = o_final + NQ;  // [NQ] one phase per work item: O read out
   uint64_t* mma_final = o_free + NQ;
+  uint64_t* l_ready = mma_final + 1;  // [NQ][2]: 1 / l written, per item parity
+  uint64_t* p_half = l_ready + 2 * NQ;  // [NQ]: first half of P written (P_SPLIT)
+  float* inv_l_buf = reinterpret_cast<float*>(smem + L::STAT_OFF);  // [2][NQ][TILE_M]
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::MISC_OFF);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::MISC_OFF + 4);
 
@@ -310,16 +433,19 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       mbar_init(&o_done[w], 1);
       mbar_init(&o_final[w], 1);
       mbar_init(&o_free[w], TILE_M);
+      mbar_init(&l_ready[2 * w], TILE_M);
+      mbar_init(&l_ready[2 * w + 1], TILE_M);
+      mbar_init(&p_half[w], TILE_M);
     }
     mbar_init(mma_final, 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
-  if (warp == 9) {
+  if (warp == WARP_MMA) {
     tmem_alloc(tmem_slot, TMEM_COLS);
     tmem_relinquish();
   }
-  if (warp == 8 && lane == 0) {
+  if (warp == WARP_PRODUCER && lane == 0) {
     tma_prefetch_desc(&tm_q);
     tma_prefetch_desc(&tm_k);
     tma_prefetch_desc(&tm_v);
@@ -329,7 +455,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
 
-  if (warp == 8) {
+  if (warp >= 12) {
+   asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(REGS_OTHER));
+   if (warp == WARP_PRODUCER) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
       int kv = 0;        // key tiles loaded so far (all work items)
@@ -379,9 +507,18 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       for (int u = max(0, loaded - NSLOT); u < loaded; ++u)
         mbar_wait_drain(&full[u % NSLOT], (u / NSLOT) & 1);
     }
-  } else if (warp == 9) {
+   } else if (warp == WARP_MMA) {
     // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
+    if (MMA_WARP || lane == 0) {
+      // waits of the issue loop: warp-collective when the whole warp runs it
+      auto mwait = [&](uint64_t* bar, uint32_t parity) {
+        if constexpr (MMA_WARP) return mbar_wait_warp(bar, parity, abort_flag);
+        else return mbar_wait(bar, parity, abort_flag);
+      };
+      auto commit = [&](uint64_t* bar) {
+        if constexpr (MMA_WARP) mma_commit_w(bar);
+        else mma_commit(bar);
+      };
       constexpr uint32_t IDESC_S =
           F8 ? idesc_e4m3_f32(TILE_M, BLOCK_N) : idesc_bf16_f32(TILE_M, BLOCK_N, false, false);
       constexpr uint32_t IDESC_O =
@@ -408,52 +545,75 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 #pragma unroll
           for (int kk = 0; kk < D / 32; ++kk) {  // 32 e4m3 = 32 bytes per step
             const uint64_t off = static_cast<uint64_t>(((kk >> 2) * PANEL_BYTES + (kk & 3) * 32) >> 4);
-            mma_f8_ss(dS, qd + off, kd + off, IDESC_S, kk > 0 ? 1u : 0u);
+            if constexpr (MMA_WARP) mma_f8_ss_w(dS, qd + off, kd + off, IDESC_S, kk > 0 ? 1u : 0u);
+            else mma_f8_ss(dS, qd + off, kd + off, IDESC_S, kk > 0 ? 1u : 0u);
           }
         } else {
 #pragma unroll
           for (int kk = 0; kk < D / 16; ++kk) {
             const uint64_t off = static_cast<uint64_t>(((kk >> 2) * PANEL_BYTES + (kk & 3) * 32) >> 4);
-            mma_bf16_ss(dS, qd + off, kd + off, IDESC_S, kk > 0 ? 1u : 0u);
+            if constexpr (MMA_WARP) mma_bf16_ss_w(dS, qd + off, kd + off, IDESC_S, kk > 0 ? 1u : 0u);
+            else mma_bf16_ss(dS, qd + off, kd + off, IDESC_S, kk > 0 ? 1u : 0u);
           }
         }
-        mma_commit(&s_full[w]);
+        commit(&s_full[w]);
       };
       // O_w (+)= P_w V with V in ring slot `slot`, once warpgroup w wrote P_w
       auto issue_pv = [&](int w, int slot, bool first, bool last) -> bool {
-        if (!mbar_wait(&p_full[w], pcount[w] & 1, abort_flag)) return false;
-        ++pcount[w];
-        tc_fence_after();
         const uint32_t tO = tmem_base + 256 + w * 128;
-        if constexpr (F8) {
-          // A = P_w (queries x keys) and B = V_j^T (d x keys), both K-major
-          const uint64_t pd = p_desc0 + static_cast<uint64_t>((w * PANEL_BYTES) >> 4);
-          const uint64_t vd = ring_kdesc0 + static_cast<uint64_t>((slot * L::TILE) >> 4);
+        // keys [16 kk0, 16 kk1) (bf16) or [32 kk0, 32 kk1) (e4m3)
+        auto pv_range = [&](int kk0, int kk1) {
+          if constexpr (F8) {
+            // A = P_w (queries x keys) and B = V_j^T (d x keys), both K-major
+            const uint64_t pd = p_desc0 + static_cast<uint64_t>((w * PANEL_BYTES) >> 4);
+            const uint64_t vd = ring_kdesc0 + static_cast<uint64_t>((slot * L::TILE) >> 4);
 #pragma unroll
-          for (int kk = 0; kk < BLOCK_N / 32; ++kk) {
-            const uint64_t off = static_cast<uint64_t>((kk * 32) >> 4);
-            mma_f8_ss(tO, pd + off, vd + off, IDESC_O, (!first || kk > 0) ? 1u : 0u);
+            for (int kk = kk0; kk < kk1; ++kk) {
+              const uint64_t off = static_cast<uint64_t>((kk * 32) >> 4);
+              if constexpr (MMA_WARP)
+                mma_f8_ss_w(tO, pd + off, vd + off, IDESC_O, (!first || kk > 0) ? 1u : 0u);
+              else
+                mma_f8_ss(tO, pd + off, vd + off, IDESC_O, (!first || kk > 0) ? 1u : 0u);
+            }
+          } else {
+            const uint64_t vd = ring_vdesc0 + static_cast<uint64_t>((slot * L::TILE) >> 4);
+            const uint32_t tP = tmem_base + w * 128;
+#pragma unroll
+            for (int kk = kk0; kk < kk1; ++kk) {
+              // keys 16kk .. 16kk+15: P columns 8kk.., V rows 16kk.. (2048 bytes per step)
+              const uint64_t vdk = vd + static_cast<uint64_t>((kk * 2048) >> 4);
+              if constexpr (MMA_WARP)
+                mma_bf16_ts_w(tO, tP + kk * 8, vdk, IDESC_O, (!first || kk > 0) ? 1u : 0u);
+              else
+                mma_bf16_ts(tO, tP + kk * 8, vdk, IDESC_O, (!first || kk > 0) ? 1u : 0u);
+            }
           }
+        };
+        constexpr int KK = F8 ? BLOCK_N / 32 : BLOCK_N / 16;
+        if constexpr (P_SPLIT) {
+          if (!mwait(&p_half[w], pcount[w] & 1)) return false;
+          tc_fence_after();
+          pv_range(0, KK / 2);
+          if (!mwait(&p_full[w], pcount[w] & 1)) return false;
+          ++pcount[w];
+          tc_fence_after();
+          pv_range(KK / 2, KK);
         } else {
-          const uint64_t vd = ring_vdesc0 + static_cast<uint64_t>((slot * L::TILE) >> 4);
-          const uint32_t tP = tmem_base + w * 128;
-#pragma unroll
-          for (int kk = 0; kk < BLOCK_N / 16; ++kk) {
-            // keys 16kk .. 16kk+15: P columns 8kk.., V rows 16kk.. (2048 bytes per step)
-            mma_bf16_ts(tO, tP + kk * 8, vd + static_cast<uint64_t>((kk * 2048) >> 4), IDESC_O,
-                        (!first || kk > 0) ? 1u : 0u);
-          }
+          if (!mwait(&p_full[w], pcount[w] & 1)) return false;
+          ++pcount[w];
+          tc_fence_after();
+          pv_range(0, KK);
         }
-        mma_commit(&o_done[w]);
-        if (last) mma_commit(&o_final[w]);
+        commit(&o_done[w]);
+        if (last) commit(&o_final[w]);
         return true;
       };
 
       int kv = 0;  // key tiles consumed so far (all work items)
       auto kslot = [&](int g) { return (2 * g) % NSLOT; };
       auto vslot = [&](int g) { return (2 * g + 1) % NSLOT; };
-      auto kwait = [&](int g) { return mbar_wait(&full[kslot(g)], ((2 * g) / NSLOT) & 1, abort_flag); };
-      auto vwait = [&](int g) { return mbar_wait(&full[vslot(g)], ((2 * g + 1) / NSLOT) & 1, abort_flag); };
+      auto kwait = [&](int g) { return mwait(&full[kslot(g)], ((2 * g) / NSLOT) & 1); };
+      auto vwait = [&](int g) { return mwait(&full[vslot(g)], ((2 * g + 1) / NSLOT) & 1); };
       bool ok = true;
       for (int k = 0; ok; ++k) {
         const int item = cta_item(cta, k, G);
@@ -461,12 +621,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         const ItemGeo g = item_geo<VARLEN>(p, item);
         const int n0 = n_kv_of(g, 0);
         const int n1 = n_kv_of(g, 1);
-        if (!mbar_wait(q_full, k & 1, abort_flag) || !kwait(kv)) { ok = false; break; }
+        if (!mwait(q_full, k & 1) || !kwait(kv)) { ok = false; break; }
         tc_fence_after();
         issue_s(0, kslot(kv));
         issue_s(1, kslot(kv));
-        mma_commit(&empty[kslot(kv)]);
-        if (n1 == 1) mma_commit(q_empty);
+        commit(&empty[kslot(kv)]);
+        if (n1 == 1) commit(q_empty);
         for (int j = 0; j < n1; ++j) {
           const int g = kv + j;
           const bool more = j + 1 < n1;
@@ -474,7 +634,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           if (j < n0) {
             // the first product of an item overwrites O_0: its read-out by the
             // previous item's epilogue must be complete
-            if (j == 0 && k > 0 && !mbar_wait(&o_free[0], (k - 1) & 1, abort_flag)) { ok = false; break; }
+            if (j == 0 && k > 0 && !mwait(&o_free[0], (k - 1) & 1)) { ok = false; break; }
             if (!issue_pv(0, vslot(g), j == 0, j == n0 - 1)) { ok = false; break; }
           }
           if (more) {
@@ -482,22 +642,76 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             tc_fence_after();
             if (j + 1 < n0) issue_s(0, kslot(g + 1));
           }
-          if (j == 0 && k > 0 && !mbar_wait(&o_free[1], (k - 1) & 1, abort_flag)) { ok = false; break; }
+          if (j == 0 && k > 0 && !mwait(&o_free[1], (k - 1) & 1)) { ok = false; break; }
           if (!issue_pv(1, vslot(g), j == 0, j == n1 - 1)) { ok = false; break; }
-          mma_commit(&empty[vslot(g)]);
+          commit(&empty[vslot(g)]);
           if (more) {
             issue_s(1, kslot(g + 1));
-            mma_commit(&empty[kslot(g + 1)]);
-            if (j + 2 == n1) mma_commit(q_empty);  // last S of this item issued
+            commit(&empty[kslot(g + 1)]);
+            if (j + 2 == n1) commit(q_empty);  // last S of this item issued
           }
         }
         kv += n1;
       }
       // All MMAs must retire before tensor memory is released.
-      mma_commit(mma_final);
+      commit(mma_final);
       mbar_wait_drain(mma_final, 0);
     }
+   }
+  } else if (warp >= 8) {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(REGS_EPILOGUE));
+    // ------------------------------------------------------------ epilogue
+    // Thread t of the warpgroup owns row t of each query tile: tensor-memory
+    // lanes 32 (warp % 4) .. +31 are this warp's.
+    const int row = threadIdx.x - 8 * 32;
+    const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
+    bool ok = true;
+    for (int k = 0; ok; ++k) {
+      const int item = cta_item(cta, k, G);
+      if (item >= p.total_items) break;
+      const ItemGeo g = item_geo<VARLEN>(p, item);
+      for (int w = 0; w < NQ; ++w) {
+        // the tile's last O += P V has completed, and its 1 / l is written
+        if (!mbar_wait_warp(&o_final[w], k & 1, abort_flag) ||
+            !mbar_wait_warp(&l_ready[2 * w + (k & 1)], (k >> 1) & 1, abort_flag)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const float inv_l = inv_l_buf[((k & 1) * NQ + w) * TILE_M + row];
+        const uint32_t tO = tmem_base + 256 + w * 128 + lane_off;
+        const int row_g = g.tile * BLOCK_M + w * TILE_M + row;  // within the sequence
+        const size_t orow_off = static_cast<size_t>(g.head) * p.o_head +
+                                static_cast<size_t>(g.q0 + row_g) * p.o_row;
+        const bool valid = row_g < g.Nq && dbg_ok(orow_off + D <= p.o_elems);
+        __nv_bfloat16* orow_g = p.o + orow_off;
+#pragma unroll
+        for (int c = 0; c < D; c += 32) {
+          uint32_t orow[32];
+          tmem_ld32(tO + c, orow);
+          tmem_ld_wait();
+          if (c + 32 == D) {
+            // O_w has been read: the next item's first O += P V may overwrite it.
+            tc_fence_before();
+            mbar_arrive(&o_free[w]);
+          }
+          uint32_t pk[16];
+#pragma unroll
+          for (int e = 0; e < 32; e += 2)
+            pk[e >> 1] = pack_bf16x2(__uint_as_float(orow[e]) * inv_l,
+                                     __uint_as_float(orow[e + 1]) * inv_l);
+          if (valid) {
+            uint4* dst = reinterpret_cast<uint4*>(orow_g + c);
+#pragma unroll
+            for (int v4 = 0; v4 < 4; ++v4)
+              dst[v4] = make_uint4(pk[4 * v4], pk[4 * v4 + 1], pk[4 * v4 + 2], pk[4 * v4 + 3]);
+          }
+        }
+      }
+    }
+    tmem_ld_wait();
   } else {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(REGS_SOFTMAX));
     // ------------------------------------------------------------ softmax
     const int w = warp >> 2;                       // query tile of this warpgroup
     const int row = threadIdx.x - w * TILE_M;      // 0..127, TMEM lane
@@ -555,8 +769,34 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         const bool warp_grow = __any_sync(0xffffffffu, grow);
         const float m_use = warp_grow ? m_new : m;
         const float m_ref = (m_use == -INFINITY) ? 0.f : m_use;
-        const float alpha = ex2_approx(m - m_ref);  // 0 when m = -inf
-        float rs[4] = {0.f, 0.f, 0.f, 0.f};
+        // 1 unless the maximum moves (then 0 when m = -inf).  Evaluated only
+        // when needed: on the critical path an exponential would queue behind
+        // the other warpgroup's exponentials on the shared MUFU unit.
+        const float alpha = warp_grow ? ex2_approx(m - m_ref) : 1.f;
+        if (warp_grow && j > 0) {
+          // O holds P_0 V_0 + ... + P_{j-1} V_{j-1} relative to the old max:
+          // rescale it before this step's P is handed over.  S_w,j was issued
+          // after O_w += P_{j-1} V_{j-1}, so o_done[w] has completed exactly
+          // pv_base + j times; the wait only confirms it.
+          if (!mbar_wait_warp(&o_done[w], (pv_base + j - 1) & 1, abort_flag)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          // eight columns at a time: S is still live in registers here
+#pragma unroll 1
+          for (int c = 0; c < D; c += 8) {
+            uint32_t orow[8];
+            tmem_ld8(tO + c, orow);
+            tmem_ld_wait();
+#pragma unroll
+            for (int e = 0; e < 8; ++e)
+              orow[e] = __float_as_uint(__uint_as_float(orow[e]) * alpha);
+            tmem_st8(tO + c, orow);
+          }
+        }
+        // row sum in four packed two-lane chains (one f32x2 addition per pair)
+        uint64_t rs2[4] = {0, 0, 0, 0};
         // Exponentials: MUFU ex2; in unmasked tiles EMU_PAIRS of every 4 pairs
         // may go to the FMA-pipe polynomial.  Masked tiles use ex2 only, so
         // excluded keys give exactly 0.
@@ -574,13 +814,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                       negm_2);
             float p0, p1;
             if (((e >> 1) & 3) >= 4 - EMU_PAIRS && !need_mask) {
-              p0 = ex2_poly3(x0);
-              p1 = ex2_poly3(x1);
+              ex2_poly3_x2(x0, x1, p0, p1);
             } else {
               p0 = ex2_approx(x0);
               p1 = ex2_approx(x1);
             }
-            rs[(e >> 1) & 3] += p0 + p1;
+            add_f32x2(rs2[(e >> 1) & 3], p0, p1);
             if constexpr (F8) {
               pf[e] = p0;
               pf[e + 1] = p1;
@@ -604,65 +843,34 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           } else {
             tmem_st16(tS + (c >> 1), pk);
           }
+          if (P_SPLIT && c == 32) {
+            // keys 0-63 of P are written: the first half of O += P V may start
+            if constexpr (F8) fence_proxy_async_smem();
+            else tmem_st_wait();
+            tc_fence_before();
+            mbar_arrive(&p_half[w]);
+          }
         }
         // e4m3 P is read by the async proxy (tensor core) from shared memory
         if constexpr (F8) fence_proxy_async_smem();
-        l = l * alpha + ((rs[0] + rs[1]) + (rs[2] + rs[3]));
-        if (warp_grow && j > 0) {
-          // O holds P_0 V_0 + ... + P_{j-1} V_{j-1} relative to the old max.
-          // S_w,j was issued after O_w += P_{j-1} V_{j-1}, so o_done[w] has
-          // completed exactly pv_base + j times; the wait only confirms it.
-          if (!mbar_wait_warp(&o_done[w], (pv_base + j - 1) & 1, abort_flag)) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-#pragma unroll
-          for (int c = 0; c < D; c += 32) {
-            uint32_t orow[32];
-            tmem_ld32(tO + c, orow);
-            tmem_ld_wait();
-#pragma unroll
-            for (int e = 0; e < 32; ++e)
-              orow[e] = __float_as_uint(__uint_as_float(orow[e]) * alpha);
-            tmem_st32(tO + c, orow);
-          }
-        }
+        l = l * alpha + ((sum_f32x2(rs2[0]) + sum_f32x2(rs2[1])) +
+                         (sum_f32x2(rs2[2]) + sum_f32x2(rs2[3])));
         m = m_use;
         tmem_st_wait();
         tc_fence_before();
         mbar_arrive(&p_full[w]);
       }
-      if (!ok || !mbar_wait_warp(&o_final[w], k & 1, abort_flag)) {
-        ok = false;
-        break;
-      }
-      tc_fence_after();
-      const float inv_l = (l > 0.f) ? p.o_scale / l : 0.f;
-      const bool valid = row_g < g.Nq;
-      __nv_bfloat16* orow_g = p.o + static_cast<size_t>(g.head) * p.o_head +
-                              static_cast<size_t>(g.q0 + row_g) * p.o_row;
-#pragma unroll
-      for (int c = 0; c < D; c += 32) {
-        uint32_t orow[32];
-        tmem_ld32(tO + c, orow);
-        tmem_ld_wait();
-        uint32_t pk[16];
-#pragma unroll
-        for (int e = 0; e < 32; e += 2)
-          pk[e >> 1] = pack_bf16x2(__uint_as_float(orow[e]) * inv_l,
-                                   __uint_as_float(orow[e + 1]) * inv_l);
-        if (valid) {
-          uint4* dst = reinterpret_cast<uint4*>(orow_g + c);
-#pragma unroll
-          for (int v4 = 0; v4 < 4; ++v4)
-            dst[v4] = make_uint4(pk[4 * v4], pk[4 * v4 + 1], pk[4 * v4 + 2], pk[4 * v4 + 3]);
-        }
-      }
-      // O_w has been read: the next item's first O += P V may overwrite it.
-      tc_fence_before();
-      mbar_arrive(&o_free[w]);
-      if (valid && p.lse != nullptr) {
+      if (!ok) break;
+      // End of the work item for this tile: LSE, and 1 / l for the epilogue
+      // warpgroup (which normalises O once the last O += P V has completed).
+      // The buffer and barrier alternate with the item's parity: the next
+      // item of this tile can finish its softmax before the epilogue has
+      // read this one, but not the item after it (its first P V waits until
+      // the epilogue has read this item's O).
+      inv_l_buf[((k & 1) * NQ + w) * TILE_M + row] = (l > 0.f) ? p.o_scale / l : 0.f;
+      mbar_arrive(&l_ready[2 * w + (k & 1)]);
+      if (row_g < g.Nq && p.lse != nullptr &&
+          dbg_ok(static_cast<size_t>(g.head) * p.lse_head + g.q0 + row_g < p.lse_elems)) {
         // LSE = ln(sum exp(scale * s)) = (m + log2 l) * ln 2, m in log2 units.
         const float lse = (l > 0.f) ? (m + lg2_approx(l)) * 0.6931471805599453f : -INFINITY;
         p.lse[static_cast<size_t>(g.head) * p.lse_head + g.q0 + row_g] = lse;
@@ -675,7 +883,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 9) {
+  if (warp == WARP_MMA) {
     __syncwarp();
     tc_fence_after();
     tmem_dealloc(tmem_base, TMEM_COLS);
@@ -774,6 +982,8 @@ fa_status launch_fwd(const void* q, const void* k, const void* v, void* o, float
   prm.o_head = static_cast<size_t>(Nq) * d;
   prm.o_row = static_cast<size_t>(d);
   prm.lse_head = static_cast<size_t>(Nq);
+  prm.o_elems = static_cast<size_t>(BH) * Nq * d;
+  prm.lse_elems = static_cast<size_t>(BH) * Nq;
   if (d == 128)
     return causal ? fwd::launch<128, true, false>(tq, tk, tv, prm, grid, stream)
                   : fwd::launch<128, false, false>(tq, tk, tv, prm, grid, stream);
@@ -825,6 +1035,8 @@ fa_status launch_fwd_varlen(const void* q, const void* k, const void* v, void* o
   prm.o_head = static_cast<size_t>(d);
   prm.o_row = static_cast<size_t>(H) * d;
   prm.lse_head = static_cast<size_t>(total_q);
+  prm.o_elems = static_cast<size_t>(total_q) * H * d;
+  prm.lse_elems = static_cast<size_t>(H) * total_q;
   const int grid = static_cast<int>(items);
   if (d == 128)
     return causal ? fwd::launch<128, true, true>(tq, tk, tv, prm, grid, stream)
@@ -895,6 +1107,8 @@ fa_status launch_fwd_fp8(const void* q, const void* k, const void* vt, void* o, 
   prm.o_head = static_cast<size_t>(Nq) * d;
   prm.o_row = static_cast<size_t>(d);
   prm.lse_head = static_cast<size_t>(Nq);
+  prm.o_elems = static_cast<size_t>(BH) * Nq * d;
+  prm.lse_elems = static_cast<size_t>(BH) * Nq;
   return causal ? fwd::launch<128, true, false, true>(tq, tk, tv, prm, grid, stream)
                 : fwd::launch<128, false, false, true>(tq, tk, tv, prm, grid, stream);
 }

@@ -37,6 +37,20 @@ __device__ __forceinline__ void record_error(int code) {
   atomicCAS(&g_device_error, 0, code);
 }
 
+// Debug build (compiled with -DFA_DEBUG): every computed global address and
+// TMA coordinate is checked before it is used; a failed check records
+// FA_ERR_BOUNDS (6) in the device error word and the caller skips the access
+// (nothing traps).  In the normal build the check is the constant true and
+// compiles to nothing.
+#ifdef FA_DEBUG
+__device__ __forceinline__ bool dbg_ok(bool cond) {
+  if (!cond) record_error(6 /* FA_ERR_BOUNDS */);
+  return cond;
+}
+#else
+__device__ __forceinline__ constexpr bool dbg_ok(bool) { return true; }
+#endif
+
 // ------------------------------------------------------------------ mbarrier
 __device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
   asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count)
@@ -121,6 +135,8 @@ __device__ __forceinline__ void tma_prefetch_desc(const void* desc) {
 // 16-bit data so that the copy starts on a 16-byte boundary.
 __device__ __forceinline__ void tma_load_3d(void* smem_dst, const void* desc, uint64_t* bar,
                                             int c0, int c1, int c2) {
+  // every 3-D map here has 16-element aligned column boxes (64 bf16, 128 bytes)
+  if (!dbg_ok(c0 >= 0 && (c0 & 15) == 0)) return;
   asm volatile(
       "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
       " [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(smem_u32(smem_dst)),
@@ -133,6 +149,9 @@ __device__ __forceinline__ void tma_load_3d(void* smem_dst, const void* desc, ui
 // elements outside the tensor are skipped.
 __device__ __forceinline__ void tma_reduce_add_3d(const void* desc, const void* smem_src, int c0,
                                                   int c1, int c2) {
+  // a reduction must not start at a negative coordinate; fp32 boxes start on
+  // 16-byte boundaries
+  if (!dbg_ok(c0 >= 0 && (c0 & 3) == 0 && c1 >= 0 && c2 >= 0)) return;
   asm volatile(
       "cp.reduce.async.bulk.tensor.3d.global.shared::cta.add.bulk_group [%0, {%2, %3, %4}], [%1];"
       ::"l"(desc), "r"(smem_u32(smem_src)), "r"(c0), "r"(c1), "r"(c2)

@@ -23,7 +23,8 @@ _lib = None
 
 FA_OK = 0
 STATUS_NAMES = {0: "FA_OK", 1: "FA_ERR_INVALID_ARG", 2: "FA_ERR_UNSUPPORTED",
-                3: "FA_ERR_WORKSPACE", 4: "FA_ERR_CUDA", 5: "FA_ERR_TIMEOUT"}
+                3: "FA_ERR_WORKSPACE", 4: "FA_ERR_CUDA", 5: "FA_ERR_TIMEOUT",
+                6: "FA_ERR_BOUNDS"}
 
 # Public entry points and their C signatures (restype, argtypes).
 _P, _I, _F, _S = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t

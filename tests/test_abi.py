@@ -36,7 +36,7 @@ def test_library_exports_every_declared_symbol(fa_mod):
 
 
 def test_status_strings(fa_mod):
-    for code in range(6):
+    for code in range(7):
         assert fa_mod.status_string(code)
     assert fa_mod.lib().fa_version() >= 100
 
