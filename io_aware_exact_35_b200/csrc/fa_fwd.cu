@@ -131,7 +131,7 @@ __device__ __forceinline__ void mma_commit_w(uint64_t* bar) {
 namespace fwd {
 
 #ifndef FA_FWD_MMA_WARP
-#define FA_FWD_MMA_WARP 0
+#define FA_FWD_MMA_WARP 1
 #endif
 // 1: the whole MMA warp runs the issue loop converged (elect.sync per
 // instruction); 0: lane 0 alone runs it.
@@ -181,6 +181,30 @@ __device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t (&r)[8])
                  "r"(r[6]), "r"(r[7])
                : "memory");
 }
+
+// Two fp32 values rounded to bf16 (half away from zero: adding 2^15 to the
+// bit pattern carries into the kept half exactly when the dropped half is at
+// least one half-ulp) and packed, lo in the low half, with integer operations
+// only: the conversion instruction would share the MUFU/XU pipe with ex2.
+// Inputs are finite or +inf.
+__device__ __forceinline__ uint32_t pack_bf16x2_alu(float lo, float hi) {
+  return __byte_perm(__float_as_uint(lo) + 0x8000u, __float_as_uint(hi) + 0x8000u, 0x7632);
+}
+
+#ifndef FA_FWD_MAX_CHAINS
+#define FA_FWD_MAX_CHAINS 4
+#endif
+constexpr int MAX_CHAINS = FA_FWD_MAX_CHAINS;  // a power of two
+
+#ifndef FA_FWD_ST_AT_END
+#define FA_FWD_ST_AT_END 0
+#endif
+// 1: the softmax computes all of a row's P before storing it to tensor memory
+constexpr bool ST_AT_END = FA_FWD_ST_AT_END != 0;
+
+#ifndef FA_FWD_ALU_PACK
+#define FA_FWD_ALU_PACK 0
+#endif
 
 // acc += (a0, a1) lane by lane, one packed f32x2 addition.
 __device__ __forceinline__ void add_f32x2(uint64_t& acc, float a0, float a1) {
@@ -747,9 +771,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         const int key0 = j * BLOCK_N;
         const bool need_mask = (key0 + BLOCK_N > g.Nk) ||
                                (CAUSAL && key0 + BLOCK_N - 1 > q_row0 + g.off);
-        // four independent max chains (latency, not throughput, bounds this
-        // loop), each taking two new values per three-input max
-        float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+        // MAX_CHAINS independent max chains (latency, not throughput, bounds
+        // this loop), each taking two new values per three-input max
+        float mx[MAX_CHAINS];
+#pragma unroll
+        for (int i = 0; i < MAX_CHAINS; ++i) mx[i] = -INFINITY;
         if (need_mask) {
           // last admissible key (below 0: none, the row stays at -inf)
           const int lim = CAUSAL ? min(g.Nk - 1, row_g + g.off) : g.Nk - 1;
@@ -761,9 +787,14 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         }
 #pragma unroll
         for (int c = 0; c < 128; c += 2)
-          mx[(c >> 1) & 3] = fmax3(mx[(c >> 1) & 3], __uint_as_float(sr[c]), __uint_as_float(sr[c + 1]));
+          mx[(c >> 1) % MAX_CHAINS] =
+              fmax3(mx[(c >> 1) % MAX_CHAINS], __uint_as_float(sr[c]), __uint_as_float(sr[c + 1]));
+#pragma unroll
+        for (int h = MAX_CHAINS / 2; h >= 1; h /= 2)
+#pragma unroll
+          for (int i = 0; i < h; ++i) mx[i] = fmaxf(mx[i], mx[i + h]);
         // scale * log2(e) > 0, so the maximum of the scaled row is the scaled maximum
-        const float m_new = fmaxf(m, fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])) * sl2);
+        const float m_new = fmaxf(m, mx[0] * sl2);
         // true when m = -inf < m_new; false while the whole row is masked
         const bool grow = (m_new - m) > RESCALE_THRESHOLD;
         const bool warp_grow = __any_sync(0xffffffffu, grow);
@@ -803,6 +834,21 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         // x = s * scale * log2(e) - m for two keys per packed f32x2 FMA
         const uint64_t sl2_2 = pack_f32x2(sl2, sl2);
         const uint64_t negm_2 = pack_f32x2(-m_ref, -m_ref);
+        if constexpr (!F8 && ST_AT_END && !P_SPLIT) {
+          // all 128 probabilities first, then P in two 64-column stores
+          uint32_t pk[64];
+#pragma unroll
+          for (int e = 0; e < 128; e += 2) {
+            float x0, x1;
+            fma_f32x2(x0, x1, __uint_as_float(sr[e]), __uint_as_float(sr[e + 1]), sl2_2, negm_2);
+            const float p0 = ex2_approx(x0);
+            const float p1 = ex2_approx(x1);
+            add_f32x2(rs2[(e >> 1) & 3], p0, p1);
+            pk[e >> 1] = pack_bf16x2(p0, p1);
+          }
+          tmem_st32(tS, *reinterpret_cast<const uint32_t(*)[32]>(&pk[0]));
+          tmem_st32(tS + 32, *reinterpret_cast<const uint32_t(*)[32]>(&pk[32]));
+        } else
 #pragma unroll
         for (int c = 0; c < 128; c += 32) {
           uint32_t pk[16];
@@ -824,7 +870,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
               pf[e] = p0;
               pf[e + 1] = p1;
             } else {
-              pk[e >> 1] = pack_bf16x2(p0, p1);
+              pk[e >> 1] = FA_FWD_ALU_PACK ? pack_bf16x2_alu(p0, p1) : pack_bf16x2(p0, p1);
             }
           }
           if constexpr (F8) {

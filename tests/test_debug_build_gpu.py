@@ -77,7 +77,7 @@ check_o(od.cpu(), ro); check_lse(ld.cpu(), rl)
 check_o(op.cpu(), ro); check_lse(lp.cpu(), rl)
 
 # e4m3 forward
-q8, k8, vt8, (qs, ks, vs) = inputs.fp8_inputs(1, 2, 300, 128, seed=15)
+q8, k8, vt8, (qs, ks, vs) = inputs.fp8_inputs(1, 2, 300, 128, seed=15, Nk=304)
 o8, _ = fa.fwd_fp8(q8.to(dev), k8.to(dev), vt8.to(dev), qs, ks, vs, causal=True)
 clean()
 print("debug build ok")

@@ -8,7 +8,19 @@ derived from the e4m3 rounding of P: each probability carries an independent
 relative error of at most 2^-4 (uniform, sigma = 2^-4 / sqrt(3) = 0.036), and
 with O = sum P v / l that makes the relative L2 error of O about sigma.  The
 test allows 6e-2.  LSE comes from the f32 scores alone (products of e4m3
-values are exact in f32), so it keeps the bf16 path's 1e-3."""
+values are exact in f32), so it keeps the bf16 path's 1e-3.
+
+Each output element must also lie within a worst-case bound derived from the
+same arithmetic.  Write P_ij = p_ij / l_i for the exact probabilities.  The
+kernel exponentiates against a running maximum that is at most the row's
+true maximum, so its unnormalised p lie at or above p_ij / max_j p_ij and its
+row sum l is at least 1 / max_j P_ij.  Rounding one p to e4m3 errs by at most
+2^-4 of it in the normal range (>= 2^-6) and by at most 2^-10 below it
+(subnormal spacing 2^-9; values under 2^-10 flush to 0).  Hence
+  |O_ic - O*_ic| <= 2^-4 sum_j P_ij |v_jc|
+                    + 2^-10 max_j P_ij sum_{j: P_ij < 2^-6 max_j P_ij} |v_jc|
+                    + 2^-8 |O*_ic| (bf16 output) + 1e-5 (f32 sums),
+evaluated from the oracle's P (read out through V = identity)."""
 import numpy as np
 import pytest
 import torch
@@ -40,7 +52,23 @@ def _check(q8, k8, vt8, scales, causal, fa_mod, scale=None):
     rl = rel_l2(g, o_ref)
     assert rl <= FP8_O_REL_L2, f"O relative L2 {rl:.3e} > {FP8_O_REL_L2}"
     check_lse(lse.cpu(), lse_ref)
+    bound = _fp8_o_bound(q, k, v, o_ref, causal, scale)
+    err = np.abs(g - o_ref)
+    worst = float(np.max(err - bound))
+    assert worst <= 0.0, f"O exceeds the e4m3 worst-case bound by {worst:.3e}"
     return rl
+
+
+def _fp8_o_bound(q, k, v, o_ref, causal, scale):
+    """Element-wise worst-case error bound of the e4m3 forward (module doc)."""
+    nk, hkv, H = k.shape[-2], k.shape[1], q.shape[1]
+    eye = np.broadcast_to(np.eye(nk), (k.shape[0], hkv, nk, nk)).copy()
+    P, _ = oracle.attention_forward(q, k, eye, causal, scale)   # [B, H, Nq, Nk]
+    absv = oracle.expand_kv_heads(np.abs(v), H)                 # [B, H, Nk, d]
+    pmax = P.max(axis=-1, keepdims=True)
+    small = (P < 2.0 ** -6 * pmax).astype(np.float64)
+    return (2.0 ** -4 * (P @ absv) + 2.0 ** -10 * pmax * (small @ absv)
+            + 2.0 ** -8 * np.abs(o_ref) + 1e-5)
 
 
 CASES = [  # (B, H, Hkv, Nq, Nk); Nk is a multiple of 16 (rows of vt)
