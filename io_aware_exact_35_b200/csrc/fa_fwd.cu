@@ -196,6 +196,20 @@ __device__ __forceinline__ uint32_t pack_bf16x2_alu(float lo, float hi) {
 #endif
 constexpr int MAX_CHAINS = FA_FWD_MAX_CHAINS;  // a power of two
 
+#ifndef FA_FWD_WARP_ARRIVE
+#define FA_FWD_WARP_ARRIVE 1
+#endif
+// 1: the softmax signals P ready with one arrival per warp (after the warp's
+// lanes have synchronised) instead of one per thread
+constexpr bool WARP_ARRIVE = FA_FWD_WARP_ARRIVE != 0;
+constexpr int P_ARRIVALS = WARP_ARRIVE ? TILE_M / 32 : TILE_M;
+
+#ifndef FA_FWD_LANE0_WAIT
+#define FA_FWD_LANE0_WAIT 0
+#endif
+// 1: one lane of each softmax warp polls for S, then the warp synchronises
+constexpr bool LANE0_WAIT = FA_FWD_LANE0_WAIT != 0;
+
 #ifndef FA_FWD_ST_AT_END
 #define FA_FWD_ST_AT_END 0
 #endif
@@ -453,13 +467,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     }
     for (int w = 0; w < NQ; ++w) {
       mbar_init(&s_full[w], 1);
-      mbar_init(&p_full[w], TILE_M);
+      mbar_init(&p_full[w], P_ARRIVALS);
       mbar_init(&o_done[w], 1);
       mbar_init(&o_final[w], 1);
       mbar_init(&o_free[w], TILE_M);
       mbar_init(&l_ready[2 * w], TILE_M);
       mbar_init(&l_ready[2 * w + 1], TILE_M);
-      mbar_init(&p_half[w], TILE_M);
+      mbar_init(&p_half[w], P_ARRIVALS);
     }
     mbar_init(mma_final, 1);
     *abort_flag = 0;
@@ -756,7 +770,15 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       float m = -INFINITY;  // running max of scale * log2(e) * s
       float l = 0.f;
       for (int j = 0; j < n_kv; ++j) {
-        if (!mbar_wait_warp(&s_full[w], scount & 1, abort_flag)) {
+        bool s_ok;
+        if constexpr (LANE0_WAIT) {
+          s_ok = lane == 0 ? mbar_wait(&s_full[w], scount & 1, abort_flag) : true;
+          s_ok = __shfl_sync(0xffffffffu, s_ok, 0);
+          __syncwarp();
+        } else {
+          s_ok = mbar_wait_warp(&s_full[w], scount & 1, abort_flag);
+        }
+        if (!s_ok) {
           ok = false;
           break;
         }
@@ -894,7 +916,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             if constexpr (F8) fence_proxy_async_smem();
             else tmem_st_wait();
             tc_fence_before();
-            mbar_arrive(&p_half[w]);
+            if (WARP_ARRIVE) __syncwarp();
+            if (!WARP_ARRIVE || lane == 0) mbar_arrive(&p_half[w]);
           }
         }
         // e4m3 P is read by the async proxy (tensor core) from shared memory
@@ -904,7 +927,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         m = m_use;
         tmem_st_wait();
         tc_fence_before();
-        mbar_arrive(&p_full[w]);
+        if (WARP_ARRIVE) __syncwarp();
+        if (!WARP_ARRIVE || lane == 0) mbar_arrive(&p_full[w]);
       }
       if (!ok) break;
       // End of the work item for this tile: LSE, and 1 / l for the epilogue
