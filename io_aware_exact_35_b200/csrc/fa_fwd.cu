@@ -130,13 +130,6 @@ __device__ __forceinline__ void mma_commit_w(uint64_t* bar) {
 
 namespace fwd {
 
-#ifndef FA_FWD_MMA_WARP
-#define FA_FWD_MMA_WARP 1
-#endif
-// 1: the whole MMA warp runs the issue loop converged (elect.sync per
-// instruction); 0: lane 0 alone runs it.
-constexpr bool MMA_WARP = FA_FWD_MMA_WARP != 0;
-
 constexpr int TILE_M = 128;   // rows per softmax warpgroup
 constexpr int NQ = 2;         // query tiles per CTA
 constexpr int BLOCK_M = TILE_M * NQ;
@@ -145,11 +138,16 @@ constexpr int NUM_THREADS = 512;
 constexpr int WARP_PRODUCER = 12;
 constexpr int WARP_MMA = 13;
 // Registers per thread after setmaxnreg (launch: 65536 / 512 = 128 each):
-// 2 x 128 x 184 + 128 x 48 + 128 x 96 = 65536 (the producer / MMA warpgroup
-// needs more than the epilogue: its issue loops keep many descriptors live).
+// 2 x 128 x 184 + 128 x 48 + 128 x 96 = 65536.  The producer / MMA warpgroup
+// needs 96: its issue loops are fully unrolled with precomputed descriptors,
+// because the issue of a tensor-core instruction waits until the tensor pipe
+// accepts it, so any instruction between two of them lengthens every step
+// (measured: rolled loops made the forward 12% slower).
 constexpr int REGS_SOFTMAX = 184;
 constexpr int REGS_EPILOGUE = 48;
 constexpr int REGS_OTHER = 96;
+static_assert(2 * 128 * REGS_SOFTMAX + 128 * REGS_EPILOGUE + 128 * REGS_OTHER <= 65536,
+              "setmaxnreg.inc would wait forever: the split exceeds the launch's registers");
 constexpr int PANEL_BYTES = 128 * 128;   // 128 rows x 64 bf16 (one swizzle panel)
 constexpr uint32_t TMEM_COLS = 512;
 constexpr float RESCALE_THRESHOLD = 8.0f;  // log2 units
@@ -182,43 +180,11 @@ __device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t (&r)[8])
                : "memory");
 }
 
-// Two fp32 values rounded to bf16 (half away from zero: adding 2^15 to the
-// bit pattern carries into the kept half exactly when the dropped half is at
-// least one half-ulp) and packed, lo in the low half, with integer operations
-// only: the conversion instruction would share the MUFU/XU pipe with ex2.
-// Inputs are finite or +inf.
-__device__ __forceinline__ uint32_t pack_bf16x2_alu(float lo, float hi) {
-  return __byte_perm(__float_as_uint(lo) + 0x8000u, __float_as_uint(hi) + 0x8000u, 0x7632);
-}
-
-#ifndef FA_FWD_MAX_CHAINS
-#define FA_FWD_MAX_CHAINS 4
-#endif
-constexpr int MAX_CHAINS = FA_FWD_MAX_CHAINS;  // a power of two
-
-#ifndef FA_FWD_WARP_ARRIVE
-#define FA_FWD_WARP_ARRIVE 1
-#endif
-// 1: the softmax signals P ready with one arrival per warp (after the warp's
-// lanes have synchronised) instead of one per thread
-constexpr bool WARP_ARRIVE = FA_FWD_WARP_ARRIVE != 0;
-constexpr int P_ARRIVALS = WARP_ARRIVE ? TILE_M / 32 : TILE_M;
-
-#ifndef FA_FWD_LANE0_WAIT
-#define FA_FWD_LANE0_WAIT 0
-#endif
-// 1: one lane of each softmax warp polls for S, then the warp synchronises
-constexpr bool LANE0_WAIT = FA_FWD_LANE0_WAIT != 0;
-
-#ifndef FA_FWD_ST_AT_END
-#define FA_FWD_ST_AT_END 0
-#endif
-// 1: the softmax computes all of a row's P before storing it to tensor memory
-constexpr bool ST_AT_END = FA_FWD_ST_AT_END != 0;
-
-#ifndef FA_FWD_ALU_PACK
-#define FA_FWD_ALU_PACK 0
-#endif
+// The softmax signals "P ready" with one arrival per warp (after the warp's
+// lanes have synchronised), not one per thread: 4 arrivals per step instead
+// of 128 on the same barrier.
+constexpr int P_ARRIVALS = TILE_M / 32;
+constexpr int MAX_CHAINS = 4;  // independent chains of the row maximum
 
 // acc += (a0, a1) lane by lane, one packed f32x2 addition.
 __device__ __forceinline__ void add_f32x2(uint64_t& acc, float a0, float a1) {
@@ -265,12 +231,6 @@ __device__ __forceinline__ void ex2_poly3_x2(float x0, float x1, float& y0, floa
 #define FA_FWD_EMU_PAIRS 0
 #endif
 constexpr int EMU_PAIRS = FA_FWD_EMU_PAIRS;  // of every 4 exp pairs, on the FMA pipe
-#ifndef FA_FWD_P_SPLIT
-#define FA_FWD_P_SPLIT 0
-#endif
-// P handed to the tensor core in two halves (keys 0-63, then 64-127), so that
-// the first half of O += P V runs while the second half is exponentiated.
-constexpr bool P_SPLIT = FA_FWD_P_SPLIT != 0;
 
 // Shared-memory plan.  A panel is 128 rows x 128 bytes (64 bf16 or 128 e4m3
 // values per row).  With 8-bit inputs (F8) the ring carries K_j and V_j^T
@@ -286,9 +246,9 @@ struct Smem {
   static constexpr int P_OFF = RING_OFF + NSLOT * TILE;  // F8: NQ tiles of 128 x 128 e4m3
   static constexpr int BAR_OFF = P_OFF + (F8 ? NQ * PANEL_BYTES : 0);
   // barriers: q_full, q_empty, full[NSLOT], empty[NSLOT],
-  //           s_full[NQ], p_full[NQ], o_done[NQ], o_final[NQ], o_free[NQ], mma_final,
-  //           l_ready[NQ][2], p_half[NQ]
-  static constexpr int NBAR = 2 + 2 * NSLOT + 5 * NQ + 1 + 2 * NQ + NQ;
+  //           s_full[NQ], p_full[NQ], o_final[NQ], o_free[NQ], mma_final,
+  //           l_ready[NQ][2]
+  static constexpr int NBAR = 2 + 2 * NSLOT + 4 * NQ + 1 + 2 * NQ;
   // 1 / l of every row, per query tile, for work items of even / odd index
   static constexpr int STAT_OFF = BAR_OFF + NBAR * 8;
   static constexpr int MISC_OFF = STAT_OFF + 2 * NQ * TILE_M * 4;
@@ -426,12 +386,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   uint64_t* empty = full + NSLOT;   // [NSLOT] ring slot consumed
   uint64_t* s_full = empty + NSLOT; // [NQ]
   uint64_t* p_full = s_full + NQ;   // [NQ]
-  uint64_t* o_done = p_full + NQ;   // [NQ] one phase per O += P V
-  uint64_t* o_final = o_done + NQ;  // [NQ] one phase per work item: its last O += P V
+  uint64_t* o_final = p_full + NQ;  // [NQ] one phase per work item: its last O += P V
   uint64_t* o_free = o_final + NQ;  // [NQ] one phase per work item: O read out
   uint64_t* mma_final = o_free + NQ;
   uint64_t* l_ready = mma_final + 1;  // [NQ][2]: 1 / l written, per item parity
-  uint64_t* p_half = l_ready + 2 * NQ;  // [NQ]: first half of P written (P_SPLIT)
   float* inv_l_buf = reinterpret_cast<float*>(smem + L::STAT_OFF);  // [2][NQ][TILE_M]
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::MISC_OFF);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::MISC_OFF + 4);
@@ -468,12 +426,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     for (int w = 0; w < NQ; ++w) {
       mbar_init(&s_full[w], 1);
       mbar_init(&p_full[w], P_ARRIVALS);
-      mbar_init(&o_done[w], 1);
       mbar_init(&o_final[w], 1);
       mbar_init(&o_free[w], TILE_M);
       mbar_init(&l_ready[2 * w], TILE_M);
       mbar_init(&l_ready[2 * w + 1], TILE_M);
-      mbar_init(&p_half[w], P_ARRIVALS);
     }
     mbar_init(mma_final, 1);
     *abort_flag = 0;
@@ -547,16 +503,14 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     }
    } else if (warp == WARP_MMA) {
     // ------------------------------------------------------------ MMA issuer
-    if (MMA_WARP || lane == 0) {
-      // waits of the issue loop: warp-collective when the whole warp runs it
+    {
+      // The whole warp runs the issue loop converged, and elect.sync picks
+      // the lane that issues each tensor-core instruction: lane 0 alone
+      // (a divergent branch) issued measurably slower.
       auto mwait = [&](uint64_t* bar, uint32_t parity) {
-        if constexpr (MMA_WARP) return mbar_wait_warp(bar, parity, abort_flag);
-        else return mbar_wait(bar, parity, abort_flag);
+        return mbar_wait_warp(bar, parity, abort_flag);
       };
-      auto commit = [&](uint64_t* bar) {
-        if constexpr (MMA_WARP) mma_commit_w(bar);
-        else mma_commit(bar);
-      };
+      auto commit = [&](uint64_t* bar) { mma_commit_w(bar); };
       constexpr uint32_t IDESC_S =
           F8 ? idesc_e4m3_f32(TILE_M, BLOCK_N) : idesc_bf16_f32(TILE_M, BLOCK_N, false, false);
       constexpr uint32_t IDESC_O =
@@ -583,15 +537,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 #pragma unroll
           for (int kk = 0; kk < D / 32; ++kk) {  // 32 e4m3 = 32 bytes per step
             const uint64_t off = static_cast<uint64_t>(((kk >> 2) * PANEL_BYTES + (kk & 3) * 32) >> 4);
-            if constexpr (MMA_WARP) mma_f8_ss_w(dS, qd + off, kd + off, IDESC_S, kk > 0 ? 1u : 0u);
-            else mma_f8_ss(dS, qd + off, kd + off, IDESC_S, kk > 0 ? 1u : 0u);
+            mma_f8_ss_w(dS, qd + off, kd + off, IDESC_S, kk > 0 ? 1u : 0u);
           }
         } else {
 #pragma unroll
           for (int kk = 0; kk < D / 16; ++kk) {
             const uint64_t off = static_cast<uint64_t>(((kk >> 2) * PANEL_BYTES + (kk & 3) * 32) >> 4);
-            if constexpr (MMA_WARP) mma_bf16_ss_w(dS, qd + off, kd + off, IDESC_S, kk > 0 ? 1u : 0u);
-            else mma_bf16_ss(dS, qd + off, kd + off, IDESC_S, kk > 0 ? 1u : 0u);
+            mma_bf16_ss_w(dS, qd + off, kd + off, IDESC_S, kk > 0 ? 1u : 0u);
           }
         }
         commit(&s_full[w]);
@@ -608,10 +560,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 #pragma unroll
             for (int kk = kk0; kk < kk1; ++kk) {
               const uint64_t off = static_cast<uint64_t>((kk * 32) >> 4);
-              if constexpr (MMA_WARP)
-                mma_f8_ss_w(tO, pd + off, vd + off, IDESC_O, (!first || kk > 0) ? 1u : 0u);
-              else
-                mma_f8_ss(tO, pd + off, vd + off, IDESC_O, (!first || kk > 0) ? 1u : 0u);
+              mma_f8_ss_w(tO, pd + off, vd + off, IDESC_O, (!first || kk > 0) ? 1u : 0u);
             }
           } else {
             const uint64_t vd = ring_vdesc0 + static_cast<uint64_t>((slot * L::TILE) >> 4);
@@ -620,29 +569,15 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             for (int kk = kk0; kk < kk1; ++kk) {
               // keys 16kk .. 16kk+15: P columns 8kk.., V rows 16kk.. (2048 bytes per step)
               const uint64_t vdk = vd + static_cast<uint64_t>((kk * 2048) >> 4);
-              if constexpr (MMA_WARP)
-                mma_bf16_ts_w(tO, tP + kk * 8, vdk, IDESC_O, (!first || kk > 0) ? 1u : 0u);
-              else
-                mma_bf16_ts(tO, tP + kk * 8, vdk, IDESC_O, (!first || kk > 0) ? 1u : 0u);
+              mma_bf16_ts_w(tO, tP + kk * 8, vdk, IDESC_O, (!first || kk > 0) ? 1u : 0u);
             }
           }
         };
         constexpr int KK = F8 ? BLOCK_N / 32 : BLOCK_N / 16;
-        if constexpr (P_SPLIT) {
-          if (!mwait(&p_half[w], pcount[w] & 1)) return false;
-          tc_fence_after();
-          pv_range(0, KK / 2);
-          if (!mwait(&p_full[w], pcount[w] & 1)) return false;
-          ++pcount[w];
-          tc_fence_after();
-          pv_range(KK / 2, KK);
-        } else {
-          if (!mwait(&p_full[w], pcount[w] & 1)) return false;
-          ++pcount[w];
-          tc_fence_after();
-          pv_range(0, KK);
-        }
-        commit(&o_done[w]);
+        if (!mwait(&p_full[w], pcount[w] & 1)) return false;
+        ++pcount[w];
+        tc_fence_after();
+        pv_range(0, KK);
         if (last) commit(&o_final[w]);
         return true;
       };
@@ -758,7 +693,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     const uint32_t tO = tmem_base + 256 + w * 128 + lane_off;
     const float sl2 = p.scale_log2;
     int scount = 0;   // S tiles consumed (all items)
-    int pv_base = 0;  // O += P V products of previous items
     bool ok = true;
     for (int k = 0; ok; ++k) {
       const int item = cta_item(cta, k, G);
@@ -770,15 +704,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       float m = -INFINITY;  // running max of scale * log2(e) * s
       float l = 0.f;
       for (int j = 0; j < n_kv; ++j) {
-        bool s_ok;
-        if constexpr (LANE0_WAIT) {
-          s_ok = lane == 0 ? mbar_wait(&s_full[w], scount & 1, abort_flag) : true;
-          s_ok = __shfl_sync(0xffffffffu, s_ok, 0);
-          __syncwarp();
-        } else {
-          s_ok = mbar_wait_warp(&s_full[w], scount & 1, abort_flag);
-        }
-        if (!s_ok) {
+        if (!mbar_wait_warp(&s_full[w], scount & 1, abort_flag)) {
           ok = false;
           break;
         }
@@ -828,14 +754,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         const float alpha = warp_grow ? ex2_approx(m - m_ref) : 1.f;
         if (warp_grow && j > 0) {
           // O holds P_0 V_0 + ... + P_{j-1} V_{j-1} relative to the old max:
-          // rescale it before this step's P is handed over.  S_w,j was issued
-          // after O_w += P_{j-1} V_{j-1}, so o_done[w] has completed exactly
-          // pv_base + j times; the wait only confirms it.
-          if (!mbar_wait_warp(&o_done[w], (pv_base + j - 1) & 1, abort_flag)) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
+          // rescale it before this step's P is handed over.  It is complete:
+          // S_w,j was issued after O_w += P_{j-1} V_{j-1} by the same thread,
+          // and the commit that signalled S_w,j covers every tensor-core
+          // operation that thread issued before it.
           // eight columns at a time: S is still live in registers here
 #pragma unroll 1
           for (int c = 0; c < D; c += 8) {
@@ -856,70 +778,59 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         // x = s * scale * log2(e) - m for two keys per packed f32x2 FMA
         const uint64_t sl2_2 = pack_f32x2(sl2, sl2);
         const uint64_t negm_2 = pack_f32x2(-m_ref, -m_ref);
-        if constexpr (!F8 && ST_AT_END && !P_SPLIT) {
-          // all 128 probabilities first, then P in two 64-column stores
-          uint32_t pk[64];
+        // Exponentials: MUFU ex2, except that in tiles without masked keys
+        // EMU_PAIRS of every 4 key pairs go to the FMA-pipe polynomial (masked
+        // keys must give exactly 0, which only ex2 of -inf does).  The two
+        // cases are separate loop bodies, so that the choice per pair is a
+        // compile-time one.
+        auto exps = [&](auto emu_c) {
+          constexpr int EMU = decltype(emu_c)::value;
 #pragma unroll
-          for (int e = 0; e < 128; e += 2) {
-            float x0, x1;
-            fma_f32x2(x0, x1, __uint_as_float(sr[e]), __uint_as_float(sr[e + 1]), sl2_2, negm_2);
-            const float p0 = ex2_approx(x0);
-            const float p1 = ex2_approx(x1);
-            add_f32x2(rs2[(e >> 1) & 3], p0, p1);
-            pk[e >> 1] = pack_bf16x2(p0, p1);
-          }
-          tmem_st32(tS, *reinterpret_cast<const uint32_t(*)[32]>(&pk[0]));
-          tmem_st32(tS + 32, *reinterpret_cast<const uint32_t(*)[32]>(&pk[32]));
-        } else
+          for (int c = 0; c < 128; c += 32) {
+            uint32_t pk[16];  // bf16 P
+            float pf[32];     // e4m3 P, before rounding
+            (void)pk;
+            (void)pf;
 #pragma unroll
-        for (int c = 0; c < 128; c += 32) {
-          uint32_t pk[16];
-          float pf[32];
-#pragma unroll
-          for (int e = 0; e < 32; e += 2) {
-            float x0, x1;
-            fma_f32x2(x0, x1, __uint_as_float(sr[c + e]), __uint_as_float(sr[c + e + 1]), sl2_2,
-                      negm_2);
-            float p0, p1;
-            if (((e >> 1) & 3) >= 4 - EMU_PAIRS && !need_mask) {
-              ex2_poly3_x2(x0, x1, p0, p1);
-            } else {
-              p0 = ex2_approx(x0);
-              p1 = ex2_approx(x1);
+            for (int e = 0; e < 32; e += 2) {
+              float x0, x1;
+              fma_f32x2(x0, x1, __uint_as_float(sr[c + e]), __uint_as_float(sr[c + e + 1]), sl2_2,
+                        negm_2);
+              float p0, p1;
+              if (((e >> 1) & 3) >= 4 - EMU) {
+                ex2_poly3_x2(x0, x1, p0, p1);
+              } else {
+                p0 = ex2_approx(x0);
+                p1 = ex2_approx(x1);
+              }
+              add_f32x2(rs2[(e >> 1) & 3], p0, p1);
+              if constexpr (F8) {
+                pf[e] = p0;
+                pf[e + 1] = p1;
+              } else {
+                pk[e >> 1] = pack_bf16x2(p0, p1);
+              }
             }
-            add_f32x2(rs2[(e >> 1) & 3], p0, p1);
             if constexpr (F8) {
-              pf[e] = p0;
-              pf[e + 1] = p1;
-            } else {
-              pk[e >> 1] = FA_FWD_ALU_PACK ? pack_bf16x2_alu(p0, p1) : pack_bf16x2(p0, p1);
-            }
-          }
-          if constexpr (F8) {
-            // keys c .. c+31 of row `row`: two 16-byte chunks of the 128-byte
-            // row, 128-byte swizzle (chunk index xor row % 8)
-            uint8_t* prow = smem + L::P_OFF + w * PANEL_BYTES + row * 128;
+              // keys c .. c+31 of row `row`: two 16-byte chunks of the 128-byte
+              // row, 128-byte swizzle (chunk index xor row % 8)
+              uint8_t* prow = smem + L::P_OFF + w * PANEL_BYTES + row * 128;
 #pragma unroll
-            for (int h = 0; h < 2; ++h) {
-              const uint32_t ch = static_cast<uint32_t>((c >> 4) + h) ^ static_cast<uint32_t>(row & 7);
-              const float* f = pf + 16 * h;
-              *reinterpret_cast<uint4*>(prow + ch * 16) =
-                  make_uint4(pack_e4m3x4(f[0], f[1], f[2], f[3]), pack_e4m3x4(f[4], f[5], f[6], f[7]),
-                             pack_e4m3x4(f[8], f[9], f[10], f[11]),
-                             pack_e4m3x4(f[12], f[13], f[14], f[15]));
+              for (int h = 0; h < 2; ++h) {
+                const uint32_t ch =
+                    static_cast<uint32_t>((c >> 4) + h) ^ static_cast<uint32_t>(row & 7);
+                const float* f = pf + 16 * h;
+                *reinterpret_cast<uint4*>(prow + ch * 16) = make_uint4(
+                    pack_e4m3x4(f[0], f[1], f[2], f[3]), pack_e4m3x4(f[4], f[5], f[6], f[7]),
+                    pack_e4m3x4(f[8], f[9], f[10], f[11]), pack_e4m3x4(f[12], f[13], f[14], f[15]));
+              }
+            } else {
+              tmem_st16(tS + (c >> 1), pk);
             }
-          } else {
-            tmem_st16(tS + (c >> 1), pk);
           }
-          if (P_SPLIT && c == 32) {
-            // keys 0-63 of P are written: the first half of O += P V may start
-            if constexpr (F8) fence_proxy_async_smem();
-            else tmem_st_wait();
-            tc_fence_before();
-            if (WARP_ARRIVE) __syncwarp();
-            if (!WARP_ARRIVE || lane == 0) mbar_arrive(&p_half[w]);
-          }
-        }
+        };
+        if (EMU_PAIRS > 0 && !need_mask) exps(std::integral_constant<int, EMU_PAIRS>{});
+        else exps(std::integral_constant<int, 0>{});
         // e4m3 P is read by the async proxy (tensor core) from shared memory
         if constexpr (F8) fence_proxy_async_smem();
         l = l * alpha + ((sum_f32x2(rs2[0]) + sum_f32x2(rs2[1])) +
@@ -927,8 +838,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         m = m_use;
         tmem_st_wait();
         tc_fence_before();
-        if (WARP_ARRIVE) __syncwarp();
-        if (!WARP_ARRIVE || lane == 0) mbar_arrive(&p_full[w]);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&p_full[w]);
       }
       if (!ok) break;
       // End of the work item for this tile: LSE, and 1 / l for the epilogue
@@ -945,7 +856,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         const float lse = (l > 0.f) ? (m + lg2_approx(l)) * 0.6931471805599453f : -INFINITY;
         p.lse[static_cast<size_t>(g.head) * p.lse_head + g.q0 + row_g] = lse;
       }
-      pv_base += n_kv;
     }
     tmem_ld_wait();
     tmem_st_wait();
