@@ -28,10 +28,14 @@
 //              V_j through one ring of NSLOT tile-sized slots that holds K and
 //              V tiles in the order they are consumed (K_0 V_0 K_1 V_1 ...), so
 //              loads run about two key tiles ahead of the tensor core.
-//   warp 13    tensor-memory allocator and MMA issuer (one thread).  The two
+//   warp 13    tensor-memory allocator and MMA issuer (the whole warp runs
+//              converged; elect.sync picks the lane that issues).  The two
 //              query tiles ping-pong: while warpgroup 0 exponentiates S_0,j the
 //              tensor core runs O_1 += P_1 V_{j-1} and S_1,j, and vice versa:
 //                S0(0) S1(0) | PV0(0) S0(1) PV1(0) S1(1) | PV0(1) S0(2) ...
+//              Since S_w(j+1) is written over the columns that hold P_w(j), it
+//              follows O_w += P_w(j) V_j: per tile, softmax, P V and the next
+//              S run in series, and the two tiles overlap their chains.
 //   warps 14-15 idle (they complete the fourth warpgroup).
 //
 // Tensor memory (512 columns x 128 lanes, fp32): S_0 [0,128), S_1 [128,256),
