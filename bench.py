@@ -372,27 +372,58 @@ def time_main_kernel(r, steps, world, dev):
 
 
 def time_e2e(r, steps, warmup, world, dev):
-    """End-to-end through the public API: pinned host -> device, the call, and
-    the result back to the host, every step."""
+    """End-to-end through the public API: every step copies its inputs from
+    pinned host memory to the device, makes the call, and copies its results
+    back to pinned host memory.  Steps are pipelined as a user streaming
+    batches would run them: inputs are double-buffered on a copy-in stream,
+    the calls run on a compute stream and the results go back on a copy-out
+    stream, so step k+1's inputs travel while step k computes and its results
+    travel back (both directions of the host link at once).  Events order the
+    reuse of every buffer; the timed region runs from the first copy in to
+    the last copy out."""
     host = [t.pin_memory() for t in r.host]
-    dbufs = [torch.empty_like(t, device=dev) for t in r.host]
+    dbufs = [[torch.empty_like(t, device=dev) for t in r.host] for _ in range(2)]
     h2d = sum(t.numel() * t.element_size() for t in host)
     d2h = sum(t.numel() * t.element_size() for t in r.out_host)
+    s_in, s_comp, s_out = torch.cuda.Stream(), torch.cuda.Stream(), torch.cuda.Stream()
+    comp_done = [torch.cuda.Event() for _ in range(2)]  # buffer k % 2 free again
+    in_done = [torch.cuda.Event() for _ in range(2)]
+    out_done = torch.cuda.Event()                       # results of the last step read
+    state = {"k": 0}
 
     def one():
-        for hb, db in zip(host, dbufs):
-            db.copy_(hb, non_blocking=True)
-        for out, oh in zip(r.step(dbufs), r.out_host):
-            oh.copy_(out, non_blocking=True)
+        k = state["k"]
+        b = k & 1
+        with torch.cuda.stream(s_in):
+            if k >= 2:
+                s_in.wait_event(comp_done[b])  # the call of step k-2 has read buffer b
+            for hb, db in zip(host, dbufs[b]):
+                db.copy_(hb, non_blocking=True)
+            in_done[b].record(s_in)
+        with torch.cuda.stream(s_comp):
+            s_comp.wait_event(in_done[b])
+            if k >= 1:
+                s_comp.wait_event(out_done)    # step k-1's results have left the outputs
+            outs = r.step(dbufs[b])
+            comp_done[b].record(s_comp)
+        with torch.cuda.stream(s_out):
+            s_out.wait_event(comp_done[b])
+            for out, oh in zip(outs, r.out_host):
+                oh.copy_(out, non_blocking=True)
+            out_done.record(s_out)
+        state["k"] = k + 1
 
     for _ in range(max(1, warmup)):
         one()
+    torch.cuda.synchronize()
     barrier(world)
     st, en = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    st.record()
+    st.record(s_in)
+    s_in.wait_event(out_done)  # start from an idle pipeline
     for _ in range(steps):
         one()
-    en.record()
+    en.record(s_out)
+    torch.cuda.synchronize()
     barrier(world)
     sec = max_over_ranks(st.elapsed_time(en) * 1e-3 / steps, world, dev)
     return sec, h2d, d2h
