@@ -328,9 +328,16 @@ def time_device(r, steps, warmup, world, dev):
         r.step()
     starts = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
     ends = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    for ev in starts + ends:
+        ev.record(stream)  # creates the CUDA event behind it, outside the timed loop
     sampler = ClockSampler(dev.index or 0)
     sampler.start()
     time.sleep(0.3)
+    # the sampler's start-up left the GPU idle: bring it back to speed
+    for _ in range(min(warmup, 3)):
+        if r.flush is not None:
+            r.flush.zero_()
+        r.step()
     barrier(world)
     t0 = time.perf_counter()
     for i in range(steps):
