@@ -274,6 +274,10 @@ struct Params {
                      // the longest sequence (ragged batch)
   int total_items;   // BH * n_cta_tiles
   int lpt_order;     // 1: all heads' longest tiles first; 0: head-major
+  // 1: a work item is one 128-row tile of two query heads that share a
+  // key/value head (grouped heads, an even group); item coordinates then count
+  // head pairs and 128-row tiles.  0: two consecutive 128-row tiles of one head.
+  int pair_heads;
   float scale_log2;  // scale * log2(e) (times the q and k descales for e4m3)
   float o_scale;     // multiplies O / l: 1, or the v descale for e4m3
   // ragged batch (token-major packing): sequence b owns rows cu_q[b] ..
@@ -289,7 +293,7 @@ struct Params {
   size_t o_elems, lse_elems;  // sizes of O and LSE, for the debug build's checks
 };
 
-// Work item -> (batch*head, 256-row tile).  In LPT order the longest tiles of
+// Work item -> (batch*head (or head pair), query tile).  In LPT order the longest tiles of
 // every head come first (good balance; used when all K/V fit in L2); in
 // head-major order the tiles of one head are adjacent, longest first (K/V of
 // the resident CTAs stay in L2 for long sequences).
@@ -307,8 +311,12 @@ __device__ __forceinline__ void item_coords(const Params& p, int item, int& bh, 
 // Where a work item lives.  Rows are counted within the sequence; q0 / k0 are
 // the sequence's first rows in the tensor maps (0 for the padded layout).
 struct ItemGeo {
-  int tile;        // 256-row query tile of the sequence
-  int head;        // head coordinate of Q / O / LSE
+  int tile;        // query tile of the sequence (256 rows, or 128 with paired heads)
+  // query tile w starts at row qrow0 + w * qstep of the sequence and has the
+  // head coordinate (of Q / O / LSE) hd0 + w * hstep
+  int qrow0, qstep, hd0, hstep;
+  __device__ __forceinline__ int qrow(int w) const { return qrow0 + w * qstep; }
+  __device__ __forceinline__ int hd(int w) const { return hd0 + w * hstep; }
   int kv_head;     // head coordinate of K / V
   int q0, k0;
   int Nq, Nk, off; // lengths of the sequence and Nk - Nq
@@ -321,8 +329,24 @@ __device__ __forceinline__ ItemGeo item_geo(const Params& p, int item) {
   int bh;
   item_coords(p, item, bh, g.tile);
   if constexpr (!VARLEN) {
-    g.head = bh;
-    g.kv_head = bh / p.group;
+    if (p.pair_heads) {
+      // bh counts head pairs: heads 2i and 2i+1 of one batch row, the same
+      // rows of both, one key/value head (the group is even)
+      const int half = p.H >> 1;
+      const int b = bh / half;
+      const int h0 = b * p.H + 2 * (bh - b * half);
+      g.hd0 = h0;
+      g.hstep = 1;
+      g.qrow0 = g.tile * TILE_M;
+      g.qstep = 0;
+      g.kv_head = h0 / p.group;
+    } else {
+      g.hd0 = bh;
+      g.hstep = 0;
+      g.qrow0 = g.tile * BLOCK_M;
+      g.qstep = TILE_M;
+      g.kv_head = bh / p.group;
+    }
     g.q0 = 0;
     g.k0 = 0;
     g.Nq = p.Nq;
@@ -330,7 +354,10 @@ __device__ __forceinline__ ItemGeo item_geo(const Params& p, int item) {
   } else {
     const int b = bh / p.H;
     const int h = bh - b * p.H;
-    g.head = h;
+    g.hd0 = h;
+    g.hstep = 0;
+    g.qrow0 = g.tile * BLOCK_M;
+    g.qstep = TILE_M;
     g.kv_head = h / p.group;
     g.q0 = p.cu_q[b];
     g.k0 = p.cu_k[b];
@@ -408,7 +435,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   // pipeline once and come out fully masked: O = 0, LSE = -inf.
   auto n_kv_of = [&](const ItemGeo& g, int w) {
     if (!CAUSAL) return g.n_kv_total;
-    const int last_key = g.tile * BLOCK_M + w * TILE_M + TILE_M - 1 + g.off;
+    const int last_key = g.qrow(w) + TILE_M - 1 + g.off;
     return last_key < 0 ? 1 : min(last_key / BLOCK_N + 1, g.n_kv_total);
   };
   if constexpr (VARLEN) {
@@ -473,7 +500,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         for (int w = 0; w < NQ; ++w)
           for (int pn = 0; pn < L::NPANEL; ++pn)
             load_rows<VARLEN>(smem + L::Q_OFF + w * L::TILE + pn * PANEL_BYTES, &tm_q, q_full,
-                              pn * XSTEP, g.q0 + g.tile * BLOCK_M + w * TILE_M, g.head);
+                              pn * XSTEP, g.q0 + g.qrow(w), g.hd(w));
         ++n_items;
         for (int j = 0; j < n_kv1 && ok; ++j, ++kv) {
           // K_kv is ring tile 2 kv, V_kv is ring tile 2 kv + 1
@@ -657,8 +684,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         tc_fence_after();
         const float inv_l = inv_l_buf[((k & 1) * NQ + w) * TILE_M + row];
         const uint32_t tO = tmem_base + 256 + w * 128 + lane_off;
-        const int row_g = g.tile * BLOCK_M + w * TILE_M + row;  // within the sequence
-        const size_t orow_off = static_cast<size_t>(g.head) * p.o_head +
+        const int row_g = g.qrow(w) + row;  // within the sequence
+        const size_t orow_off = static_cast<size_t>(g.hd(w)) * p.o_head +
                                 static_cast<size_t>(g.q0 + row_g) * p.o_row;
         const bool valid = row_g < g.Nq && dbg_ok(orow_off + D <= p.o_elems);
         __nv_bfloat16* orow_g = p.o + orow_off;
@@ -702,7 +729,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       const int item = cta_item(cta, k, G);
       if (item >= p.total_items) break;
       const ItemGeo g = item_geo<VARLEN>(p, item);
-      const int q_row0 = g.tile * BLOCK_M + w * TILE_M;  // within the sequence
+      const int q_row0 = g.qrow(w);  // within the sequence
       const int row_g = q_row0 + row;
       const int n_kv = n_kv_of(g, w);
       float m = -INFINITY;  // running max of scale * log2(e) * s
@@ -855,10 +882,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       inv_l_buf[((k & 1) * NQ + w) * TILE_M + row] = (l > 0.f) ? p.o_scale / l : 0.f;
       mbar_arrive(&l_ready[2 * w + (k & 1)]);
       if (row_g < g.Nq && p.lse != nullptr &&
-          dbg_ok(static_cast<size_t>(g.head) * p.lse_head + g.q0 + row_g < p.lse_elems)) {
+          dbg_ok(static_cast<size_t>(g.hd(w)) * p.lse_head + g.q0 + row_g < p.lse_elems)) {
         // LSE = ln(sum exp(scale * s)) = (m + log2 l) * ln 2, m in log2 units.
         const float lse = (l > 0.f) ? (m + lg2_approx(l)) * 0.6931471805599453f : -INFINITY;
-        p.lse[static_cast<size_t>(g.head) * p.lse_head + g.q0 + row_g] = lse;
+        p.lse[static_cast<size_t>(g.hd(w)) * p.lse_head + g.q0 + row_g] = lse;
       }
     }
     tmem_ld_wait();
@@ -923,8 +950,16 @@ fa_status launch_fwd(const void* q, const void* k, const void* v, void* o, float
         static_cast<__nv_bfloat16*>(o), lse, static_cast<size_t>(BH) * Nq, d);
     return cuda_status(cudaGetLastError());
   }
-  const long long n_cta_tiles = (Nq + fwd::BLOCK_M - 1) / fwd::BLOCK_M;
-  const long long items = static_cast<long long>(BH) * n_cta_tiles;
+  // Grouped heads with an even group: a work item is one 128-row tile of two
+  // query heads that share a key/value head, so both of its query tiles see
+  // the same keys (no step in which one tile waits while the other finishes
+  // its diagonal key tile) and still share every K/V tile.  Otherwise two
+  // consecutive 128-row tiles of one head.
+  const bool pair = (H / Hkv) % 2 == 0;
+  const int item_rows = pair ? fwd::TILE_M : fwd::BLOCK_M;
+  const long long n_cta_tiles = (Nq + item_rows - 1) / item_rows;
+  const long long item_bh = pair ? BH / 2 : BH;
+  const long long items = item_bh * n_cta_tiles;
   if (items > 0x7fffffffLL) return FA_ERR_INVALID_ARG;
   CUtensorMap tq, tk, tv;
   fa_status st;
@@ -951,7 +986,8 @@ fa_status launch_fwd(const void* q, const void* k, const void* v, void* o, float
   prm.Nq = Nq;
   prm.Nk = Nk;
   prm.causal_off = Nk - Nq;
-  prm.BH = BH;
+  prm.BH = static_cast<int>(item_bh);
+  prm.pair_heads = pair ? 1 : 0;
   prm.group = H / Hkv;
   prm.n_cta_tiles = static_cast<int>(n_cta_tiles);
   prm.total_items = static_cast<int>(items);
@@ -1005,6 +1041,7 @@ fa_status launch_fwd_varlen(const void* q, const void* k, const void* v, void* o
   prm.Nk = 0;
   prm.causal_off = 0;
   prm.BH = B * H;
+  prm.pair_heads = 0;
   prm.group = H / Hkv;
   prm.n_cta_tiles = static_cast<int>(n_cta_tiles);
   prm.total_items = static_cast<int>(items);
@@ -1076,6 +1113,7 @@ fa_status launch_fwd_fp8(const void* q, const void* k, const void* vt, void* o, 
   prm.Nk = Nk;
   prm.causal_off = Nk - Nq;
   prm.BH = BH;
+  prm.pair_heads = 0;
   prm.group = H / Hkv;
   prm.n_cta_tiles = static_cast<int>(n_cta_tiles);
   prm.total_items = static_cast<int>(items);
