@@ -278,6 +278,9 @@ struct Params {
   // key/value head (grouped heads, an even group); item coordinates then count
   // head pairs and 128-row tiles.  0: two consecutive 128-row tiles of one head.
   int pair_heads;
+  // with paired heads and no grouping: the two heads have their own K / V, and
+  // the ring carries each tile's keys and values separately
+  int kv_split;
   float scale_log2;  // scale * log2(e) (times the q and k descales for e4m3)
   float o_scale;     // multiplies O / l: 1, or the v descale for e4m3
   // ragged batch (token-major packing): sequence b owns rows cu_q[b] ..
@@ -317,7 +320,8 @@ struct ItemGeo {
   int qrow0, qstep, hd0, hstep;
   __device__ __forceinline__ int qrow(int w) const { return qrow0 + w * qstep; }
   __device__ __forceinline__ int hd(int w) const { return hd0 + w * hstep; }
-  int kv_head;     // head coordinate of K / V
+  int kv_head;     // head coordinate of K / V of query tile 0
+  int kv_hstep;    // ... of query tile w: kv_head + w * kv_hstep
   int q0, k0;
   int Nq, Nk, off; // lengths of the sequence and Nk - Nq
   int n_kv_total;  // key tiles of the sequence, at least 1
@@ -340,12 +344,14 @@ __device__ __forceinline__ ItemGeo item_geo(const Params& p, int item) {
       g.qrow0 = g.tile * TILE_M;
       g.qstep = 0;
       g.kv_head = h0 / p.group;
+      g.kv_hstep = p.kv_split;  // own K / V (no grouping), or the shared head
     } else {
       g.hd0 = bh;
       g.hstep = 0;
       g.qrow0 = g.tile * BLOCK_M;
       g.qstep = TILE_M;
       g.kv_head = bh / p.group;
+      g.kv_hstep = 0;
     }
     g.q0 = 0;
     g.k0 = 0;
@@ -359,6 +365,7 @@ __device__ __forceinline__ ItemGeo item_geo(const Params& p, int item) {
     g.qrow0 = g.tile * BLOCK_M;
     g.qstep = TILE_M;
     g.kv_head = h / p.group;
+    g.kv_hstep = 0;
     g.q0 = p.cu_q[b];
     g.k0 = p.cu_k[b];
     g.Nq = p.cu_q[b + 1] - g.q0;
@@ -502,27 +509,39 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             load_rows<VARLEN>(smem + L::Q_OFF + w * L::TILE + pn * PANEL_BYTES, &tm_q, q_full,
                               pn * XSTEP, g.q0 + g.qrow(w), g.hd(w));
         ++n_items;
-        for (int j = 0; j < n_kv1 && ok; ++j, ++kv) {
-          // K_kv is ring tile 2 kv, V_kv is ring tile 2 kv + 1
-          for (int half = 0; half < 2; ++half) {
-            const int u = 2 * kv + half;
-            const int slot = u % NSLOT;
-            if (u >= NSLOT && !mbar_wait(&empty[slot], (u / NSLOT - 1) & 1, abort_flag)) {
-              ok = false;
-              break;
-            }
-            mbar_arrive_expect_tx(&full[slot], L::TILE);
-            if (F8 && half) {
-              // V_j^T: rows d, columns keys j*128 ..
-              tma_load_3d(smem + L::RING_OFF + slot * L::TILE, &tm_v, &full[slot], j * BLOCK_N, 0,
-                          g.kv_head);
-            } else {
-              for (int pn = 0; pn < L::NPANEL; ++pn)
-                load_rows<VARLEN>(smem + L::RING_OFF + slot * L::TILE + pn * PANEL_BYTES,
-                                  half ? &tm_v : &tm_k, &full[slot], pn * XSTEP,
-                                  g.k0 + j * BLOCK_N, g.kv_head);
-            }
-            ++loaded;
+        // one ring tile: K or V, key tile j, of key/value head kvh
+        auto ring = [&](bool is_v, int j, int kvh) -> bool {
+          const int u = loaded;
+          const int slot = u % NSLOT;
+          if (u >= NSLOT && !mbar_wait(&empty[slot], (u / NSLOT - 1) & 1, abort_flag))
+            return false;
+          mbar_arrive_expect_tx(&full[slot], L::TILE);
+          if (F8 && is_v) {
+            // V_j^T: rows d, columns keys j*128 ..
+            tma_load_3d(smem + L::RING_OFF + slot * L::TILE, &tm_v, &full[slot], j * BLOCK_N, 0,
+                        kvh);
+          } else {
+            for (int pn = 0; pn < L::NPANEL; ++pn)
+              load_rows<VARLEN>(smem + L::RING_OFF + slot * L::TILE + pn * PANEL_BYTES,
+                                is_v ? &tm_v : &tm_k, &full[slot], pn * XSTEP,
+                                g.k0 + j * BLOCK_N, kvh);
+          }
+          ++loaded;
+          return true;
+        };
+        if (!p.kv_split) {
+          // both tiles read K_j and V_j: ring tiles K_0 V_0 K_1 V_1 ...
+          for (int j = 0; j < n_kv1 && ok; ++j, ++kv)
+            ok = ring(false, j, g.kv_head) && ring(true, j, g.kv_head);
+        } else {
+          // each tile has its own K / V, in the order the MMA warp takes them:
+          // K0_0 K1_0 | V0_j K0_{j+1} V1_j K1_{j+1} | ...  (n0 = n1)
+          const int kv0 = g.kv_head, kv1 = g.kv_head + g.kv_hstep;
+          ok = ring(false, 0, kv0) && ring(false, 0, kv1);
+          for (int j = 0; j < n_kv1 && ok; ++j) {
+            const bool more = j + 1 < n_kv1;
+            ok = ring(true, j, kv0) && (!more || ring(false, j + 1, kv0)) && ring(true, j, kv1) &&
+                 (!more || ring(false, j + 1, kv1));
           }
         }
       }
@@ -619,7 +638,54 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       auto kwait = [&](int g) { return mwait(&full[kslot(g)], ((2 * g) / NSLOT) & 1); };
       auto vwait = [&](int g) { return mwait(&full[vslot(g)], ((2 * g + 1) / NSLOT) & 1); };
       bool ok = true;
-      for (int k = 0; ok; ++k) {
+      if (p.kv_split) {
+        // Paired heads with their own K / V: every ring tile is used by one
+        // product and released right after it, in the order they are taken.
+        int racq = 0;
+        auto acq = [&](int& slot) {
+          slot = racq % NSLOT;
+          const bool r = mwait(&full[slot], (racq / NSLOT) & 1);
+          ++racq;
+          return r;
+        };
+        for (int k = 0; ok; ++k) {
+          const int item = cta_item(cta, k, G);
+          if (item >= p.total_items) break;
+          const ItemGeo g = item_geo<VARLEN>(p, item);
+          const int n = n_kv_of(g, 1);  // both tiles: the same rows
+          int sl = 0;
+          if (!mwait(q_full, k & 1)) { ok = false; break; }
+          for (int w = 0; w < NQ && ok; ++w) {
+            if (!acq(sl)) { ok = false; break; }
+            tc_fence_after();
+            issue_s(w, sl);
+            commit(&empty[sl]);
+          }
+          if (!ok) break;
+          if (n == 1) commit(q_empty);
+          for (int j = 0; j < n && ok; ++j) {
+            const bool more = j + 1 < n;
+            for (int w = 0; w < NQ; ++w) {
+              // the first product of an item overwrites O_w: its read-out by
+              // the previous item's epilogue must be complete
+              if (!acq(sl) || (j == 0 && k > 0 && !mwait(&o_free[w], (k - 1) & 1)) ||
+                  !issue_pv(w, sl, j == 0, j == n - 1)) {
+                ok = false;
+                break;
+              }
+              commit(&empty[sl]);
+              if (more) {
+                if (!acq(sl)) { ok = false; break; }
+                tc_fence_after();
+                issue_s(w, sl);
+                commit(&empty[sl]);
+              }
+            }
+            if (ok && j + 2 == n) commit(q_empty);  // last S of this item issued
+          }
+        }
+      }
+      for (int k = 0; ok && !p.kv_split; ++k) {
         const int item = cta_item(cta, k, G);
         if (item >= p.total_items) break;
         const ItemGeo g = item_geo<VARLEN>(p, item);
@@ -955,7 +1021,13 @@ fa_status launch_fwd(const void* q, const void* k, const void* v, void* o, float
   // the same keys (no step in which one tile waits while the other finishes
   // its diagonal key tile) and still share every K/V tile.  Otherwise two
   // consecutive 128-row tiles of one head.
-  const bool pair = (H / Hkv) % 2 == 0;
+  // Without grouping, persistent causal problems pair heads too: the two
+  // heads then read their own K / V (about twice the tile loads, all from L2),
+  // which pays for itself where items are short.
+  const int group = H / Hkv;
+  const double kv_bytes = 4.0 * B * Hkv * static_cast<double>(Nk) * d;
+  const bool small_kv = kv_bytes <= 96.0 * 1024 * 1024;
+  const bool pair = group % 2 == 0 || (group == 1 && H % 2 == 0 && causal && small_kv);
   const int item_rows = pair ? fwd::TILE_M : fwd::BLOCK_M;
   const long long n_cta_tiles = (Nq + item_rows - 1) / item_rows;
   const long long item_bh = pair ? BH / 2 : BH;
@@ -969,9 +1041,8 @@ fa_status launch_fwd(const void* q, const void* k, const void* v, void* o, float
   const uint64_t BHkv = static_cast<uint64_t>(B) * Hkv;
   if ((st = make_tmap_bf16_3d(&tk, k, d, Nk, BHkv, fwd::BLOCK_N)) != FA_OK) return st;
   if ((st = make_tmap_bf16_3d(&tv, v, d, Nk, BHkv, fwd::BLOCK_N)) != FA_OK) return st;
-  const double kv_bytes = 4.0 * B * Hkv * static_cast<double>(Nk) * d;
   const int mode = fwd::schedule_mode();
-  bool persistent = causal && items > sms && kv_bytes <= 96.0 * 1024 * 1024;
+  bool persistent = causal && items > sms && small_kv;
   int grid = persistent ? sms : static_cast<int>(items);
   if (mode == FA_SCHEDULE_GRID) {
     persistent = false;
@@ -988,6 +1059,7 @@ fa_status launch_fwd(const void* q, const void* k, const void* v, void* o, float
   prm.causal_off = Nk - Nq;
   prm.BH = static_cast<int>(item_bh);
   prm.pair_heads = pair ? 1 : 0;
+  prm.kv_split = (pair && group == 1) ? 1 : 0;
   prm.group = H / Hkv;
   prm.n_cta_tiles = static_cast<int>(n_cta_tiles);
   prm.total_items = static_cast<int>(items);
@@ -1042,6 +1114,7 @@ fa_status launch_fwd_varlen(const void* q, const void* k, const void* v, void* o
   prm.causal_off = 0;
   prm.BH = B * H;
   prm.pair_heads = 0;
+  prm.kv_split = 0;
   prm.group = H / Hkv;
   prm.n_cta_tiles = static_cast<int>(n_cta_tiles);
   prm.total_items = static_cast<int>(items);
@@ -1114,6 +1187,7 @@ fa_status launch_fwd_fp8(const void* q, const void* k, const void* vt, void* o, 
   prm.causal_off = Nk - Nq;
   prm.BH = BH;
   prm.pair_heads = 0;
+  prm.kv_split = 0;
   prm.group = H / Hkv;
   prm.n_cta_tiles = static_cast<int>(n_cta_tiles);
   prm.total_items = static_cast<int>(items);
