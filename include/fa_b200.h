@@ -159,8 +159,9 @@ fa_status fa_fwd_fp8(const void* q, const void* k, const void* vt, void* o, floa
 /*
  * Bytes of device workspace fa_bwd needs: D = rowsum(dO * O) and
  * log2(e) * LSE as float32 [B, H, Np] with Np = N rounded up to a multiple
- * of 128, followed by the float32 dQ accumulator [B, H, N, d], each region
- * 256-byte aligned.  Returns 0 for invalid sizes.
+ * of 128, the float32 dQ accumulator [B, H, N, d] and one uint32
+ * completion counter per (b, h), each region 256-byte aligned.  Returns 0
+ * for invalid sizes.
  */
 size_t fa_bwd_workspace_size(int B, int H, int N, int d);
 

@@ -269,9 +269,11 @@ size_t fa_bwd_workspace_size(int B, int H, int N, int d) {
   if (check_shape(B, H, N, d) != FA_OK) return 0;
   const size_t bh = static_cast<size_t>(B) * H;
   const size_t padded = bh * bwd_row_pad(N);
-  // D and log2(e) * LSE on 128-padded rows, then the fp32 dQ accumulator
+  // D and log2(e) * LSE on 128-padded rows, the fp32 dQ accumulator, then
+  // one completion counter per (batch, head)
   return 2 * align_up(padded * sizeof(float), 256) +
-         align_up(bh * static_cast<size_t>(N) * d * sizeof(float), 256);
+         align_up(bh * static_cast<size_t>(N) * d * sizeof(float), 256) +
+         align_up(bh * sizeof(unsigned), 256);
 }
 
 fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, const void* dout,

@@ -7,8 +7,10 @@
 //   P = exp(S - LSE),  dV = P^T dO,  dP = dO V^T,  D = rowsum(dO * O),
 //   dS = P * (dP - D),  dQ = scale dS K,  dK = scale dS^T Q.
 //
-// Three kernels:
-//   fa_bwd_preprocess  D = rowsum(dO * O) (fp32) and a zeroed fp32 dQ accumulator.
+// Three kernels; the second and third are launched with programmatic stream
+// serialisation (each may start before the kernel before it has ended):
+//   fa_bwd_preprocess  D = rowsum(dO * O) (fp32), a zeroed fp32 dQ accumulator
+//                      and zeroed completion counters, one per key/value head.
 //   fa_bwd_kernel      one CTA per 128-key tile j of one (batch, head); it keeps
 //                      dK_j and dV_j in tensor memory and loops over the query
 //                      tiles i that can see key tile j (causal: those holding a
@@ -18,7 +20,17 @@
 //                        dV += P^T dO_i, dK += dS^T Q_i            (A from TMEM)
 //                        dQ_i = dS K_j  (A = dS from shared memory), added to
 //                        an fp32 accumulator with bulk tensor reductions.
-//   fa_bwd_dq_convert  dQ = scale * accumulator, rounded to bf16.
+//                      Its set-up and K_j / V_j loads overlap the end of the
+//                      preprocess; every thread waits for the preprocess
+//                      (griddepcontrol.wait) before the first table load.
+//                      When its last reduction has completed, a CTA adds one
+//                      to its key/value head's completion counter.
+//   fa_bwd_dq_convert  dQ = scale * accumulator, rounded to bf16.  A CTA of
+//                      it converts rows of one query head once the counter of
+//                      that head's key/value head reaches the number of key
+//                      tiles, so the heads finished first (the grid of the
+//                      main kernel runs head by head) are converted on SMs
+//                      that the main kernel's last CTAs leave idle.
 //
 // Warp roles of fa_bwd_kernel (448 threads):
 //   warps 0-7  two P^T / dS^T warpgroups: thread t of warpgroup g owns key row t
@@ -104,6 +116,9 @@ struct Params {
   // element strides of dK / dV: [head][row] at head * kv_head + row * kv_row
   size_t kv_head, kv_row;
   size_t kv_elems;   // elements of dK (= of dV), for the debug build's checks
+  // completion counter per key/value head (padded layout), zeroed by the
+  // preprocess; nullptr: the conversion waits for the whole kernel instead
+  unsigned* done_cnt;
 };
 
 // First row of sequence b in the ragged LSE / D tables: a multiple of 4 (a
@@ -262,6 +277,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  // The next grid (the dQ conversion) may be scheduled once every thread of
+  // every CTA has got here, i.e. after the preprocess has completed: its
+  // counters are zero by then.
+  if (warp != 12) {
+    griddep_wait();
+    griddep_launch_dependents();
+  }
   const uint32_t tmem_base = *tmem_slot;
   const uint32_t tSt = tmem_base;
   const uint32_t tdPt = tmem_base + 128;
@@ -273,7 +295,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     if (lane == 0) {
       tma_prefetch_desc(&tm_q);
       tma_prefetch_desc(&tm_do);
-      int last_q[2] = {-1, -1}, last_do[2] = {-1, -1};
       mbar_arrive_expect_tx(kv_full, 2 * L::TILE);
       for (int pn = 0; pn < L::NPANEL; ++pn) {
         load_rows<VARLEN>(smem + L::K_OFF + pn * PANEL_BYTES, &tm_k, kv_full, pn * 64,
@@ -281,6 +302,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         load_rows<VARLEN>(smem + L::V_OFF + pn * PANEL_BYTES, &tm_v, kv_full, pn * 64,
                           geo.k0 + key0, geo.kv_head);
       }
+    }
+    // the LSE / D tables come from the preprocess
+    griddep_wait();
+    griddep_launch_dependents();
+    if (lane == 0) {
+      int last_q[2] = {-1, -1}, last_do[2] = {-1, -1};
       for (int it = 0; it < n_it; ++it) {
         const int st = it & 1;
         const int r = it >> 1;
@@ -571,7 +598,15 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         mbar_arrive(&do_empty[st]);  // dO_i's stage may be reloaded
       }
     }
-    if (t == 0) bulk_wait_group0();
+    if (t == 0) {
+      bulk_wait_group0();
+      if (!VARLEN && p.done_cnt != nullptr) {
+        // this CTA's reductions have completed: publish them
+        fence_proxy_async_global();
+        __threadfence();
+        atomicAdd(p.done_cnt + geo.kv_head, 1u);
+      }
+    }
     tmem_ld_wait();
   }
 
@@ -585,16 +620,24 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 }
 
 // For every padded row (bh, n), n < Np: D = sum_k dO_k O_k and
-// lse2 = log2(e) * LSE when n < N, else D = 0 and lse2 = +inf; and dQacc = 0.
-// A row whose LSE is -inf saw no key; its lse2 is +inf as well, so that every
-// P of it is exactly 0.
+// lse2 = log2(e) * LSE when n < N, else D = 0 and lse2 = +inf; dQacc = 0;
+// and the n_cnt completion counters = 0.  A row whose LSE is -inf saw no
+// key; its lse2 is +inf as well, so that every P of it is exactly 0.
 template <int D>
 __global__ void __launch_bounds__(256)
     fa_bwd_preprocess_kernel(const __nv_bfloat16* __restrict__ o,
                              const __nv_bfloat16* __restrict__ dout,
                              const float* __restrict__ lse, float* __restrict__ dd,
-                             float* __restrict__ lse2, float* __restrict__ dqacc, int N, int Np,
+                             float* __restrict__ lse2, float* __restrict__ dqacc,
+                             unsigned* __restrict__ cnt, int n_cnt, int N, int Np,
                              long long padded_rows) {
+  // the main kernel may start its set-up now; it waits for this grid's
+  // completion before it reads anything written here
+  griddep_launch_dependents();
+  {
+    const long long gi = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
+    if (gi < n_cnt) cnt[gi] = 0u;
+  }
   constexpr int LPR = D / 8;     // lanes per row, 16 bytes each
   constexpr int RPW = 32 / LPR;  // rows per warp
   const int lane = threadIdx.x & 31;
@@ -638,6 +681,7 @@ __global__ void __launch_bounds__(256)
                                     const float* __restrict__ lse, float* __restrict__ dd,
                                     float* __restrict__ lse2, const int* __restrict__ cu_q, int B,
                                     int H, int total_q, long long P) {
+  griddep_launch_dependents();
   constexpr int LPR = D / 8;     // lanes per row, 16 bytes each
   constexpr int RPW = 32 / LPR;  // rows per warp
   const int lane = threadIdx.x & 31;
@@ -680,14 +724,45 @@ __global__ void __launch_bounds__(256)
   }
 }
 
-// dQ = scale * dQacc in bf16, 8 elements per thread.
+// Bounded wait until *c >= need (acquire); false at once if the device error
+// word is set (a CTA of the main kernel gave up, so the count may never be
+// reached), and after the time limit, with FA_ERR_TIMEOUT recorded.
+__device__ __forceinline__ bool wait_counter(const unsigned* c, unsigned need) {
+  const uint64_t t0 = globaltimer_ns();
+  for (;;) {
+    unsigned v;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(c) : "memory");
+    if (v >= need) return true;
+    if (*static_cast<volatile int*>(&g_device_error) != 0) return false;
+    if (globaltimer_ns() - t0 > FA_WAIT_TIMEOUT_NS) {
+      record_error(5 /* FA_ERR_TIMEOUT */);
+      return false;
+    }
+    __nanosleep(256);
+  }
+}
+
+// dQ = scale * dQacc in bf16, 8 elements per thread.  Without counters the
+// grid covers all n8 groups of 8 elements.  With counters (done_cnt set) the
+// grid is (groups of one head / 256, B * H): a CTA converts part of query
+// head blockIdx.y once the counter of its key/value head, blockIdx.y /
+// group, has reached `need` (every CTA of the main kernel for that head has
+// finished adding into the accumulator).
 __global__ void __launch_bounds__(256)
     fa_bwd_dq_convert_kernel(const float* __restrict__ dqacc, __nv_bfloat16* __restrict__ dq,
-                             long long n8, float scale) {
-  const long long i = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
+                             long long n8, float scale, const unsigned* __restrict__ done_cnt,
+                             unsigned need, int group, long long head8) {
+  long long i = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (done_cnt != nullptr) {
+    __shared__ int ready;
+    if (threadIdx.x == 0) ready = wait_counter(done_cnt + blockIdx.y / group, need) ? 1 : 0;
+    __syncthreads();
+    if (!ready || i >= head8) return;
+    i += static_cast<long long>(blockIdx.y) * head8;
+  }
   if (i >= n8) return;
-  const float4 a = reinterpret_cast<const float4*>(dqacc)[2 * i];
-  const float4 b = reinterpret_cast<const float4*>(dqacc)[2 * i + 1];
+  const float4 a = __ldcg(reinterpret_cast<const float4*>(dqacc) + 2 * i);
+  const float4 b = __ldcg(reinterpret_cast<const float4*>(dqacc) + 2 * i + 1);
   reinterpret_cast<uint4*>(dq)[i] =
       make_uint4(pack_bf16x2(a.x * scale, a.y * scale), pack_bf16x2(a.z * scale, a.w * scale),
                  pack_bf16x2(b.x * scale, b.y * scale), pack_bf16x2(b.z * scale, b.w * scale));
@@ -698,11 +773,24 @@ fa_status launch_main(const CUtensorMap* maps, const Params& prm, int BH, cudaSt
   auto kern = fa_bwd_kernel<D, CAUSAL, VARLEN>;
   static SmemOptIn opt_in;  // one per instantiation of this kernel
   if (const fa_status st = opt_in.ensure(kern, Smem<D>::ALLOC); st != FA_OK) return st;
-  dim3 grid(prm.n_kt * BH);
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(prm.n_kt * BH);
+  cfg.blockDim = dim3(NUM_THREADS);
+  cfg.dynamicSmemBytes = Smem<D>::ALLOC;
+  cfg.stream = stream;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
   main_kernel_begin(stream);
-  kern<<<grid, NUM_THREADS, Smem<D>::ALLOC, stream>>>(maps[0], maps[1], maps[2], maps[3], maps[4],
-                                                      maps[5], maps[6], prm);
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, kern, maps[0], maps[1], maps[2], maps[3], maps[4],
+                                           maps[5], maps[6], prm);
   main_kernel_end(stream);
+  if (e != cudaSuccess) {
+    (void)cudaGetLastError();
+    return FA_ERR_CUDA;
+  }
   return cuda_status(cudaGetLastError());
 }
 
@@ -734,18 +822,23 @@ fa_status launch_bwd(const void* q, const void* k, const void* v, const void* o,
   float* dd = static_cast<float*>(workspace);
   float* lse2 = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + table);
   float* dqacc = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + 2 * table);
-  // 1. D, log2(e) * LSE (padded tables) and the zeroed accumulator
+  unsigned* done_cnt = reinterpret_cast<unsigned*>(
+      static_cast<uint8_t*>(workspace) + 2 * table +
+      align_up(static_cast<size_t>(rows) * d * sizeof(float), 256));
+  // the conversion's grid has one row of CTAs per query head
+  const bool counted = BH <= 65535;
+  // 1. D, log2(e) * LSE (padded tables), the zeroed accumulator and counters
   {
     const int rows_per_block = (256 / 32) * (32 / (d / 8));
     const long long blocks = (prows + rows_per_block - 1) / rows_per_block;
     if (d == 128)
       bwd::fa_bwd_preprocess_kernel<128><<<static_cast<unsigned>(blocks), 256, 0, stream>>>(
           static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(dout), lse, dd,
-          lse2, dqacc, Nq, Np, prows);
+          lse2, dqacc, done_cnt, counted ? BHkv : 0, Nq, Np, prows);
     else
       bwd::fa_bwd_preprocess_kernel<64><<<static_cast<unsigned>(blocks), 256, 0, stream>>>(
           static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(dout), lse, dd,
-          lse2, dqacc, Nq, Np, prows);
+          lse2, dqacc, done_cnt, counted ? BHkv : 0, Nq, Np, prows);
     if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
   }
   // 2. dK, dV and the dQ accumulation
@@ -791,6 +884,7 @@ fa_status launch_bwd(const void* q, const void* k, const void* v, const void* o,
   prm.kv_head = static_cast<size_t>(Nk) * d;
   prm.kv_row = static_cast<size_t>(d);
   prm.kv_elems = static_cast<size_t>(BHkv) * Nk * d;
+  prm.done_cnt = counted ? done_cnt : nullptr;
   if (d == 128)
     st = causal ? bwd::launch_main<128, true, false>(maps, prm, BHkv, stream)
                 : bwd::launch_main<128, false, false>(maps, prm, BHkv, stream);
@@ -798,13 +892,38 @@ fa_status launch_bwd(const void* q, const void* k, const void* v, const void* o,
     st = causal ? bwd::launch_main<64, true, false>(maps, prm, BHkv, stream)
                 : bwd::launch_main<64, false, false>(maps, prm, BHkv, stream);
   if (st != FA_OK) return st;
-  // 3. dQ = scale * accumulator
+  // 3. dQ = scale * accumulator, head by head as the main kernel finishes
+  // them (programmatic launch: the grid may start before the main kernel
+  // ends; each CTA waits on its head's counter)
   {
     const long long n8 = rows * d / 8;
-    const long long blocks = (n8 + 255) / 256;
-    bwd::fa_bwd_dq_convert_kernel<<<static_cast<unsigned>(blocks), 256, 0, stream>>>(
-        dqacc, static_cast<__nv_bfloat16*>(dq), n8, scale);
-    if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
+    const long long head8 = static_cast<long long>(Nq) * d / 8;
+    const float* acc = dqacc;
+    __nv_bfloat16* out = static_cast<__nv_bfloat16*>(dq);
+    cudaError_t e;
+    if (counted) {
+      cudaLaunchAttribute attr[1];
+      attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+      attr[0].val.programmaticStreamSerializationAllowed = 1;
+      cudaLaunchConfig_t cfg = {};
+      cfg.gridDim = dim3(static_cast<unsigned>((head8 + 255) / 256), static_cast<unsigned>(BH));
+      cfg.blockDim = dim3(256);
+      cfg.stream = stream;
+      cfg.attrs = attr;
+      cfg.numAttrs = 1;
+      e = cudaLaunchKernelEx(&cfg, bwd::fa_bwd_dq_convert_kernel, acc, out, n8, scale,
+                             static_cast<const unsigned*>(done_cnt),
+                             static_cast<unsigned>(prm.n_kt), H / Hkv, head8);
+    } else {
+      const long long blocks = (n8 + 255) / 256;
+      bwd::fa_bwd_dq_convert_kernel<<<static_cast<unsigned>(blocks), 256, 0, stream>>>(
+          acc, out, n8, scale, nullptr, 0u, 1, 0LL);
+      e = cudaGetLastError();
+    }
+    if (e != cudaSuccess) {
+      (void)cudaGetLastError();
+      return FA_ERR_CUDA;
+    }
   }
   return FA_OK;
 }
@@ -888,6 +1007,7 @@ fa_status launch_bwd_varlen(const void* q, const void* k, const void* v, const v
   prm.kv_head = static_cast<size_t>(d);
   prm.kv_row = static_cast<size_t>(Hkv) * d;
   prm.kv_elems = static_cast<size_t>(total_k) * Hkv * d;
+  prm.done_cnt = nullptr;
   if (static_cast<long long>(prm.n_kt) * prm.BHkv > 0x7fffffffLL) return FA_ERR_INVALID_ARG;
   if (d == 128)
     st = causal ? bwd::launch_main<128, true, true>(maps, prm, prm.BHkv, stream)
@@ -901,7 +1021,7 @@ fa_status launch_bwd_varlen(const void* q, const void* k, const void* v, const v
     const long long n8 = static_cast<long long>(dq_elems / 8);
     const long long blocks = (n8 + 255) / 256;
     bwd::fa_bwd_dq_convert_kernel<<<static_cast<unsigned>(blocks), 256, 0, stream>>>(
-        dqacc, static_cast<__nv_bfloat16*>(dq), n8, scale);
+        dqacc, static_cast<__nv_bfloat16*>(dq), n8, scale, nullptr, 0u, 1, 0LL);
     if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
   }
   return FA_OK;
