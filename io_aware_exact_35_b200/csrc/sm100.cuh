@@ -179,24 +179,6 @@ __device__ __forceinline__ void named_barrier(int id, int count) {
 __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
-// Orders this thread's completed bulk (async-proxy) writes to global memory
-// before its later generic accesses, e.g. a release that publishes them.
-__device__ __forceinline__ void fence_proxy_async_global() {
-  asm volatile("fence.proxy.async.global;" ::: "memory");
-}
-
-// ------------------------------------------------------------------ programmatic dependent launch
-// In a kernel launched with programmatic stream serialisation: wait until the
-// preceding grid has completed and its writes are visible (a no-op when the
-// launch had no such dependency).
-__device__ __forceinline__ void griddep_wait() {
-  asm volatile("griddepcontrol.wait;" ::: "memory");
-}
-// Allow the next grid in the stream, if launched with programmatic stream
-// serialisation, to start before this one has finished.
-__device__ __forceinline__ void griddep_launch_dependents() {
-  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-}
 
 // ------------------------------------------------------------------ tcgen05
 __device__ __forceinline__ void tmem_alloc(uint32_t* smem_slot, uint32_t ncols) {
