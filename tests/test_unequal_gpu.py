@@ -122,3 +122,31 @@ def test_bwd_empty_sides(fa_mod, cuda_device):
     q, k, v, do = inputs.bwd_inputs(B, H, 90, d, seed=4101, Nk=0)
     dq, dk, dv = _fwd_bwd(fa_mod, q, k, v, do, False, 0.125)
     assert torch.all(dq == 0) and dk.shape == (B, H, 0, d)
+
+
+@pytest.mark.parametrize("case", [(2, 4, 2, 300, 700, 128, True), (1, 2, 1, 520, 260, 64, True),
+                                  (2, 2, 2, 640, 640, 128, False)],
+                         ids=lambda c: "B%dH%dHkv%dNq%dNk%dd%dc%d" % c)
+def test_bwd_workspace_contents_ignored(fa_mod, cuda_device, case):
+    """The backward's workspace holds the dQ accumulator and one completion
+    counter per key/value head, which the dQ conversion waits on; both are
+    reset by every call.  A workspace filled with 0xFF (every counter already
+    past its target) and then reused by a second call must give the oracle's
+    gradients both times."""
+    B, H, Hkv, Nq, Nk, d, causal = case
+    q, k, v, do = inputs.bwd_inputs(B, H, Nq, d, seed=4200 + Nq + Nk, Hkv=Hkv, Nk=Nk)
+    scale = 1.0 / np.sqrt(d)
+    rq, rk, rv, _ = oracle.attention_backward(*(inputs.to_f64(t) for t in (q, k, v, do)),
+                                              causal, scale)
+    qd, kd, vd, dod = (t.to(DEV) for t in (q, k, v, do))
+    o, lse = fa_mod.fwd(qd, kd, vd, causal=causal, scale=scale)
+    ws = torch.full((fa_mod.bwd_workspace_size(B, H, Nq, d),), 0xFF, dtype=torch.uint8,
+                    device=DEV)
+    for call in range(2):
+        dq, dk, dv = fa_mod.bwd(qd, kd, vd, o, dod, lse, causal=causal, scale=scale,
+                                workspace=ws)
+        torch.cuda.synchronize()
+        assert fa_mod.get_device_error() == 0
+        check_grad(dq.cpu(), rq, f"dQ (call {call})")
+        check_grad(dk.cpu(), rk, f"dK (call {call})")
+        check_grad(dv.cpu(), rv, f"dV (call {call})")
