@@ -77,3 +77,19 @@ def test_bwd_both_cta_orders(fa_mod, cuda_device, order):
                     check_grad(dv[b, h], rv, f"dV[{b},{h}]")
     finally:
         fa_mod.set_schedule()
+
+
+def test_bwd_more_than_65535_heads(fa_mod, cuda_device):
+    """B * H above 65535: the dQ conversion's grid cannot give each query head
+    a row of CTAs, so it runs as a plain pass after the main kernel.  Sampled
+    heads on both sides of the 65535 boundary against the oracle."""
+    B, H, N, d = 1, 65600, 5, 64
+    q, k, v, do = inputs.bwd_inputs(B, H, N, d, seed=3400)
+    scale = 1.0 / np.sqrt(d)
+    dq, dk, dv = _run(fa_mod, q, k, v, do, True, scale)
+    for h in (0, 1, 777, 65534, 65535, 65536, 65599):
+        rq, rk, rv, _ = oracle.attention_backward(
+            *(inputs.to_f64(t[0, h]) for t in (q, k, v, do)), True, scale)
+        check_grad(dq[0, h], rq, f"dQ[{h}]")
+        check_grad(dk[0, h], rk, f"dK[{h}]")
+        check_grad(dv[0, h], rv, f"dV[{h}]")
