@@ -274,6 +274,7 @@ struct Params {
                      // the longest sequence (ragged batch)
   int total_items;   // BH * n_cta_tiles
   int lpt_order;     // 1: all heads' longest tiles first; 0: head-major
+  int head_band;     // head-major order: heads per band (>= 1)
   // 1: a work item is one 128-row tile of two query heads that share a
   // key/value head (grouped heads, an even group); item coordinates then count
   // head pairs and 128-row tiles.  0: two consecutive 128-row tiles of one head.
@@ -297,17 +298,26 @@ struct Params {
 };
 
 // Work item -> (batch*head (or head pair), query tile).  In LPT order the longest tiles of
-// every head come first (good balance; used when all K/V fit in L2); in
-// head-major order the tiles of one head are adjacent, longest first (K/V of
-// the resident CTAs stay in L2 for long sequences).
+// every head come first (good balance; used when all K/V fit in L2).  In
+// head-major order the heads go in bands of head_band adjacent heads, a
+// band's tiles longest first across its heads: the resident CTAs share a
+// band's K/V in L2 for long sequences, and the last CTAs to start are short
+// ones (with one head per band the last head's longest tile would start
+// near the end and run alone).
 __device__ __forceinline__ void item_coords(const Params& p, int item, int& bh, int& tile) {
   if (p.lpt_order) {
     const int r = item / p.BH;
     bh = item - r * p.BH;
     tile = p.n_cta_tiles - 1 - r;
   } else {
-    bh = item / p.n_cta_tiles;
-    tile = p.n_cta_tiles - 1 - (item - bh * p.n_cta_tiles);
+    const int per = p.head_band * p.n_cta_tiles;
+    const int band = item / per;
+    const int in_band = item - band * per;
+    const int h0 = band * p.head_band;
+    const int nb = min(p.head_band, p.BH - h0);
+    const int r = in_band / nb;
+    bh = h0 + (in_band - r * nb);
+    tile = p.n_cta_tiles - 1 - r;
   }
 }
 
@@ -987,6 +997,16 @@ fa_status launch(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap
 // one of the two.
 int schedule_mode() { return g_fwd_schedule.load(std::memory_order_relaxed); }
 
+// Heads per band of the head-major order: as many adjacent (query) heads as
+// keep their K and V within about 40 MB of L2 (a band and the next one's
+// first CTAs are resident together), at most 8.  kv_bytes: K and V of one
+// key/value head; share: query heads (or head pairs) reading it.
+int head_band(double kv_bytes, int share) {
+  const double per_head = kv_bytes / (share > 0 ? share : 1);
+  const double n = 40.0 * 1024 * 1024 / (per_head > 1.0 ? per_head : 1.0);
+  return n >= 8.0 ? 8 : (n < 1.0 ? 1 : static_cast<int>(n));
+}
+
 // Rows with no key at all (Nk = 0): O = 0, LSE = -inf, the same values the
 // main kernel gives a fully masked row.
 __global__ void fa_fwd_no_keys_kernel(__nv_bfloat16* o, float* lse, size_t rows, int d) {
@@ -1064,6 +1084,7 @@ fa_status launch_fwd(const void* q, const void* k, const void* v, void* o, float
   prm.n_cta_tiles = static_cast<int>(n_cta_tiles);
   prm.total_items = static_cast<int>(items);
   prm.lpt_order = persistent ? 1 : 0;
+  prm.head_band = fwd::head_band(4.0 * Nk * d, pair ? group / 2 : group);
   prm.scale_log2 = scale * 1.4426950408889634f;
   prm.o_scale = 1.f;
   prm.cu_q = nullptr;
@@ -1119,6 +1140,7 @@ fa_status launch_fwd_varlen(const void* q, const void* k, const void* v, void* o
   prm.n_cta_tiles = static_cast<int>(n_cta_tiles);
   prm.total_items = static_cast<int>(items);
   prm.lpt_order = 0;  // one CTA per tile, a head's tiles adjacent, longest first
+  prm.head_band = 1;  // a sequence's tiles adjacent
   prm.scale_log2 = scale * 1.4426950408889634f;
   prm.o_scale = 1.f;
   prm.cu_q = cu_q;
@@ -1192,6 +1214,7 @@ fa_status launch_fwd_fp8(const void* q, const void* k, const void* vt, void* o, 
   prm.n_cta_tiles = static_cast<int>(n_cta_tiles);
   prm.total_items = static_cast<int>(items);
   prm.lpt_order = persistent ? 1 : 0;
+  prm.head_band = fwd::head_band(2.0 * Nk * d, H / Hkv);  // e4m3: 1 byte per element
   // scores of the real (descaled) values: q_scale * k_scale * (Q8 K8^T)
   prm.scale_log2 = scale * q_scale * k_scale * 1.4426950408889634f;
   prm.o_scale = v_scale;
