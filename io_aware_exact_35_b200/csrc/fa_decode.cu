@@ -43,6 +43,17 @@ constexpr int WARPS = 4;
 constexpr int THREADS = WARPS * 32;
 constexpr int UNROLL = 8;
 
+// The split kernels let the combine kernel (launched after them with
+// programmatic stream serialisation) be scheduled once all their CTAs have
+// started; the combine kernel waits for their completion before it reads a
+// partial, so only its launch overlaps their tail.
+__device__ __forceinline__ void allow_combine_launch() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+__device__ __forceinline__ void wait_for_splits() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+
 __device__ __forceinline__ uint4 ld_stream(const void* p) {
   uint4 r;
   asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
@@ -154,6 +165,7 @@ __global__ void __launch_bounds__(THREADS)
   constexpr int LPK = D / 8;         // lanes per key
   constexpr int KPW = 32 / LPK;      // keys per warp step
   constexpr int HW = WARPS * KPW;    // key groups per CTA
+  allow_combine_launch();
   const int split = blockIdx.x;
   const int h = blockIdx.y;
   const int b = blockIdx.z;
@@ -325,6 +337,7 @@ __global__ void __launch_bounds__(THREADS)
   constexpr int MT = D / 16;         // m-tiles of O^T
   constexpr int NKL = D / 32;        // 16-byte loads per K row per lane
   constexpr int NVL = D / 64;        // 16-byte loads per V row per lane
+  allow_combine_launch();
   const int split = blockIdx.x;
   const int h0 = blockIdx.y * qh;    // first query head of this CTA
   const int b = blockIdx.z;
@@ -590,6 +603,7 @@ __global__ void __launch_bounds__(D)
     fa_decode_combine_kernel(const float* __restrict__ part, const int* __restrict__ seqlens,
                              __nv_bfloat16* __restrict__ o, float* __restrict__ lse, int H,
                              int Lmax, int S, int chunk) {
+  wait_for_splits();
   const int bh = blockIdx.x;
   const int b = bh / H;
   const int t = threadIdx.x;
@@ -694,9 +708,23 @@ fa_status launch(const void* q, const void* kc, const void* vc, const int* seqle
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return FA_ERR_CUDA;
   }
-  fa_decode_combine_kernel<D><<<B * H, D, 0, stream>>>(part, seqlens,
-                                                       static_cast<__nv_bfloat16*>(o), lse, H,
-                                                       Lmax, S > 0 ? S : 1, chunk);
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(B * H);
+  cfg.blockDim = dim3(D);
+  cfg.stream = stream;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  const float* cpart = part;
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, fa_decode_combine_kernel<D>, cpart, seqlens,
+                                           static_cast<__nv_bfloat16*>(o), lse, H, Lmax,
+                                           S > 0 ? S : 1, chunk);
+  if (e != cudaSuccess) {
+    (void)cudaGetLastError();
+    return FA_ERR_CUDA;
+  }
   return cuda_status(cudaGetLastError());
 }
 
