@@ -47,6 +47,12 @@ def test_workspace_sizes(fa_mod):
     rows = B * H * N
     assert ws >= rows * 4 + rows * d * 4
     assert ws % 256 == 0
+    # D and log2(e) LSE on 128-padded rows, the fp32 dQ accumulator and one
+    # uint32 completion counter per (batch, head), each 256-byte aligned
+    up = lambda x: (x + 255) // 256 * 256
+    padded = B * H * ((N + 127) // 128 * 128)
+    assert ws == 2 * up(padded * 4) + up(rows * d * 4) + up(B * H * 4)
+    assert fa_mod.bwd_workspace_size(1, 3, 1, 64) == 2 * up(3 * 128 * 4) + up(3 * 64 * 4) + up(12)
     assert fa_mod.bwd_workspace_size(0, 1, 1, 128) == 0
     assert fa_mod.bwd_workspace_size(1, 1, 1, 96) == 0
     wd = fa_mod.decode_workspace_size(16, 32, 16384, 128)
